@@ -1,0 +1,370 @@
+/*
+ * NVFP4 CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, obviously-correct restatement of what the NVFP4 hot path
+ * computes.  Only the test suite, the package's smoke check and the CPU
+ * baseline leg of the benchmark may load this library; the product path
+ * never does.  It shares no code, header or table with the CUDA kernels.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -msse2
+ *        -mfpmath=sse -fPIC -shared  (so every float operation below is one
+ *        IEEE binary32 operation rounded to nearest-even; no FMA contraction,
+ *        no flush-to-zero).
+ *
+ * Sources (web pages; section in parentheses):
+ *  [P1] "NVIDIA shrank GLM-5.2 to 4 bits" (iwan.kr), section 3 "Glossary --
+ *       quantization and NVFP4": 15 distinct 4-bit values, 16-value blocks
+ *       with one FP8 scale each, one FP32 scale per tensor.
+ *  [P2] "NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens"
+ *       (axbrief.com), section "E2M1 format and two-level scaling": E2M1 =
+ *       1 sign, 2 exponent, 1 mantissa bit with values +-0, 0.5, 1, 1.5, 2,
+ *       3, 4, 6; blocks of 16 with an E4M3 scale; FP32 tensor-level scale;
+ *       block amax mapped close to the FP4 maximum.
+ *  [P5] "FP4 KV-cache quantization" (theddari.com), section "FP4 formats
+ *       compared": 0.5625 bytes per value (4.5 bits) including scales.
+ *  The FP32 evaluation order below is the convention the hot path is
+ *  specified with: global g = 448*6/amax_tensor, block scale
+ *  s = e4m3_rne(amax_block/6*g), code = e2m1_rne(x*g/s), with x*g/s taken as
+ *  x*(g/s) (one division per block).  Every point the pages leave open is
+ *  marked READING below.
+ *
+ * Parity status: every function here is pinned by the oracle tests
+ * (exhaustive sweeps against brute-force nearest-value search, the pages'
+ * value list and storage figures, exact round trips, integer-exact GEMM).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+
+#define NVO_OK 0
+#define NVO_ERR_SHAPE 3
+#define NVO_ERR_NONFINITE 4
+#define NVO_ERR_RANGE 5
+
+#define NVO_SF_SWIZZLED 0
+#define NVO_SF_LINEAR 1
+
+/* ---------------------------------------------------------------- BF16 */
+
+float nvo_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round a binary32 to bfloat16, nearest-even on the 16 dropped bits. */
+uint16_t nvo_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu))
+        return (uint16_t)((u >> 16) | 0x0040u);          /* quiet NaN */
+    uint32_t low = u & 0xFFFFu;
+    uint32_t hi = u >> 16;
+    if (low > 0x8000u || (low == 0x8000u && (hi & 1u)))
+        hi += 1u;
+    return (uint16_t)hi;
+}
+
+/* ---------------------------------------------------------------- E2M1 */
+
+/* [P2] value list; code bits s.ee.m, bias 1, exponent field 0 = subnormal
+ * (m * 0.5).  Both 0x0 and 0x8 decode to zero: 16 codes, 15 values [P1]. */
+float nvo_e2m1_decode(uint8_t code)
+{
+    int e = (code >> 1) & 3, m = code & 1;
+    float mag = (e == 0) ? 0.5f * (float)m
+                         : ldexpf(1.0f + 0.5f * (float)m, e - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+/* Round y to the nearest E2M1 value, ties to the even code (mantissa bit
+ * 0), magnitudes at or above 6 saturate to 6 (E2M1 has no infinity).  The
+ * sign bit is copied from y, so -0 and tiny negatives give code 0x8
+ * (READING: the pages do not say which zero a negative underflow keeps). */
+uint8_t nvo_e2m1_rne_satfinite(float y)
+{
+    uint8_t sign = signbit(y) ? 8 : 0;
+    double a = fabs((double)y);
+    if (a >= 6.0)
+        return sign | 7;
+    int ex;
+    frexp(a, &ex);                 /* a = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                /* floor(log2 a) for a > 0 */
+    if (a == 0.0 || E < 0)
+        E = 0;                     /* [0, 2) shares the quantum 0.5 */
+    double q = ldexp(1.0, E - 1);  /* spacing of the grid in this binade */
+    double r = nearbyint(a / q) * q;  /* default mode: half to even */
+    if (r >= 6.0)
+        return sign | 7;
+    uint8_t code;
+    if (r < 1.0) {
+        code = (uint8_t)(r / 0.5);             /* 0 or 1 (subnormal) */
+    } else {
+        int e2;
+        frexp(r, &e2);
+        int E2 = e2 - 1;                       /* 0, 1 or 2 */
+        int m = (int)((r / ldexp(1.0, E2) - 1.0) * 2.0);
+        code = (uint8_t)(((E2 + 1) << 1) | m);
+    }
+    return sign | code;
+}
+
+/* ---------------------------------------------------------------- E4M3 */
+
+/* E4M3 (the block-scale format named in [P2]): bias 7, exponent field 0 is
+ * subnormal m/8 * 2^-6, S.1111.111 is NaN, largest finite 448. */
+float nvo_e4m3_decode(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    float mag;
+    if (e == 15 && m == 7)
+        mag = NAN;
+    else if (e == 0)
+        mag = ldexpf((float)m / 8.0f, -6);
+    else
+        mag = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return (b & 0x80) ? -mag : mag;
+}
+
+/* Round v >= 0 to the nearest finite E4M3 value, ties to even mantissa,
+ * subnormals kept, values past the largest finite (448) saturate to it. */
+uint8_t nvo_e4m3_rne_satfinite(float v)
+{
+    if (!(v > 0.0f))
+        return 0;                  /* +0, -0 (and NaN, never passed) */
+    if (v >= 448.0f)
+        return 0x7E;
+    int ex;
+    frexp((double)v, &ex);
+    int E = ex - 1;
+    if (E < -6)
+        E = -6;                    /* subnormals share binade -6's quantum */
+    double q = ldexp(1.0, E - 3);
+    double r = nearbyint((double)v / q) * q;
+    if (r == 0.0)
+        return 0;
+    if (r >= 448.0)
+        return 0x7E;
+    int e2;
+    frexp(r, &e2);
+    int E2 = e2 - 1;
+    if (E2 < -6)
+        return (uint8_t)(r / ldexp(1.0, -9));        /* subnormal m */
+    int m = (int)((r / ldexp(1.0, E2) - 1.0) * 8.0);
+    return (uint8_t)(((E2 + 7) << 3) | m);
+}
+
+/* ------------------------------------------------------- scale layouts */
+
+/* READING (pages silent): GEMM operands keep their block scales in the
+ * 128x4 tiled layout the block-scaled tensor-core MMA consumes -- per 128
+ * rows and 4 scale columns one 512-byte tile, row r%32 at 16-byte stride,
+ * (r%128)/32 at 4-byte stride, scale column c%4 at 1-byte stride; tiles run
+ * along the scale columns first.  Rows pad to 128 and scale columns to 4,
+ * padding holds zero.  The KV cache uses the plain row-major
+ * [rows x cols/16] layout. */
+int64_t nvo_sf_cols(int64_t cols) { return cols / 16; }
+
+int64_t nvo_scales_bytes(int64_t rows, int64_t cols, int layout)
+{
+    int64_t s = cols / 16;
+    if (layout == NVO_SF_LINEAR)
+        return rows * s;
+    int64_t sp = (s + 3) / 4 * 4;
+    int64_t rp = (rows + 127) / 128 * 128;
+    return rp * sp;
+}
+
+int64_t nvo_sf_offset(int64_t r, int64_t c, int64_t rows, int64_t cols, int layout)
+{
+    (void)rows;
+    int64_t s = cols / 16;
+    if (layout == NVO_SF_LINEAR)
+        return r * s + c;
+    int64_t sp = (s + 3) / 4 * 4;
+    return ((r / 128) * (sp / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+int64_t nvo_codes_bytes(int64_t rows, int64_t cols) { return rows * cols / 2; }
+
+/* ------------------------------------------------------------ quantize */
+
+/* Tensor amax: max |x| over all elements, exact (a max of BF16 values).
+ * Returns NVO_ERR_NONFINITE if any element is Inf or NaN. */
+int nvo_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, float *amax)
+{
+    float m = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float v = fabsf(nvo_bf16_to_f32(x[r * ld + c]));
+            if (!isfinite(v))
+                return NVO_ERR_NONFINITE;
+            if (v > m)
+                m = v;
+        }
+    *amax = m;
+    return NVO_OK;
+}
+
+/* Global (tensor) scale g = RN(448*6 / amax).  READINGS: amax == 0 gives
+ * g = 1 (all blocks then quantize to zero); g must stay at or below 2^118 so
+ * that every per-block factor g/s (s >= 2^-9) is finite -- smaller amax is
+ * reported as NVO_ERR_RANGE. */
+int nvo_global_scale(float amax, float *g)
+{
+    if (!isfinite(amax))
+        return NVO_ERR_NONFINITE;
+    if (amax == 0.0f) {
+        *g = 1.0f;
+        return NVO_OK;
+    }
+    float v = 2688.0f / amax;
+    *g = v;
+    if (!(v <= 0x1p118f))
+        return NVO_ERR_RANGE;
+    return NVO_OK;
+}
+
+/* Encode one row-major BF16 tensor with a given global scale g:
+ * per 16-block along the row, s = e4m3(RN(RN(amax_b/6)*g)),
+ * e = s ? RN(g/f32(s)) : 0, code = e2m1(RN(x*e)).  Codes pack two per byte,
+ * element 2i in the low nibble (READING: the pages give no nibble order;
+ * this is the order the FP4 tensor-core operand uses).  `scales` must hold
+ * nvo_scales_bytes() bytes; padding entries are written as zero. */
+void nvo_quantize_with_global(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                              float g, uint8_t *codes, uint8_t *scales, int layout)
+{
+    memset(scales, 0, (size_t)nvo_scales_bytes(rows, cols, layout));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            const uint16_t *xb = x + r * ld + b * 16;
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float v = fabsf(nvo_bf16_to_f32(xb[i]));
+                if (v > amax_b)
+                    amax_b = v;
+            }
+            float t = amax_b / 6.0f;
+            t = t * g;
+            uint8_t s = nvo_e4m3_rne_satfinite(t);
+            float sf = nvo_e4m3_decode(s);
+            float e = (s == 0) ? 0.0f : g / sf;
+            scales[nvo_sf_offset(r, b, rows, cols, layout)] = s;
+            uint8_t *cb = codes + r * (cols / 2) + b * 8;
+            for (int i = 0; i < 8; ++i) {
+                float y0 = nvo_bf16_to_f32(xb[2 * i]) * e;
+                float y1 = nvo_bf16_to_f32(xb[2 * i + 1]) * e;
+                uint8_t c0 = nvo_e2m1_rne_satfinite(y0);
+                uint8_t c1 = nvo_e2m1_rne_satfinite(y1);
+                cb[i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+}
+
+/* Full two-level quantize: amax -> g -> encode.  Returns a status; on error
+ * the outputs are unspecified.  *g_out receives the global scale. */
+int nvo_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                 uint8_t *codes, uint8_t *scales, int layout, float *g_out)
+{
+    if (cols % 16 != 0 || rows < 0 || cols < 0)
+        return NVO_ERR_SHAPE;
+    float amax, g;
+    int st = nvo_tensor_amax(x, rows, cols, ld, &amax);
+    if (st != NVO_OK)
+        return st;
+    st = nvo_global_scale(amax, &g);
+    *g_out = g;
+    if (st != NVO_OK)
+        return st;
+    nvo_quantize_with_global(x, rows, cols, ld, g, codes, scales, layout);
+    return NVO_OK;
+}
+
+/* ---------------------------------------------------------- dequantize */
+
+/* x_hat = bf16(RN(f32(e2m1(code)) * d)), d = RN(f32(s) / g) per block: the
+ * block scale restores the block's range and the tensor scale is divided
+ * back out ([P1] section 3, [P2] two-level scaling). */
+void nvo_dequantize(const uint8_t *codes, const uint8_t *scales, int layout, float g,
+                    int64_t rows, int64_t cols, uint16_t *y, int64_t ld)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            float sf = nvo_e4m3_decode(scales[nvo_sf_offset(r, b, rows, cols, layout)]);
+            float d = sf / g;
+            for (int i = 0; i < 16; ++i) {
+                int64_t c = b * 16 + i;
+                uint8_t byte = codes[r * (cols / 2) + c / 2];
+                uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+                float v = nvo_e2m1_decode(code) * d;
+                y[r * ld + c] = nvo_f32_to_bf16(v);
+            }
+        }
+}
+
+/* ----------------------------------------------------------------- GEMM */
+
+/* Exact real value of one quantized element as a double:
+ * e2m1(code) * s / g.  Both factors are exact in double. */
+static double elem_f64(const uint8_t *codes, const uint8_t *scales, int layout, double g,
+                       int64_t rows, int64_t cols, int64_t r, int64_t c)
+{
+    uint8_t byte = codes[r * (cols / 2) + c / 2];
+    uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+    double s = (double)nvo_e4m3_decode(scales[nvo_sf_offset(r, c / 16, rows, cols, layout)]);
+    return (double)nvo_e2m1_decode(code) * s / g;
+}
+
+/* Reference W4A4 linear, sampled: for t < count,
+ *   ref[t] = sum_k Ahat[i_t,k] * What[j_t,k]     (FP64)
+ *   abs[t] = sum_k |Ahat[i_t,k] * What[j_t,k]|   (FP64, for the tolerance)
+ * with Ahat/What the dequantized operands in FP64 (A is M x K, W is N x K,
+ * both row-major over K; D = A * W^T).  gw holds one tensor scale per
+ * sample so grouped (per-expert) weights use the same routine. */
+void nvo_gemm_ref(const uint8_t *a_codes, const uint8_t *a_sf, int a_layout, float ga, int64_t m,
+                  const uint8_t *w_codes, const uint8_t *w_sf, int w_layout, const float *gw,
+                  int64_t n, int64_t k, const int64_t *i_idx, const int64_t *j_idx,
+                  int64_t count, double *ref, double *abs_sum)
+{
+    for (int64_t t = 0; t < count; ++t) {
+        int64_t i = i_idx[t], j = j_idx[t];
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t kk = 0; kk < k; ++kk) {
+            double p = elem_f64(a_codes, a_sf, a_layout, (double)ga, m, k, i, kk) *
+                       elem_f64(w_codes, w_sf, w_layout, (double)gw[t], n, k, j, kk);
+            acc += p;
+            aacc += fabs(p);
+        }
+        ref[t] = acc;
+        abs_sum[t] = aacc;
+    }
+}
+
+/* Integer-exact form of the same dot product, before the tensor scales:
+ *   sum_k (2*e2m1(a)) * (512*sA) * (2*e2m1(w)) * (512*sW)
+ * Every factor is an integer (codes*2 in [-12,12], E4M3*512 in [0,229376]),
+ * so the int64 sum is exact for K up to ~1.2e6.  The real value is this
+ * sum / 2^20 / (gA*gW). */
+int64_t nvo_dot_exact_i64(const uint8_t *a_codes, const uint8_t *a_sf, int a_layout, int64_t m,
+                          const uint8_t *w_codes, const uint8_t *w_sf, int w_layout, int64_t n,
+                          int64_t k, int64_t i, int64_t j)
+{
+    int64_t acc = 0;
+    for (int64_t kk = 0; kk < k; ++kk) {
+        uint8_t ab = a_codes[i * (k / 2) + kk / 2];
+        uint8_t wb = w_codes[j * (k / 2) + kk / 2];
+        uint8_t ac = (kk & 1) ? (ab >> 4) : (ab & 15);
+        uint8_t wc = (kk & 1) ? (wb >> 4) : (wb & 15);
+        int64_t a2 = (int64_t)(2.0f * nvo_e2m1_decode(ac));
+        int64_t w2 = (int64_t)(2.0f * nvo_e2m1_decode(wc));
+        int64_t sa = (int64_t)(512.0f * nvo_e4m3_decode(a_sf[nvo_sf_offset(i, kk / 16, m, k, a_layout)]));
+        int64_t sw = (int64_t)(512.0f * nvo_e4m3_decode(w_sf[nvo_sf_offset(j, kk / 16, n, k, w_layout)]));
+        acc += a2 * sa * w2 * sw;
+    }
+    return acc;
+}

@@ -1,0 +1,193 @@
+"""ctypes front end of the NVFP4 CPU oracle (test infrastructure only).
+
+All arrays are numpy; BF16 tensors travel as their uint16 bit patterns.
+Torch CPU BF16 tensors are accepted wherever a BF16 array is expected.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from .build import LIB, build
+
+__all__ = [
+    "SF_SWIZZLED", "SF_LINEAR", "OK", "ERR_SHAPE", "ERR_NONFINITE", "ERR_RANGE",
+    "lib", "bf16_bits", "bf16_to_f32", "f32_to_bf16", "e2m1_decode", "e2m1_rne",
+    "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
+    "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
+    "dot_exact_i64", "Quantized",
+]
+
+SF_SWIZZLED, SF_LINEAR = 0, 1
+OK, ERR_SHAPE, ERR_NONFINITE, ERR_RANGE = 0, 3, 4, 5
+
+_lib = None
+_p = C.c_void_p
+_i64 = C.c_int64
+
+
+def lib() -> C.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = C.CDLL(LIB)
+        sig = {
+            "nvo_bf16_to_f32": (C.c_float, [C.c_uint16]),
+            "nvo_f32_to_bf16": (C.c_uint16, [C.c_float]),
+            "nvo_e2m1_decode": (C.c_float, [C.c_uint8]),
+            "nvo_e2m1_rne_satfinite": (C.c_uint8, [C.c_float]),
+            "nvo_e4m3_decode": (C.c_float, [C.c_uint8]),
+            "nvo_e4m3_rne_satfinite": (C.c_uint8, [C.c_float]),
+            "nvo_scales_bytes": (_i64, [_i64, _i64, C.c_int]),
+            "nvo_codes_bytes": (_i64, [_i64, _i64]),
+            "nvo_sf_offset": (_i64, [_i64, _i64, _i64, _i64, C.c_int]),
+            "nvo_tensor_amax": (C.c_int, [_p, _i64, _i64, _i64, C.POINTER(C.c_float)]),
+            "nvo_global_scale": (C.c_int, [C.c_float, C.POINTER(C.c_float)]),
+            "nvo_quantize_with_global": (None, [_p, _i64, _i64, _i64, C.c_float, _p, _p, C.c_int]),
+            "nvo_quantize": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int, C.POINTER(C.c_float)]),
+            "nvo_dequantize": (None, [_p, _p, C.c_int, C.c_float, _i64, _i64, _p, _i64]),
+            "nvo_gemm_ref": (None, [_p, _p, C.c_int, C.c_float, _i64, _p, _p, C.c_int, _p,
+                                    _i64, _i64, _p, _p, _i64, _p, _p]),
+            "nvo_dot_exact_i64": (_i64, [_p, _p, C.c_int, _i64, _p, _p, C.c_int, _i64,
+                                         _i64, _i64, _i64]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def bf16_bits(x) -> np.ndarray:
+    """uint16 bit patterns of a BF16 array (torch CPU tensor or numpy u16)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(v: float) -> int:
+    return int(lib().nvo_f32_to_bf16(float(v)))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().nvo_e2m1_decode(code))
+
+
+def e2m1_rne(y: float) -> int:
+    return int(lib().nvo_e2m1_rne_satfinite(float(np.float32(y))))
+
+
+def e4m3_decode(b: int) -> float:
+    return float(lib().nvo_e4m3_decode(b))
+
+
+def e4m3_rne(v: float) -> int:
+    return int(lib().nvo_e4m3_rne_satfinite(float(np.float32(v))))
+
+
+def scales_bytes(rows: int, cols: int, layout: int) -> int:
+    return int(lib().nvo_scales_bytes(rows, cols, layout))
+
+
+def sf_offset(r: int, c: int, rows: int, cols: int, layout: int) -> int:
+    return int(lib().nvo_sf_offset(r, c, rows, cols, layout))
+
+
+def tensor_amax(x) -> tuple[int, float]:
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    out = C.c_float()
+    st = lib().nvo_tensor_amax(_ptr(b), rows, cols, cols, C.byref(out))
+    return st, float(out.value)
+
+
+def global_scale(amax: float) -> tuple[int, float]:
+    out = C.c_float()
+    st = lib().nvo_global_scale(float(np.float32(amax)), C.byref(out))
+    return st, float(out.value)
+
+
+class Quantized:
+    """Oracle NVFP4 tensor: codes [rows, cols/2] u8, scales (flat u8), g."""
+
+    def __init__(self, codes, scales, g, rows, cols, layout):
+        self.codes, self.scales, self.g = codes, scales, np.float32(g)
+        self.rows, self.cols, self.layout = rows, cols, layout
+
+    def dequantize(self) -> np.ndarray:
+        return dequantize(self.codes, self.scales, self.layout, self.g, self.rows, self.cols)
+
+
+def quantize_with_global(x, g: float, layout: int = SF_SWIZZLED) -> Quantized:
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    lib().nvo_quantize_with_global(_ptr(b), rows, cols, cols, float(np.float32(g)),
+                                   _ptr(codes), _ptr(scales), layout)
+    return Quantized(codes, scales, g, rows, cols, layout)
+
+
+def quantize(x, layout: int = SF_SWIZZLED) -> tuple[int, Quantized]:
+    """Two-level quantize (amax -> g -> encode).  Returns (status, tensor)."""
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    g = C.c_float(0.0)
+    st = lib().nvo_quantize(_ptr(b), rows, cols, cols, _ptr(codes), _ptr(scales), layout,
+                            C.byref(g))
+    return st, Quantized(codes, scales, g.value, rows, cols, layout)
+
+
+def dequantize(codes, scales, layout, g, rows, cols) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    y = np.zeros((rows, cols), np.uint16)
+    lib().nvo_dequantize(_ptr(codes), _ptr(scales), layout, float(np.float32(g)), rows, cols,
+                         _ptr(y), cols)
+    return y
+
+
+def gemm_ref(a: Quantized, w: Quantized, i_idx, j_idx, gw=None):
+    """Sampled FP64 reference of D = Ahat * What^T at pairs (i_idx, j_idx).
+
+    ``gw`` (per sample) overrides w.g, for per-expert weight scales.
+    Returns (ref, abs_sum) float64 arrays."""
+    assert a.cols == w.cols
+    i_idx = np.ascontiguousarray(i_idx, np.int64)
+    j_idx = np.ascontiguousarray(j_idx, np.int64)
+    n = len(i_idx)
+    if gw is None:
+        gw = np.full(n, w.g, np.float32)
+    gw = np.ascontiguousarray(gw, np.float32)
+    ref = np.zeros(n, np.float64)
+    ab = np.zeros(n, np.float64)
+    lib().nvo_gemm_ref(_ptr(a.codes), _ptr(a.scales), a.layout, float(a.g), a.rows,
+                       _ptr(w.codes), _ptr(w.scales), w.layout, _ptr(gw), w.rows, a.cols,
+                       _ptr(i_idx), _ptr(j_idx), n, _ptr(ref), _ptr(ab))
+    return ref, ab
+
+
+def dot_exact_i64(a: Quantized, w: Quantized, i: int, j: int) -> int:
+    return int(lib().nvo_dot_exact_i64(_ptr(a.codes), _ptr(a.scales), a.layout, a.rows,
+                                       _ptr(w.codes), _ptr(w.scales), w.layout, w.rows,
+                                       a.cols, i, j))
+
+
+if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):
+    lib()
