@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 hot path on B200.
+
+One step = one W4A4 linear layer of the dense-FFN workload (the 12B hybrid
+model's FFN shape): quantize the BF16 activations A [8192 x 5120] to NVFP4
+(tensor amax, then block scales + codes) and run the block-scaled FP4 GEMM
+against the pre-quantized weight W [20480 x 5120], writing D [8192 x 20480]
+BF16.  Metric: NVFP4 GEMM TFLOP/s over the whole step (2*M*N*K per step).
+The same run measures standalone quantize GB/s on the 2^28-value tensor of
+the quantize sweep (the metric's second half) as ``quantize``.
+
+Launch: ``python bench.py [--gpus N] [--steps K] [--warmup W]``; for N > 1
+under torch.distributed.run, one rank per GPU.  The path has no data
+exchange, so N > 1 runs N replicas (weak scaling) and only the timing is
+reduced across ranks (max).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, K = 8192, 20480, 5120
+SWEEP_N = 1 << 28
+METRIC = "NVFP4 GEMM TFLOPS (% of FP4 peak); quantize GB/s (% of HBM BW), 1 B200"
+WORKLOAD = "w4a4_linear_ffn_M8192_N20480_K5120 (quantize A + block-scaled FP4 GEMM)"
+L2_FLUSH_BYTES = 256 << 20
+# Algorithmic bytes per value of a two-pass quantize (amax read 2 B, then
+# read 2 B + write 0.5 B codes + 0.0625 B scales) and of the encode pass.
+QUANT_BYTES_PER_VALUE_2PASS = 4.5625
+ENCODE_BYTES_PER_VALUE = 2.5625
+FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs"), d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons every few ms during a region."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x100: "sync_boost"}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.stop_ev = threading.Event()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "source": "nvml" if self.ok else "unavailable"}
+        mhz = [s[0] for s in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = sorted({name for bit, name in self.REASONS.items() if mask & bit} - {"gpu_idle"})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz), "source": "nvml"}
+
+
+# ------------------------------------------------------------ GPU workload
+class Workload:
+    def __init__(self, device):
+        from nvfp4_block_scaled_22_b200 import binding as nb
+        from nvfp4_block_scaled_22_b200 import inputs
+        self.nb = nb
+        self.dev = device
+        nb.lib()
+        self.ws = nb.Workspace(device)
+        w = inputs.ffn_weight(device=device)
+        self.qw = nb.nvfp4_quantize(w, workspace=self.ws)
+        del w
+        self.a = inputs.ffn_activation(M, device=device)
+        self.qa = nb.NVFP4Tensor.empty(M, K, device=device)
+        self.d = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+        st = nb.nvfp4_check_status(self.ws)
+        if st != 0:
+            raise RuntimeError(f"setup status {st}")
+
+    def flush(self):
+        self.flush_buf.zero_()
+
+    def quantize(self):
+        self.nb.nvfp4_quantize(self.a, out=self.qa, workspace=self.ws)
+
+    def gemm(self):
+        self.nb.nvfp4_gemm(self.qa, self.qw, out=self.d, workspace=self.ws)
+
+
+def time_steps(wl: Workload, steps: int, warmup: int):
+    """Device time of each step (flush outside the events)."""
+    for _ in range(warmup):
+        wl.flush()
+        wl.quantize()
+        wl.gemm()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    n0 = wl.nb.nvfp4_launch_count()
+    for i in range(steps):
+        wl.flush()
+        ev[i][0].record()
+        wl.quantize()
+        ev[i][1].record()
+        wl.gemm()
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    launches = wl.nb.nvfp4_launch_count() - n0
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    return step_ms, quant_ms, gemm_ms, launches
+
+
+def time_sweep_quantize(nb, device, iters=10):
+    from nvfp4_block_scaled_22_b200 import inputs
+    x = inputs.sweep_tensor(SWEEP_N, device=device)
+    q = nb.NVFP4Tensor.empty(x.shape[0], x.shape[1], device=device)
+    ws = nb.Workspace(device)
+    for _ in range(3):
+        nb.nvfp4_quantize(x, out=q, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for a, b in evs:                 # 512 MiB input > L2: no flush needed
+        a.record()
+        nb.nvfp4_quantize(x, out=q, workspace=ws)
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    # encode pass alone (caller-supplied tensor scale)
+    for a, b in evs:
+        a.record()
+        nb.nvfp4_quantize(x, out=q, global_supplied=True, workspace=ws)
+        b.record()
+    torch.cuda.synchronize()
+    ms1 = statistics.median(a.elapsed_time(b) for a, b in evs)
+    st = nb.nvfp4_check_status(ws)
+    del x, q
+    return ms, ms1, st
+
+
+def time_e2e(wl: Workload, steps: int, warmup: int):
+    """Same step through the public API from pinned host memory: H2D of A,
+    quantize, GEMM, D2H of D, all inside the events."""
+    a_host = wl.a.cpu().pin_memory()
+    d_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    a_dev = torch.empty_like(wl.a)
+
+    def step():
+        a_dev.copy_(a_host, non_blocking=True)
+        wl.nb.nvfp4_quantize(a_dev, out=wl.qa, workspace=wl.ws)
+        wl.nb.nvfp4_gemm(wl.qa, wl.qw, out=wl.d, workspace=wl.ws)
+        d_host.copy_(wl.d, non_blocking=True)
+
+    for _ in range(max(1, warmup)):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, min(steps, 20))
+    s.record()
+    for _ in range(n):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / n
+    return ms, a_host.numel() * 2, d_host.numel() * 2
+
+
+# ------------------------------------------------------- CPU oracle timing
+def oracle_sample(rows: int = 1, cols: int = 4096, seed: int = 0):
+    """Oracle on a bounded sample of the step: quantize `rows` rows of A (with
+    the full-tensor amax pass) and compute their first `cols` outputs of the
+    FP64 GEMM against the oracle-quantized W.  Returns (seconds, flops)."""
+    import numpy as np
+    import oracle
+    from nvfp4_block_scaled_22_b200 import inputs
+    cache = oracle_sample.__dict__.setdefault("cache", {})
+    if "w" not in cache:
+        w = inputs.ffn_weight()
+        st, qw = oracle.quantize(w)
+        a = inputs.ffn_activation(M)
+        cache["w"], cache["a"] = qw, a
+    qw, a = cache["w"], cache["a"]
+    r0 = (seed * rows) % M
+    t0 = time.perf_counter()
+    st, amax = oracle.tensor_amax(a)
+    st, g = oracle.global_scale(amax)
+    qa = oracle.quantize_with_global(a[r0:r0 + rows], g)
+    ii, jj = np.meshgrid(np.arange(rows), np.arange(cols), indexing="ij")
+    oracle.gemm_ref(qa, qw, ii.ravel(), jj.ravel())
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * rows * cols * K
+
+
+def cpu_baseline_entry():
+    dt, flops = oracle_sample()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"1 of {M} rows of A: tensor amax over all of A, quantize the row, "
+                      f"then 4096 of {N} outputs of the FP64 GEMM (K={K}) against the "
+                      f"oracle-quantized W; single-threaded C ({dt:.2f} s)"}
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    oracle_sample()   # builds the oracle and quantizes W once (setup, untimed)
+    for i in range(args.warmup):
+        oracle_sample(seed=i)
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        dt, f = oracle_sample(seed=args.warmup + i)
+        times.append(dt)
+        flops = f
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " [oracle sample per step: 1 row x 4096 outputs]",
+                   "M": M, "N": N, "K": K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: 1 row of A quantized (after the full-tensor "
+                                   "amax) and 4096 outputs of the FP64 GEMM, K=5120"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank, local_rank, world = env_rank()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = measured_peaks()
+    fp4_peak = bf16_tf * FP4_OVER_BF16
+
+    wl = Workload(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms, quant_ms, gemm_ms, launches = time_steps(wl, args.steps, args.warmup)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    st = wl.nb.nvfp4_check_status(wl.ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed steps")
+
+    total_ms = sum(step_ms)
+    gemm_avg = sum(gemm_ms) / len(gemm_ms)
+    quant_avg = sum(quant_ms) / len(quant_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms, gemm_avg, quant_avg], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, gemm_avg, quant_avg = t.tolist()
+    flops = 2.0 * M * N * K
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    gemm_tflops = flops / (gemm_avg / 1e3) / 1e12
+
+    sweep_ms, sweep_ms1, sst = time_sweep_quantize(wl.nb, device)
+    e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup)
+    if dist is not None:
+        t = torch.tensor([sweep_ms, sweep_ms1, e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        sweep_ms, sweep_ms1, e2e_ms = t.tolist()
+
+    if rank == 0:
+        gbs_2pass = SWEEP_N * QUANT_BYTES_PER_VALUE_2PASS / (sweep_ms / 1e3) / 1e9
+        gbs_1pass = SWEEP_N * ENCODE_BYTES_PER_VALUE / (sweep_ms1 / 1e3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 accumulate, bf16 out)",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "weights": "pre-quantized once, outside the timed region"},
+            "roofline": {"kernel": "k_gemm_nvf4", "bound": "tensor",
+                         "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_peak,
+                         "peak_source": f"{peak_src} bf16 burst {bf16_tf} TFLOP/s x "
+                                        f"{FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
+                         "traffic": None, "ms_per_launch": gemm_avg},
+            "quantize": {"workload": "quantize sweep, 2^28 BF16 values [65536 x 4096]",
+                         "gbs_two_pass": gbs_2pass, "frac_two_pass": gbs_2pass / hbm_gbs,
+                         "ms_two_pass": sweep_ms,
+                         "gbs_supplied_scale": gbs_1pass, "frac_supplied_scale": gbs_1pass / hbm_gbs,
+                         "ms_supplied_scale": sweep_ms1,
+                         "bytes_per_value": {"two_pass": QUANT_BYTES_PER_VALUE_2PASS,
+                                             "supplied_scale": ENCODE_BYTES_PER_VALUE},
+                         "peak_gbs": hbm_gbs, "peak_source": f"{peak_src} hbm_gbs",
+                         "status": sst},
+            "activation_quantize_ms": quant_avg,
+            "gpu_launches": launches,
+            "e2e": {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_entry()
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,225 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so, the B200 (sm_100a) NVFP4 hot path.
+ *
+ * NVFP4 stores a tensor as 4-bit E2M1 codes (values +-0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6), one E4M3 scale per 16 consecutive values along the last dimension,
+ * and one FP32 scale per tensor.  Sources: "NVFP4: how NVIDIA pre-trained a
+ * 12B model on 10T tokens" (axbrief.com), section "E2M1 format and
+ * two-level scaling"; "NVIDIA shrank GLM-5.2 to 4 bits" (iwan.kr), section 3;
+ * "FP4 KV-cache quantization" (theddari.com), sections "KV cache size
+ * example" and "FP4 formats compared".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Memory: every pointer named d_* or held in an nvfp4_tensor is DEVICE
+ *   memory owned by the caller.  The library allocates no device memory and
+ *   keeps no handle to caller buffers after a call returns.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *   default stream).  Work is enqueued asynchronously; argument errors are
+ *   returned synchronously before anything is enqueued.
+ * - Device-side errors (non-finite input, out-of-range tensor amax, a
+ *   pipeline wait that exceeded its bound) are recorded in the 32-bit status
+ *   word at the start of the caller's workspace.  The first error sticks
+ *   until nvfp4_check_status() reads and clears it.  A workspace must be
+ *   zero-filled once before its first use.
+ * - Alignment: tensor base pointers and row pitches 16-byte aligned.
+ * - Device: compute capability 10.0 (B200, sm_100a) is required; any other
+ *   device gives NVFP4_ERR_UNSUPPORTED_DEVICE.  There is no fallback.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad enum */
+    NVFP4_ERR_ALIGNMENT = 2,        /* pointer or pitch not 16-byte aligned */
+    NVFP4_ERR_SHAPE = 3,            /* shape rule of the call violated */
+    NVFP4_ERR_NONFINITE = 4,        /* input holds Inf or NaN (device-side) */
+    NVFP4_ERR_RANGE = 5,            /* tensor amax so small that g > 2^118 */
+    NVFP4_ERR_WORKSPACE = 6,        /* workspace missing or too small */
+    NVFP4_ERR_TIMEOUT = 7,          /* a device pipeline wait gave up */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 8,
+    NVFP4_ERR_CUDA = 9              /* a CUDA runtime/driver call failed */
+} nvfp4_status;
+
+/* Block-scale layouts.
+ * SWIZZLED_128x4: the tiled layout the block-scaled tensor-core MMA reads.
+ *   For row r and scale column c (= element column / 16), with
+ *   S4 = ceil(cols/16 / 4) * 4 padded scale columns:
+ *     offset = ((r/128) * (S4/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+ *   The buffer covers ceil(rows/128)*128 rows x S4 columns; padding holds 0.
+ * LINEAR: row-major [rows x cols/16], offset = r * (cols/16) + c. */
+typedef enum {
+    NVFP4_SF_SWIZZLED_128x4 = 0,
+    NVFP4_SF_LINEAR = 1
+} nvfp4_sf_layout;
+
+/* An NVFP4 tensor of `rows` x `cols` logical values.
+ * codes : rows x cols/2 bytes, row-major, two codes per byte, element 2i in
+ *         the low nibble and 2i+1 in the high nibble.  Sign in bit 3.
+ * scales: nvfp4_scales_bytes(rows, cols, sf_layout) bytes of E4M3 scales.
+ * global: one float, the tensor scale g = 448*6 / amax(tensor) (g = 1 for an
+ *         all-zero tensor).  A value x is represented as
+ *         e2m1(code) * e4m3(scale) / g. */
+typedef struct {
+    void *codes;
+    void *scales;
+    float *global;
+    int64_t rows;
+    int64_t cols;
+    int32_t sf_layout;
+} nvfp4_tensor;
+
+/* Operation ids for nvfp4_workspace_bytes(). */
+typedef enum {
+    NVFP4_OP_QUANTIZE = 0,
+    NVFP4_OP_DEQUANTIZE = 1,
+    NVFP4_OP_GEMM = 2,
+    NVFP4_OP_GROUPED_GEMM = 3,
+    NVFP4_OP_QUANTIZE_GATHER = 4
+} nvfp4_op;
+
+/* ---- sizes ------------------------------------------------------------ */
+
+/* Bytes of the packed code array: rows * cols / 2. */
+NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the block-scale array for the given layout (see above). */
+NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout);
+
+/* Bytes of workspace the operation needs (at least 16; the first 4 bytes
+ * are the status word).  The arguments are the operation's sizes
+ * (rows/cols, or m/n/k) and the group count for grouped calls; the current
+ * implementation needs a fixed amount per operation. */
+NVFP4_API size_t nvfp4_workspace_bytes(int32_t op, int64_t a, int64_t b, int64_t c, int32_t groups);
+
+/* ---- quantize --------------------------------------------------------- */
+
+/* Two-level NVFP4 quantization of a row-major BF16 matrix.
+ * ("NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens", section
+ * "E2M1 format and two-level scaling": a per-tensor FP32 scale sets the
+ * range, an E4M3 scale per 16-value block maps each block's amax close to
+ * the FP4 maximum.)
+ *   amax = max |x|;  g = RN(2688 / amax)            (skipped if global_supplied)
+ *   per 16-block b of a row:  s_b = e4m3_rne_satfinite(RN(RN(amax_b / 6) * g))
+ *                             e_b = s_b ? RN(g / s_b) : 0
+ *   code = e2m1_rne_satfinite(RN(x * e_b)), sign kept (-0 -> 0x8)
+ * x        : device BF16, out->rows x out->cols, row pitch `ld` elements.
+ * out      : destination; codes/scales/global are written.  out->cols must
+ *            be a multiple of 16, out->rows >= 0.
+ * global_supplied: 0 = compute amax and g and store g to *out->global;
+ *            1 = use the g already stored at *out->global (one pass).
+ * Errors: argument checks synchronously; Inf/NaN in x -> NVFP4_ERR_NONFINITE
+ *   and amax below 2688 * 2^-118 -> NVFP4_ERR_RANGE, both via the status word
+ *   (outputs then unspecified). */
+NVFP4_API nvfp4_status nvfp4_quantize(const void *x, int64_t ld, const nvfp4_tensor *out,
+                            int32_t global_supplied, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Tensor scale only: *d_global = RN(2688 / max|x|) over a rows x cols BF16
+ * matrix with pitch ld (1.0 if all zero).  Same status rules as
+ * nvfp4_quantize.  Lets a caller share one g between tensors or take g from
+ * a tensor other than the one encoded (nvfp4_quantize_gather). */
+NVFP4_API nvfp4_status nvfp4_global_scale(const void *x, int64_t ld, int64_t rows, int64_t cols,
+                                float *d_global, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* Quantize rows gathered through a row map, for MoE expert batches.
+ * Output row r takes source row d_gather[r] of x (src_rows x out->cols,
+ * pitch ld); d_gather[r] == -1 makes row r a zero padding row (all codes
+ * and scales 0).  out->rows is the number of gathered rows.  A map entry
+ * >= src_rows is not read: its row is zeroed and NVFP4_ERR_INVALID_ARG is
+ * recorded in the status word.
+ * global_supplied: 1 = use *out->global (e.g. from nvfp4_global_scale over
+ *   the whole source), 0 = amax over the gathered (non -1) rows.
+ * ("NVIDIA shrank GLM-5.2 to 4 bits", section 1: weights and activations of
+ * the MoE expert linears are NVFP4; section 2: 256 experts, 8 per token.) */
+NVFP4_API nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
+                                   const int32_t *d_gather, const nvfp4_tensor *out,
+                                   int32_t global_supplied, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/* ---- dequantize ------------------------------------------------------- */
+
+/* NVFP4 -> BF16:  y = bf16_rne(RN(e2m1(code) * d_b)),  d_b = RN(s_b / g).
+ * (The block scale and tensor scale restore each value's range; "NVIDIA
+ * shrank GLM-5.2 to 4 bits", section 3.)  y: device BF16 in->rows x in->cols,
+ * pitch ld.  Both scale layouts are accepted. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void *stream);
+
+/* ---- GEMM ------------------------------------------------------------- */
+
+/* W4A4 linear layer on the FP4 tensor cores (block-scaled MMA, FP32
+ * accumulation):  D[i,j] = bf16_rne(alpha * sum_k a_ik * w_jk), where a and w
+ * are the E2M1 codes times their E4M3 block scales and
+ * alpha = RN(1 / RN(gA * gW)) is formed on the device from *A->global and
+ * *W->global.  ("NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens",
+ * section "MXFP4 vs 36% token efficiency and Blackwell speed": FP4 GEMM on
+ * Blackwell; section "Four stabilisation devices": Fprop/Dgrad/Wgrad GEMMs
+ * in NVFP4.)
+ * A: M x K, W: N x K (both K-major, i.e. D = A * W^T), both with
+ *    NVFP4_SF_SWIZZLED_128x4 scales.  K % 64 == 0; M, N >= 1 arbitrary.
+ * D: device BF16 M x N, row pitch ldd >= N (ldd % 8 == 0).
+ * Accuracy: |D - exact| <= 1e-3 * sum_k |a_ik w_jk| / (gA gW) + BF16 rounding. */
+NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Grouped W4A4 GEMM over MoE experts (one launch for all groups).
+ * A: stacked activation rows, group g occupying padded rows
+ *    [d_slot_offsets[g], d_slot_offsets[g+1]) -- every offset a multiple of
+ *    128 -- of which the first d_group_rows[g] are real rows.  Padding rows
+ *    must hold zero codes and scales (nvfp4_quantize_gather writes them).
+ *    A->rows (the padded capacity) must be a multiple of 128; at most 512
+ *    groups.  Offsets that break these rules are caught on the device: the
+ *    call then computes nothing and records NVFP4_ERR_SHAPE.
+ * W: groups stacked weights, [groups * n] x K; group g uses rows
+ *    [g*n, (g+1)*n) and tensor scale d_w_globals[g].  n % 128 == 0.
+ * D: BF16 rows in the same padded layout as A, pitch ldd >= n; only real
+ *    rows are written.  alpha_g = RN(1 / RN(gA * d_w_globals[g])).
+ * Offsets and row counts stay on the device (no host synchronisation). */
+NVFP4_API nvfp4_status nvfp4_grouped_gemm(int32_t groups, const int32_t *d_slot_offsets,
+                                const int32_t *d_group_rows, const nvfp4_tensor *A,
+                                const nvfp4_tensor *W, const float *d_w_globals, int64_t n,
+                                void *D, int64_t ldd, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* ---- status ----------------------------------------------------------- */
+
+/* Synchronise `stream`, return the workspace's status word and reset it to
+ * NVFP4_OK.  Returns NVFP4_ERR_CUDA if the synchronisation itself failed. */
+NVFP4_API nvfp4_status nvfp4_check_status(void *workspace, void *stream);
+
+/* Static, human-readable name of a status code. */
+NVFP4_API const char *nvfp4_status_string(nvfp4_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+NVFP4_API int32_t nvfp4_version(void);
+
+/* Number of kernels this library has enqueued since load (all entry points;
+ * for accounting in benchmarks). */
+NVFP4_API int64_t nvfp4_launch_count(void);
+
+/* Bound, in SM clock cycles, on every pipeline wait inside the GEMM kernels
+ * (default 2e9, about one second).  A wait that runs past it makes the
+ * kernel record NVFP4_ERR_TIMEOUT, drain what it issued and exit instead of
+ * hanging.  cycles <= 0 restores the default.  Returns the previous bound.
+ * Meant for tests of the timeout path. */
+NVFP4_API long long nvfp4_set_wait_limit_cycles(long long cycles);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

@@ -1,0 +1,277 @@
+"""Thin ctypes binding of libnvfp4.so (the C ABI in include/nvfp4.h).
+
+Argument marshalling only: every step of the NVFP4 path runs in the CUDA
+kernels of libnvfp4.so.  PyTorch supplies device memory and streams.  There
+is no CPU fallback -- loading fails loudly if the library is missing.
+
+Function names follow the C ABI (``nvfp4_quantize`` ...), taking torch
+tensors instead of raw pointers.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+
+SF_SWIZZLED = 0
+SF_LINEAR = 1
+
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_GROUPED_GEMM, OP_QUANTIZE_GATHER = range(5)
+
+STATUS_NAMES = {
+    0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_ALIGNMENT", 3: "NVFP4_ERR_SHAPE",
+    4: "NVFP4_ERR_NONFINITE", 5: "NVFP4_ERR_RANGE", 6: "NVFP4_ERR_WORKSPACE",
+    7: "NVFP4_ERR_TIMEOUT", 8: "NVFP4_ERR_UNSUPPORTED_DEVICE", 9: "NVFP4_ERR_CUDA",
+}
+
+# Symbols the header declares; the library must export every one.
+EXPORTED = (
+    "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
+    "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
+    "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
+    "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles",
+)
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class CTensor(C.Structure):
+    """Mirror of ``nvfp4_tensor``."""
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("global_", C.c_void_p),
+                ("rows", C.c_int64), ("cols", C.c_int64), ("sf_layout", C.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libnvfp4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libnvfp4.so not built at {LIB_PATH}; run "
+                              "python -m nvfp4_block_scaled_22_b200.build")
+        L = C.CDLL(LIB_PATH)
+        i64, i32, vp, sz = C.c_int64, C.c_int32, C.c_void_p, C.c_size_t
+        T = C.POINTER(CTensor)
+        sig = {
+            "nvfp4_codes_bytes": (sz, [i64, i64]),
+            "nvfp4_scales_bytes": (sz, [i64, i64, i32]),
+            "nvfp4_workspace_bytes": (sz, [i32, i64, i64, i64, i32]),
+            "nvfp4_quantize": (C.c_int, [vp, i64, T, i32, vp, sz, vp]),
+            "nvfp4_global_scale": (C.c_int, [vp, i64, i64, i64, vp, vp, sz, vp]),
+            "nvfp4_quantize_gather": (C.c_int, [vp, i64, i64, vp, T, i32, vp, sz, vp]),
+            "nvfp4_dequantize": (C.c_int, [T, vp, i64, vp]),
+            "nvfp4_gemm": (C.c_int, [T, T, vp, i64, vp, sz, vp]),
+            "nvfp4_grouped_gemm": (C.c_int, [i32, vp, vp, T, T, vp, i64, vp, i64, vp, sz, vp]),
+            "nvfp4_check_status": (C.c_int, [vp, vp]),
+            "nvfp4_status_string": (C.c_char_p, [C.c_int]),
+            "nvfp4_version": (i32, []),
+            "nvfp4_launch_count": (i64, []),
+            "nvfp4_set_wait_limit_cycles": (C.c_longlong, [C.c_longlong]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise NVFP4Error(st, where)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+# ------------------------------------------------------------------ sizes
+def nvfp4_codes_bytes(rows: int, cols: int) -> int:
+    return int(lib().nvfp4_codes_bytes(rows, cols))
+
+
+def nvfp4_scales_bytes(rows: int, cols: int, layout: int = SF_SWIZZLED) -> int:
+    return int(lib().nvfp4_scales_bytes(rows, cols, layout))
+
+
+def nvfp4_workspace_bytes(op: int, a=0, b=0, c=0, groups=0) -> int:
+    return int(lib().nvfp4_workspace_bytes(op, a, b, c, groups))
+
+
+# ---------------------------------------------------------- tensor types
+class NVFP4Tensor:
+    """Device NVFP4 tensor: packed codes, block scales and the tensor scale.
+
+    ``codes`` uint8 [rows, cols/2], ``scales`` uint8 [scales_bytes],
+    ``global_scale`` float32 [1]; all on one CUDA device."""
+
+    def __init__(self, codes, scales, global_scale, rows, cols, layout):
+        self.codes, self.scales, self.global_scale = codes, scales, global_scale
+        self.rows, self.cols, self.layout = rows, cols, layout
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, layout: int = SF_SWIZZLED, device="cuda",
+              global_scale=None):
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(nvfp4_scales_bytes(rows, cols, layout), dtype=torch.uint8,
+                             device=device)
+        if global_scale is None:
+            global_scale = torch.zeros(1, dtype=torch.float32, device=device)
+        return cls(codes, scales, global_scale, rows, cols, layout)
+
+    def c_struct(self) -> CTensor:
+        return CTensor(_ptr(self.codes), _ptr(self.scales), _ptr(self.global_scale),
+                       self.rows, self.cols, self.layout)
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.scales.numel()
+
+
+class Workspace:
+    """Zero-initialised device workspace (status word + scratch)."""
+
+    def __init__(self, device="cuda", nbytes: int | None = None):
+        if nbytes is None:
+            nbytes = max(nvfp4_workspace_bytes(op) for op in range(5))
+        self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+
+_default_ws: dict[int, Workspace] = {}
+
+
+def default_workspace(device=None) -> Workspace:
+    dev = torch.device(device or "cuda")
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    if idx not in _default_ws:
+        _default_ws[idx] = Workspace(torch.device("cuda", idx))
+    return _default_ws[idx]
+
+
+# ------------------------------------------------------------ operations
+def nvfp4_quantize(x: torch.Tensor, out: NVFP4Tensor | None = None, layout: int = SF_SWIZZLED,
+                   global_supplied: bool = False, workspace: Workspace | None = None,
+                   stream=None) -> NVFP4Tensor:
+    """Two-level NVFP4 quantization of a 2-D BF16 CUDA tensor (row pitch
+    x.stride(0)).  With ``global_supplied`` the tensor scale already in
+    ``out.global_scale`` is used."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out is None:
+        out = NVFP4Tensor.empty(rows, cols, layout, x.device)
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize(x.data_ptr(), x.stride(0), C.byref(t), int(global_supplied),
+                                ws.ptr, ws.nbytes, _stream(stream)), "nvfp4_quantize")
+    return out
+
+
+def nvfp4_global_scale(x: torch.Tensor, out: torch.Tensor | None = None,
+                       workspace: Workspace | None = None, stream=None) -> torch.Tensor:
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    if out is None:
+        out = torch.zeros(1, dtype=torch.float32, device=x.device)
+    ws = workspace or default_workspace(x.device)
+    _check(lib().nvfp4_global_scale(x.data_ptr(), x.stride(0), x.shape[0], x.shape[1],
+                                    out.data_ptr(), ws.ptr, ws.nbytes, _stream(stream)),
+           "nvfp4_global_scale")
+    return out
+
+
+def nvfp4_quantize_gather(x: torch.Tensor, gather: torch.Tensor, out: NVFP4Tensor | None = None,
+                          layout: int = SF_SWIZZLED, global_supplied: bool = False,
+                          workspace: Workspace | None = None, stream=None) -> NVFP4Tensor:
+    """Quantize rows x[gather[r]] (gather int32 CUDA, -1 = zero row)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    assert gather.dtype == torch.int32 and gather.is_contiguous()
+    rows, cols = gather.numel(), x.shape[1]
+    if out is None:
+        out = NVFP4Tensor.empty(rows, cols, layout, x.device)
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize_gather(x.data_ptr(), x.stride(0), x.shape[0], gather.data_ptr(),
+                                       C.byref(t), int(global_supplied), ws.ptr, ws.nbytes,
+                                       _stream(stream)), "nvfp4_quantize_gather")
+    return out
+
+
+def nvfp4_dequantize(t: NVFP4Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((t.rows, t.cols), dtype=torch.bfloat16, device=t.codes.device)
+    ct = t.c_struct()
+    _check(lib().nvfp4_dequantize(C.byref(ct), out.data_ptr(), out.stride(0), _stream(stream)),
+           "nvfp4_dequantize")
+    return out
+
+
+def nvfp4_gemm(a: NVFP4Tensor, w: NVFP4Tensor, out: torch.Tensor | None = None,
+               workspace: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D = A * W^T on the FP4 tensor cores, BF16 [a.rows, w.rows]."""
+    if out is None:
+        out = torch.empty((a.rows, w.rows), dtype=torch.bfloat16, device=a.codes.device)
+    ws = workspace or default_workspace(a.codes.device)
+    ca, cw = a.c_struct(), w.c_struct()
+    _check(lib().nvfp4_gemm(C.byref(ca), C.byref(cw), out.data_ptr(), out.stride(0), ws.ptr,
+                            ws.nbytes, _stream(stream)), "nvfp4_gemm")
+    return out
+
+
+def nvfp4_grouped_gemm(slot_offsets: torch.Tensor, group_rows: torch.Tensor, a: NVFP4Tensor,
+                       w: NVFP4Tensor, w_globals: torch.Tensor, n: int,
+                       out: torch.Tensor | None = None, workspace: Workspace | None = None,
+                       stream=None) -> torch.Tensor:
+    """Grouped D_g = A_g * W_g^T over expert slots (see nvfp4_grouped_gemm in
+    the header).  slot_offsets/group_rows int32 CUDA, w_globals float32 CUDA."""
+    groups = group_rows.numel()
+    if out is None:
+        out = torch.empty((a.rows, n), dtype=torch.bfloat16, device=a.codes.device)
+    ws = workspace or default_workspace(a.codes.device)
+    ca, cw = a.c_struct(), w.c_struct()
+    _check(lib().nvfp4_grouped_gemm(groups, slot_offsets.data_ptr(), group_rows.data_ptr(),
+                                    C.byref(ca), C.byref(cw), w_globals.data_ptr(), n,
+                                    out.data_ptr(), out.stride(0), ws.ptr, ws.nbytes,
+                                    _stream(stream)), "nvfp4_grouped_gemm")
+    return out
+
+
+def nvfp4_check_status(workspace: Workspace | None = None, stream=None) -> int:
+    """Synchronise, return and clear the workspace status word (0 = OK)."""
+    ws = workspace or default_workspace()
+    return int(lib().nvfp4_check_status(ws.ptr, _stream(stream)))
+
+
+def nvfp4_status_string(status: int) -> str:
+    return lib().nvfp4_status_string(status).decode()
+
+
+def nvfp4_launch_count() -> int:
+    return int(lib().nvfp4_launch_count())
+
+
+def nvfp4_set_wait_limit_cycles(cycles: int) -> int:
+    return int(lib().nvfp4_set_wait_limit_cycles(cycles))

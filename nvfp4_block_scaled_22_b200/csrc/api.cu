@@ -1,0 +1,402 @@
+// Host side of libnvfp4.so: the C ABI declared in include/nvfp4.h.
+// Argument validation, device check, tensor-map encoding and launches.
+// No device memory is allocated here; every buffer belongs to the caller.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "nvfp4.h"
+
+using namespace nvfp4;
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kStatusBytes = 256;          // status word + reserved
+constexpr int kMaxPartials = 1024;            // CTAs of the amax pass
+constexpr long long kDefaultTimeoutCycles = 2000000000ll;   // ~1 s at 1.9 GHz
+
+struct DeviceInfo {
+    bool checked = false;
+    bool supported = false;
+    int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+long long g_timeout_cycles = kDefaultTimeoutCycles;
+
+nvfp4_status current_device(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.supported = (major == 10 && minor == 0);
+        d.sms = sms;
+        d.checked = true;
+    }
+    if (!d.supported) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    *sms = d.sms;
+    return NVFP4_OK;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+nvfp4_status launched(cudaError_t e, int n = 1) {
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    g_launches.fetch_add(n, std::memory_order_relaxed);
+    return NVFP4_OK;
+}
+
+nvfp4_status check_tensor(const nvfp4_tensor *t) {
+    if (t == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (t->rows < 0 || t->cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (t->sf_layout != NVFP4_SF_SWIZZLED_128x4 && t->sf_layout != NVFP4_SF_LINEAR)
+        return NVFP4_ERR_INVALID_ARG;
+    if (t->cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (t->global == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(t->global) & 3u) != 0) return NVFP4_ERR_ALIGNMENT;
+    if (t->rows > 0 && t->cols > 0) {
+        if (t->codes == nullptr || t->scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(t->codes) || !aligned16(t->scales)) return NVFP4_ERR_ALIGNMENT;
+    }
+    return NVFP4_OK;
+}
+
+nvfp4_status check_workspace(void *ws, size_t bytes, size_t need) {
+    if (ws == nullptr || bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGNMENT;
+    return NVFP4_OK;
+}
+
+// ---------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+nvfp4_status get_encode() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// Packed-code matrix [rows x cols/2 bytes] as a 2-D uint8 tensor, boxes of
+// 128 bytes x box_rows, 128-byte swizzle (the MMA's K-major operand layout).
+nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, int64_t cols,
+                              uint32_t box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)(cols / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
+    cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32_t *gather,
+                        const nvfp4_tensor *out, int32_t global_supplied, void *ws,
+                        cudaStream_t stream, int sms) {
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kStatusBytes);
+    int n_partials = 0;
+    if (!global_supplied) {
+        int64_t warps_needed = ceil_div(out->rows, 1);
+        int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(warps_needed, 8), 4 * sms),
+                                          kMaxPartials);
+        if (grid < 1) grid = 1;
+        k_amax<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), ld, out->rows,
+                                         out->cols, gather, src_rows, partials, status);
+        nvfp4_status st = launched(cudaGetLastError());
+        if (st != NVFP4_OK) return st;
+        n_partials = grid;
+    }
+    EncodeParams p;
+    p.x = static_cast<const uint16_t *>(x);
+    p.ld = ld;
+    p.rows = out->rows;
+    p.cols = out->cols;
+    p.gather = gather;
+    p.src_rows = src_rows;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = out->global;
+    p.global_supplied = global_supplied;
+    p.partials = partials;
+    p.n_partials = n_partials;
+    p.status = status;
+    const int64_t tasks = ceil_div(out->rows, 128) * ceil_div(out->cols, 64);
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    if (grid < 1) grid = 1;
+    k_encode<<<grid, 256, 0, stream>>>(p);
+    return launched(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return (size_t)(rows * (cols / 2));
+}
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout) {
+    if (rows < 0 || cols < 0) return 0;
+    const int64_t s = cols / 16;
+    if (sf_layout == NVFP4_SF_LINEAR) return (size_t)(rows * s);
+    return (size_t)(ceil_div(rows, 128) * 128 * ceil_div(s, 4) * 4);
+}
+
+size_t nvfp4_workspace_bytes(int32_t op, int64_t, int64_t, int64_t, int32_t) {
+    switch (op) {
+        case NVFP4_OP_QUANTIZE:
+        case NVFP4_OP_QUANTIZE_GATHER:
+            return kStatusBytes + 4 * kMaxPartials;
+        default:
+            return kStatusBytes;
+    }
+}
+
+nvfp4_status nvfp4_quantize(const void *x, int64_t ld, const nvfp4_tensor *out,
+                            int32_t global_supplied, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    if (out->rows > 0 && out->cols > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < out->cols) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return run_encode(x, ld, out->rows, nullptr, out, global_supplied, workspace,
+                      static_cast<cudaStream_t>(stream), sms);
+}
+
+nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
+                                   const int32_t *d_gather, const nvfp4_tensor *out,
+                                   int32_t global_supplied, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    if (src_rows < 0) return NVFP4_ERR_INVALID_ARG;
+    if (out->rows > 0 && out->cols > 0) {
+        if (x == nullptr || d_gather == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < out->cols) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_GATHER, out->rows, out->cols, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return run_encode(x, ld, src_rows, d_gather, out, global_supplied, workspace,
+                      static_cast<cudaStream_t>(stream), sms);
+}
+
+nvfp4_status nvfp4_global_scale(const void *x, int64_t ld, int64_t rows, int64_t cols,
+                                float *d_global, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    if (rows < 0 || cols < 0 || d_global == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(d_global) & 3u) != 0) return NVFP4_ERR_ALIGNMENT;
+    if (rows > 0 && cols > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < cols) return NVFP4_ERR_SHAPE;
+    }
+    nvfp4_status st = check_workspace(workspace, workspace_bytes,
+                                      nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, cols, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
+    uint32_t *partials =
+        reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(rows, 8), 4 * sms), kMaxPartials);
+    if (grid < 1) grid = 1;
+    k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(x), ld, rows, cols, nullptr, rows,
+                                partials, status);
+    st = launched(cudaGetLastError());
+    if (st != NVFP4_OK) return st;
+    k_finalize_g<<<1, 256, 0, s>>>(partials, grid, d_global, status);
+    return launched(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void *stream) {
+    nvfp4_status st = check_tensor(in);
+    if (st != NVFP4_OK) return st;
+    if (in->rows > 0 && in->cols > 0) {
+        if (y == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(y) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < in->cols) return NVFP4_ERR_SHAPE;
+    }
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    if (in->rows == 0 || in->cols == 0) return NVFP4_OK;
+    DequantParams p;
+    p.codes = static_cast<const uint8_t *>(in->codes);
+    p.scales = static_cast<const uint8_t *>(in->scales);
+    p.layout = in->sf_layout;
+    p.global = in->global;
+    p.rows = in->rows;
+    p.cols = in->cols;
+    p.y = static_cast<uint16_t *>(y);
+    p.ld = ld;
+    const int64_t tasks = ceil_div(in->rows, 128) * ceil_div(in->cols, 64);
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    if (grid < 1) grid = 1;
+    k_dequantize<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
+static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
+                                const int32_t *d_group_rows, const nvfp4_tensor *A,
+                                const nvfp4_tensor *W, const float *gw, int64_t n, void *D,
+                                int64_t ldd, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    nvfp4_status st = check_tensor(A);
+    if (st != NVFP4_OK) return st;
+    st = check_tensor(W);
+    if (st != NVFP4_OK) return st;
+    if (A->sf_layout != NVFP4_SF_SWIZZLED_128x4 || W->sf_layout != NVFP4_SF_SWIZZLED_128x4)
+        return NVFP4_ERR_INVALID_ARG;
+    const int64_t k = A->cols;
+    if (W->cols != k || k <= 0 || k % 64 != 0) return NVFP4_ERR_SHAPE;
+    if (A->rows > INT32_MAX || W->rows > INT32_MAX || k > INT32_MAX) return NVFP4_ERR_SHAPE;
+    if (groups > 0) {
+        if (groups > kMaxGroups || d_slot_offsets == nullptr || d_group_rows == nullptr ||
+            gw == nullptr)
+            return NVFP4_ERR_INVALID_ARG;
+        if (n <= 0 || n % 128 != 0 || W->rows != (int64_t)groups * n) return NVFP4_ERR_SHAPE;
+        if (A->rows % 128 != 0) return NVFP4_ERR_SHAPE;
+    }
+    const int64_t m = A->rows;
+    if (m == 0 || n == 0) return NVFP4_OK;
+    if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(D) || ldd % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (ldd < n) return NVFP4_ERR_SHAPE;
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, groups));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    st = get_encode();
+    if (st != NVFP4_OK) return st;
+    CUtensorMap tmA, tmB;
+    st = encode_codes_map(&tmA, A->codes, A->rows, k, kBM);
+    if (st != NVFP4_OK) return st;
+    st = encode_codes_map(&tmB, W->codes, W->rows, k, kBN);
+    if (st != NVFP4_OK) return st;
+
+    GemmParams p;
+    p.sfa = static_cast<const uint8_t *>(A->scales);
+    p.sfb = static_cast<const uint8_t *>(W->scales);
+    p.d = static_cast<uint16_t *>(D);
+    p.ldd = ldd;
+    p.m = (int32_t)m;
+    p.n = (int32_t)n;
+    p.k = (int32_t)k;
+    p.groups = groups;
+    p.slot_offsets = d_slot_offsets;
+    p.group_rows = d_group_rows;
+    p.ga = A->global;
+    p.gw = gw;
+    p.a_row_blocks = (int32_t)ceil_div(A->rows, 128);
+    p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
+    p.status = reinterpret_cast<uint32_t *>(workspace);
+    p.timeout_cycles = g_timeout_cycles;
+    const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, kBN);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, sms));
+    return launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    if (W == nullptr) return NVFP4_ERR_INVALID_ARG;
+    return gemm_common(0, nullptr, nullptr, A, W, W->global, W->rows, D, ldd, workspace,
+                       workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_grouped_gemm(int32_t groups, const int32_t *d_slot_offsets,
+                                const int32_t *d_group_rows, const nvfp4_tensor *A,
+                                const nvfp4_tensor *W, const float *d_w_globals, int64_t n,
+                                void *D, int64_t ldd, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    if (groups <= 0) return NVFP4_ERR_INVALID_ARG;
+    return gemm_common(groups, d_slot_offsets, d_group_rows, A, W, d_w_globals, n, D, ldd,
+                       workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_check_status(void *workspace, void *stream) {
+    if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (v != 0 && cudaMemset(workspace, 0, 4) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return static_cast<nvfp4_status>(v);
+}
+
+const char *nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_ALIGNMENT: return "pointer or pitch not 16-byte aligned";
+        case NVFP4_ERR_SHAPE: return "shape not supported by this call";
+        case NVFP4_ERR_NONFINITE: return "input holds Inf or NaN";
+        case NVFP4_ERR_RANGE: return "tensor amax too small for an FP32 tensor scale";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case NVFP4_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case NVFP4_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+        case NVFP4_ERR_CUDA: return "CUDA call failed";
+    }
+    return "unknown status";
+}
+
+int32_t nvfp4_version(void) { return 100; }
+
+int64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+// Test hook: bound (in SM clock cycles) of every pipeline wait in the GEMM
+// kernels; <= 0 restores the default.  Returns the previous bound.
+long long nvfp4_set_wait_limit_cycles(long long cycles) {
+    long long prev = g_timeout_cycles;
+    g_timeout_cycles = cycles > 0 ? cycles : kDefaultTimeoutCycles;
+    return prev;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// Kernel parameter blocks and launch entry points shared by the host API
+// (api.cu) and the kernel files.  Internal to libnvfp4.so.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+struct EncodeParams {
+    const uint16_t *x;      // BF16 source, row pitch ld elements
+    int64_t ld;
+    int64_t rows, cols;     // output (gathered) shape
+    const int32_t *gather;  // optional row map (output row -> source row, -1 = zero row)
+    int64_t src_rows;       // rows of x (gathered indices must lie below)
+    uint8_t *codes;
+    uint8_t *scales;
+    int32_t layout;         // 0 swizzled 128x4, 1 linear
+    float *global;
+    int32_t global_supplied;
+    const uint32_t *partials;
+    int32_t n_partials;
+    uint32_t *status;
+};
+
+struct DequantParams {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    int32_t layout;
+    const float *global;
+    int64_t rows, cols;
+    uint16_t *y;
+    int64_t ld;
+};
+
+// Block-scaled GEMM tile shape: 128 x 256 output tile, 256 K-values (128
+// bytes of packed codes, one 128-byte swizzle row) per pipeline stage.
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 256;
+constexpr int kStages = 4;
+constexpr int kStageA = kBM * kBK / 2;          // 16 KiB
+constexpr int kStageB = kBN * kBK / 2;          // 32 KiB
+constexpr int kStageSFA = kBM * kBK / 16;       // 2 KiB
+constexpr int kStageSFB = kBN * kBK / 16;       // 4 KiB
+constexpr int kStageBytes = kStageA + kStageB + kStageSFA + kStageSFB;
+constexpr int kMaxGroups = 512;
+constexpr int kGemmThreads = 192;               // producer, MMA, 4 epilogue warps
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ +
+                               2 * (kMaxGroups + 1) * 4 /*group tables*/;
+
+struct GemmParams {
+    const uint8_t *sfa;       // A scales, 128x4 layout
+    const uint8_t *sfb;       // W scales, 128x4 layout
+    uint16_t *d;              // BF16 output
+    int64_t ldd;
+    int32_t m;                // dense: rows of A (and D)
+    int32_t n;                // columns of D (per group when grouped)
+    int32_t k;
+    int32_t groups;           // 0 = dense
+    const int32_t *slot_offsets;  // grouped: groups+1 padded row offsets
+    const int32_t *group_rows;    // grouped: real rows per group
+    const float *ga;          // A tensor scale (device)
+    const float *gw;          // W tensor scale(s) (device), one per group
+    int32_t a_row_blocks;     // ceil(A rows / 128), bounds the grouped slots
+    int32_t b_row_blocks;     // ceil(W rows / 128), bounds the SFB reads
+    uint32_t *status;
+    long long timeout_cycles;
+};
+
+__global__ void k_amax(const uint16_t *x, int64_t ld, int64_t rows, int64_t cols,
+                       const int32_t *gather, int64_t src_rows, uint32_t *partials,
+                       uint32_t *status);
+__global__ void k_finalize_g(const uint32_t *partials, int n, float *global, uint32_t *status);
+__global__ void k_encode(EncodeParams p);
+__global__ void k_dequantize(DequantParams p);
+
+cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                        int grid, cudaStream_t stream);
+
+}  // namespace nvfp4

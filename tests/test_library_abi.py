@@ -1,0 +1,69 @@
+"""CPU checks of the C ABI library: it loads, exports every declared entry
+point, and its size arithmetic matches the storage rules.  No kernel runs."""
+import os
+import re
+
+import pytest
+
+import oracle
+from nvfp4_block_scaled_22_b200 import binding
+from nvfp4_block_scaled_22_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    return set(re.findall(r"NVFP4_API[^;(]*?\b(nvfp4_\w+)\s*\(", src))
+
+
+def test_header_declares_binding_symbols():
+    assert _declared() == set(binding.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {binding.LIB_PATH}").read()
+    exported = set(re.findall(r" T (nvfp4_\w+)", out))
+    assert _declared() <= exported
+
+
+def test_sizes_match_storage_rules(lib):
+    for rows, cols in [(1, 16), (128, 256), (130, 80), (4096, 6144), (131072, 1024)]:
+        assert binding.nvfp4_codes_bytes(rows, cols) == rows * cols // 2
+        for layout in (binding.SF_SWIZZLED, binding.SF_LINEAR):
+            assert binding.nvfp4_scales_bytes(rows, cols, layout) == \
+                oracle.scales_bytes(rows, cols, layout)
+    for op in range(5):
+        assert binding.nvfp4_workspace_bytes(op) >= 16
+
+
+def test_status_strings_and_version(lib):
+    assert binding.nvfp4_status_string(0) == "ok"
+    for s in range(1, 10):
+        assert binding.nvfp4_status_string(s) not in ("", "unknown status")
+    assert lib.nvfp4_version() >= 100
+
+
+def test_host_side_argument_errors_need_no_gpu(lib):
+    """Argument validation returns before any CUDA call."""
+    t = binding.CTensor(0, 0, 0, 4, 24, 0)
+    st = lib.nvfp4_quantize(16, 32, t, 0, 16, 1 << 16, 0)
+    assert st == 3                                  # NVFP4_ERR_SHAPE
+    t = binding.CTensor(16, 16, 0, 4, 32, 0)         # no global pointer
+    assert lib.nvfp4_quantize(16, 32, t, 0, 16, 1 << 16, 0) == 1
+    t = binding.CTensor(16, 16, 16, 4, 32, 7)        # bad layout
+    assert lib.nvfp4_quantize(16, 32, t, 0, 16, 1 << 16, 0) == 1
+    t = binding.CTensor(16, 16, 16, 4, 32, 0)
+    assert lib.nvfp4_quantize(8, 32, t, 0, 16, 1 << 16, 0) == 2   # x misaligned
+    assert lib.nvfp4_quantize(16, 32, t, 0, 16, 8, 0) == 6        # workspace too small
+    a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
+    w = binding.CTensor(16, 16, 16, 256, 96, 0)
+    assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
