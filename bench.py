@@ -298,7 +298,12 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU oracle leg")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the standalone 2^28 quantize measurement")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -343,8 +348,12 @@ def main():
     value = world * flops * args.steps / (total_ms / 1e3) / 1e12
     gemm_tflops = flops / (gemm_avg / 1e3) / 1e12
 
-    sweep_ms, sweep_ms1, sst = time_sweep_quantize(wl.nb, device)
-    e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup)
+    sweep_ms, sweep_ms1, sst = (float("nan"),) * 2 + (0,)
+    if not args.no_sweep:
+        sweep_ms, sweep_ms1, sst = time_sweep_quantize(wl.nb, device)
+    e2e_ms, h2d, d2h = float("nan"), 0, 0
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup)
     if dist is not None:
         t = torch.tensor([sweep_ms, sweep_ms1, e2e_ms], device=device, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

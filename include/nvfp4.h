@@ -172,7 +172,8 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t
  * in NVFP4.)
  * A: M x K, W: N x K (both K-major, i.e. D = A * W^T), both with
  *    NVFP4_SF_SWIZZLED_128x4 scales.  K % 64 == 0; M, N >= 1 arbitrary.
- * D: device BF16 M x N, row pitch ldd >= N (ldd % 8 == 0).
+ * D: device BF16 M x N, row pitch ldd >= N (any; 16-byte aligned D with
+ *    ldd % 8 == 0 takes the vectorised store path).
  * Accuracy: |D - exact| <= 1e-3 * sum_k |a_ik w_jk| / (gA gW) + BF16 rounding. */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,
                         void *workspace, size_t workspace_bytes, void *stream);

@@ -105,7 +105,7 @@ nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, i
                               uint32_t box_rows) {
     cuuint64_t dims[2] = {(cuuint64_t)(cols / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)(kBK / 2), box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)(kBoxK / 2), box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -306,7 +306,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     const int64_t m = A->rows;
     if (m == 0 || n == 0) return NVFP4_OK;
     if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(D) || ldd % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(D) & 1u) != 0) return NVFP4_ERR_ALIGNMENT;
     if (ldd < n) return NVFP4_ERR_SHAPE;
     st = check_workspace(workspace, workspace_bytes,
                          nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, groups));
@@ -327,6 +327,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.sfb = static_cast<const uint8_t *>(W->scales);
     p.d = static_cast<uint16_t *>(D);
     p.ldd = ldd;
+    p.d_vec16 = (aligned16(D) && ldd % 8 == 0) ? 1 : 0;
     p.m = (int32_t)m;
     p.n = (int32_t)n;
     p.k = (int32_t)k;

@@ -10,17 +10,29 @@
 // shrank GLM-5.2 to 4 bits" (section 1, weights and activations in NVFP4;
 // section 2, 256 experts with 8 active per token).
 //
-// Design (one persistent CTA per SM, 6 warps):
-//   warp 0   TMA producer: per stage a 128x256 A box and a 256x256 W box of
-//            packed codes (128-byte swizzle) plus the matching 128x4 scale
-//            tiles by bulk copy, all completing on one mbarrier.
-//   warp 1   MMA issuer: copies the stage's scales into TMEM (tcgen05.cp)
-//            and issues tcgen05.mma kind::mxf4nvf4 (M128 N256 K64, E4M3
-//            scale per 16) into a 128x256 FP32 accumulator in TMEM; commits
-//            free the stage and, after the last K step, signal the epilogue.
-//   warps 2-5 epilogue: tcgen05.ld the accumulator (each warp its 32-lane
-//            quarter), scale by alpha, round to BF16, store with row/column
-//            masks, then hand the accumulator back.
+// Design (one persistent CTA per SM, 14 warps, 4-stage ring of 256 K-values):
+//   warp 0     TMA producer: per stage a 128x128-byte A box and a 256x128-byte
+//              W box of packed codes (128-byte swizzle) on `tma_ready`, and
+//              the matching 512-byte 128x4 scale tiles by bulk copy on
+//              `sf_landed`.
+//   warps 2-5  scale writers, one per 32-lane TMEM quarter.  The tensor core
+//              reads block scales from TMEM, and tcgen05.cp spends
+//              tensor-pipe time on every instruction, so these warps read
+//              their rows of the scale tiles from shared memory and write the
+//              MMA's scale layout into TMEM with tcgen05.st.  They also wait
+//              for the stage's codes, and signal `pair_ready` once for every
+//              two stages, so the MMA issuer synchronises once per eight MMAs
+//              (a completed mbarrier wait costs the issuing thread about as
+//              long as one MMA).
+//   warp 1     MMA issuer: tcgen05.mma kind::mxf4nvf4 (M128 N256 K64, E4M3
+//              scale per 16 values) into a 128x256 FP32 accumulator in TMEM;
+//              a commit per stage frees it (and its TMEM scale columns), and
+//              a commit after the last K step of a tile wakes the epilogue.
+//   warps 6-13 epilogue: two warps per TMEM lane quarter, 128 columns each;
+//              tcgen05.ld the accumulator, scale by alpha, round to BF16 in
+//              registers, hand the accumulator back at once, then store with
+//              row/column masks while the next tile's main loop runs.  One
+//              of them also warms L2 with the next tile's W operand.
 // The grouped variant walks (group, M tile, N tile) with the group taken
 // from the device-side slot offsets, so no host synchronisation is needed.
 // Every mbarrier wait is bounded; a timeout records NVFP4_ERR_TIMEOUT, stops
@@ -38,15 +50,19 @@ namespace {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kBN;          // 256 FP32 columns
-constexpr uint32_t kSfCols = 48;            // per buffer: 16 (A) + 32 (W)
+constexpr uint32_t kSfCols = 48;            // per stage: 4 K blocks x (4 A + 8 W) columns
+constexpr int kFirstEpiWarp = 2 + kSfWarps;
 // tcgen05.mma instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1),
 // K-major, N = 256 (>> 3), UE4M3 scales (bit 23 = 0), M = 128 (>> 4).
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
+constexpr long long kDrainCycles = 2000000000ll;
 
 struct Shared {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t tma_ready[kStages];  // packed codes of the stage landed (tx)
+    uint64_t sf_landed[kStages];  // scale tiles of the stage landed (tx)
+    uint64_t pair_ready[2];       // both stages of a pair loaded, scales in TMEM
+    uint64_t empty[kStages];      // MMAs of the stage done (commit)
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -91,13 +107,17 @@ __device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, const GemmPa
             int mid = (lo + hi + 1) >> 1;
             if (s_off[mid] <= t.a_row0) lo = mid; else hi = mid - 1;
         }
-        // skip empty slots that share the same offset
-        while (lo + 1 < p.groups && s_off[lo + 1] <= t.a_row0) ++lo;
         t.group = lo;
         t.b_row0 = lo * p.n + t.nt * kBN;
         t.row_end = s_off[lo] + s_rows[lo];
     }
     return t;
+}
+
+// Ragged or unaligned output columns: element stores (kept out of line so
+// the common full-tile path holds its 64 packed words in registers).
+__device__ __noinline__ void store_ragged(uint16_t *drow, const uint32_t *o, int ncol) {
+    for (int i = 0; i < ncol; ++i) drow[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
 }
 
 }  // namespace
@@ -109,7 +129,7 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Shared *sh = reinterpret_cast<Shared *>(smem + kStages * kStageBytes);
-    int *s_off = reinterpret_cast<int *>(smem + kStages * kStageBytes + 512);
+    int *s_off = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(sh) + 512);
     int *s_rows = s_off + (kMaxGroups + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -117,11 +137,13 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sh->full[s], 1);
+            mbar_init(&sh->tma_ready[s], 1);
+            mbar_init(&sh->sf_landed[s], 1);
             mbar_init(&sh->empty[s], 1);
         }
+        for (int j = 0; j < 2; ++j) mbar_init(&sh->pair_ready[j], kSfWarps);
         mbar_init(&sh->acc_full, 1);
-        mbar_init(&sh->acc_empty, 4);
+        mbar_init(&sh->acc_empty, kEpiWarps);
         mbar_init(&sh->drain, 1);
         sh->abort_flag = 0;
         fence_barrier_init();
@@ -159,8 +181,11 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int ntiles = (p.n + kBN - 1) / kBN;
     const int tiles = mtiles * ntiles;
     const int kblocks = p.k / 64;                    // 64-value MMA steps
-    const int ktiles = (kblocks + 3) / 4;
+    const int ktiles = (kblocks + 3) / 4;            // 256-value stages
     const int64_t sf_rowblock_bytes = (int64_t)kblocks * 512;   // one 128-row band
+    const int my_tiles =
+        (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total_k = my_tiles * ktiles;           // stages this CTA runs, in order
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -184,18 +209,18 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     uint8_t *sB = sA + kStageA;
                     uint8_t *sSFA = sB + kStageB;
                     uint8_t *sSFB = sSFA + kStageSFA;
-                    mbar_arrive_expect_tx(&sh->full[stage],
-                                          kStageA + kStageB + sf_bytes * (1 + halves));
+                    mbar_arrive_expect_tx(&sh->tma_ready[stage], kStageA + kStageB);
+                    mbar_arrive_expect_tx(&sh->sf_landed[stage], sf_bytes * (1 + halves));
                     armed[stage] = true;
                     armed_phase[stage] = phase;
-                    tma_load_2d(sA, &tmA, &sh->full[stage], kt * (kBK / 2), t.a_row0);
-                    tma_load_2d(sB, &tmB, &sh->full[stage], kt * (kBK / 2), t.b_row0);
                     bulk_load(sSFA, p.sfa + sfa_base + (int64_t)kt * 2048, sf_bytes,
-                              &sh->full[stage]);
+                              &sh->sf_landed[stage]);
                     for (int h = 0; h < halves; ++h)
                         bulk_load(sSFB + h * 2048,
                                   p.sfb + (int64_t)(brb + h) * sf_rowblock_bytes + (int64_t)kt * 2048,
-                                  sf_bytes, &sh->full[stage]);
+                                  sf_bytes, &sh->sf_landed[stage]);
+                    tma_load_2d(sA, &tmA, &sh->tma_ready[stage], kt * (kBK / 2), t.a_row0);
+                    tma_load_2d(sB, &tmB, &sh->tma_ready[stage], kt * (kBK / 2), t.b_row0);
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
             }
@@ -204,98 +229,160 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 for (int s = 0; s < kStages; ++s) {
                     if (!armed[s]) continue;
                     const long long t0 = clock64();
-                    while (!mbar_try_wait(&sh->full[s], armed_phase[s]) &&
-                           clock64() - t0 < 2000000000ll) {
+                    while (!mbar_try_wait(&sh->sf_landed[s], armed_phase[s]) &&
+                           clock64() - t0 < kDrainCycles) {
+                    }
+                    while (!mbar_try_wait(&sh->tma_ready[s], armed_phase[s]) &&
+                           clock64() - t0 < kDrainCycles) {
                     }
                 }
             }
+        }
+    } else if (warp >= 2 && warp < kFirstEpiWarp) {
+        // -------------------------------------------------- scale writers
+        // TMEM scale columns of stage s start at kAccCols + s * kSfCols: A at
+        // +4*kb (K block kb), W at +16+8*kb.  Lane i of every 32-lane quarter
+        // holds, in column c, the four scales of row 32c+i: exactly row i of
+        // the 512-byte 128x4 scale tile (16 bytes = four columns).  Every
+        // quarter needs the full set, so each writer warp stores all 48
+        // columns of its own 32 lanes.
+        const int quarter = warp & 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int g = 0; g < total_k; ++g) {
+            if (!wait_or_abort(&sh->sf_landed[stage], phase, sh, p)) break;
+            const uint8_t *sSFA = smem + stage * kStageBytes + kStageA + kStageB;
+            const uint8_t *sSFB = sSFA + kStageSFA;
+            const uint32_t col = lane_base + kAccCols + (uint32_t)stage * kSfCols;
+            uint32_t v[16];
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(sSFA + 512 * kb + 16 * lane);
+                v[4 * kb] = w.x; v[4 * kb + 1] = w.y; v[4 * kb + 2] = w.z; v[4 * kb + 3] = w.w;
+            }
+            tmem_st_32x32b_x16(col, v);
+            uint32_t u[32];
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(sSFB + 2048 * h + 512 * kb + 16 * lane);
+                    const int o = 8 * kb + 4 * h;
+                    u[o] = w.x; u[o + 1] = w.y; u[o + 2] = w.z; u[o + 3] = w.w;
+                }
+            }
+            tmem_st_32x32b_x32(col + 16, u);
+            if (!wait_or_abort(&sh->tma_ready[stage], phase, sh, p)) break;
+            if ((g & 1) || g == total_k - 1) {
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                const int pj = g >> 1;
+                if (lane == 0) mbar_arrive(&sh->pair_ready[pj & 1]);
+            }
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0, kiter = 0;
+            // Descriptors are linear in the start address (field = address >> 4),
+            // so stage s and K block kb are plain additions to the stage-0 value.
+            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(smem_u32(smem) + kStageA, 16, 1024, 2);
+            static_assert(kStageBytes % 16 == 0, "stage stride must be 16-byte granular");
+            uint32_t acc_phase = 0;
             bool ok = true;
-            const uint32_t sf_lbo = 0, sf_sbo = 128;    // 8-row x 16-byte core matrices
-            for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-                if (!wait_or_abort(&sh->acc_empty, acc_phase ^ 1, sh, p)) { ok = false; break; }
-                tc_fence_after();
-                for (int kt = 0; kt < ktiles; ++kt) {
-                    if (!wait_or_abort(&sh->full[stage], phase, sh, p)) { ok = false; break; }
+            for (int g = 0; ok && g < total_k; ++g) {
+                const int stage = g & (kStages - 1);
+                const int kt = g % ktiles;
+                if ((g & 1) == 0) {
+                    const int pj = g >> 1;
+                    if (!wait_or_abort(&sh->pair_ready[pj & 1], (uint32_t)(pj >> 1) & 1u, sh, p)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const int nkb = min(4, kblocks - 4 * kt);
-                    const uint32_t sA = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t sB = sA + kStageA;
-                    const uint32_t sSFA = sB + kStageB;
-                    const uint32_t sSFB = sSFA + kStageSFA;
-                    const uint32_t sfa_col = kAccCols + (kiter & 1) * kSfCols;
-                    const uint32_t sfb_col = sfa_col + 16;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        tc_cp_32x128b_x4(tmem + sfa_col + 4 * kb,
-                                         smem_desc(sSFA + 512 * kb, sf_lbo, sf_sbo, 0));
-                        tc_cp_32x128b_x4(tmem + sfb_col + 8 * kb,
-                                         smem_desc(sSFB + 512 * kb, sf_lbo, sf_sbo, 0));
-                        tc_cp_32x128b_x4(tmem + sfb_col + 8 * kb + 4,
-                                         smem_desc(sSFB + 2048 + 512 * kb, sf_lbo, sf_sbo, 0));
-                    }
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        const uint64_t ad = smem_desc(sA + 32 * kb, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(sB + 32 * kb, 16, 1024, 2);
-                        mma_nvf4(tmem, ad, bd, kIdesc, tmem + sfa_col + 4 * kb,
-                                 tmem + sfb_col + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
-                    }
-                    tc_commit(&sh->empty[stage]);
-                    ++kiter;
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
-                if (!ok) break;
-                tc_commit(&sh->acc_full);
-                acc_phase ^= 1;
+                if (kt == 0) {   // first stage of a tile: the accumulator must be free
+                    if (!wait_or_abort(&sh->acc_empty, acc_phase ^ 1, sh, p)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                const int nkb = min(4, kblocks - 4 * kt);
+                const uint32_t sfa = tmem + kAccCols + (uint32_t)stage * kSfCols;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    if (kb < nkb) {
+                        const uint64_t off = (uint64_t)(stage * (kStageBytes / 16) + 2 * kb);
+                        mma_nvf4(tmem, adesc0 + off, bdesc0 + off, kIdesc, sfa + 4 * kb,
+                                 sfa + 16 + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
+                    }
+                }
+                tc_commit(&sh->empty[stage]);
+                if (kt == ktiles - 1) {
+                    tc_commit(&sh->acc_full);
+                    acc_phase ^= 1;
+                }
             }
-            // Wait for every issued MMA/copy before TMEM can be released.
+            // Wait for every issued MMA before TMEM can be released.
             tc_commit(&sh->drain);
             const long long t0 = clock64();
-            while (!mbar_try_wait(&sh->drain, 0) && clock64() - t0 < 2000000000ll) {
+            while (!mbar_try_wait(&sh->drain, 0) && clock64() - t0 < kDrainCycles) {
             }
         }
     } else {
         // ------------------------------------------------------ epilogue
-        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int quarter = warp & 3;                          // TMEM lane quarter
+        const int chalf = (warp - kFirstEpiWarp) / 4;          // column half of the tile
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const TileInfo t = tile_info(tile, mtiles, p, s_off, s_rows);
             if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
-            const float gw = p.gw[t.group];
-            const float alpha = __frcp_rn(__fmul_rn(*p.ga, gw));
-            const int row = t.a_row0 + quarter * 32 + lane;
-            const bool row_ok = row < t.row_end;
-            uint16_t *drow = p.d + (int64_t)row * p.ldd;
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
+            const float alpha = __frcp_rn(__fmul_rn(*p.ga, p.gw[t.group]));
+            uint32_t o[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, r);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                       (uint32_t)(chalf * 128 + 32 * c), r);
                 tmem_ld_wait();
-                const int col = t.nt * kBN + c0;
-                if (!row_ok || col >= p.n) continue;
-                uint32_t o[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    o[i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                           __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
-                if (col + 32 <= p.n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(drow + col);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                } else {
-                    for (int i = 0; i < 32 && col + i < p.n; ++i)
-                        drow[col + i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
-                }
+                    o[16 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                    __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh->acc_empty);
+            if (lane == 0) mbar_arrive(&sh->acc_empty);    // accumulator free for the next tile
             acc_phase ^= 1;
+
+            if (warp == kFirstEpiWarp && lane == 0) {
+                // Warm L2 with the W rows (codes and scales) of this CTA's next tile.
+                const int next = tile + (int)gridDim.x;
+                if (next < tiles) {
+                    const TileInfo u = tile_info(next, mtiles, p, s_off, s_rows);
+                    for (int x = 0; x < p.k / 2; x += kBoxK / 2) tma_prefetch_l2_2d(&tmB, x, u.b_row0);
+                    const int ubrb = u.b_row0 / kBM;
+                    for (int h = 0; h < 2 && ubrb + h < p.b_row_blocks; ++h)
+                        bulk_prefetch_l2(p.sfb + (int64_t)(ubrb + h) * sf_rowblock_bytes,
+                                         (uint32_t)sf_rowblock_bytes);
+                }
+            }
+
+            const int row = t.a_row0 + quarter * 32 + lane;
+            const int col0 = t.nt * kBN + chalf * 128;
+            if (row < t.row_end && col0 < p.n) {
+                uint16_t *drow = p.d + (int64_t)row * p.ldd + col0;
+                if (p.d_vec16 && col0 + 128 <= p.n) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(drow);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                } else {
+                    store_ragged(drow, o, min(128, p.n - col0));
+                }
+            }
         }
     }
 

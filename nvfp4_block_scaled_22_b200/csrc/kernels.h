@@ -33,19 +33,23 @@ struct DequantParams {
     int64_t ld;
 };
 
-// Block-scaled GEMM tile shape: 128 x 256 output tile, 256 K-values (128
-// bytes of packed codes, one 128-byte swizzle row) per pipeline stage.
+// Block-scaled GEMM tiling: 128 x 256 output tile; each pipeline stage
+// holds 256 K-values (one 128-byte swizzle column of packed codes).  The
+// MMA issuer takes stages in pairs, synchronising once per eight MMAs.
 constexpr int kBM = 128;
 constexpr int kBN = 256;
-constexpr int kBK = 256;
+constexpr int kBK = 256;                         // K values per stage
+constexpr int kBoxK = 256;                       // K values per TMA box (128 bytes)
 constexpr int kStages = 4;
-constexpr int kStageA = kBM * kBK / 2;          // 16 KiB
-constexpr int kStageB = kBN * kBK / 2;          // 32 KiB
-constexpr int kStageSFA = kBM * kBK / 16;       // 2 KiB
-constexpr int kStageSFB = kBN * kBK / 16;       // 4 KiB
+constexpr int kStageA = kBM * kBK / 2;           // 16 KiB
+constexpr int kStageB = kBN * kBK / 2;           // 32 KiB
+constexpr int kStageSFA = kBM * kBK / 16;        // 2 KiB: four 512-byte 128x4 scale tiles
+constexpr int kStageSFB = kBN * kBK / 16;        // 4 KiB: two 128-row bands
 constexpr int kStageBytes = kStageA + kStageB + kStageSFA + kStageSFB;
+constexpr int kSfWarps = 4;                      // write block scales into TMEM
+constexpr int kEpiWarps = 8;                     // two per TMEM lane quarter
 constexpr int kMaxGroups = 512;
-constexpr int kGemmThreads = 192;               // producer, MMA, 4 epilogue warps
+constexpr int kGemmThreads = 32 * (2 + kSfWarps + kEpiWarps);   // 448
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ +
                                2 * (kMaxGroups + 1) * 4 /*group tables*/;
 
@@ -54,6 +58,7 @@ struct GemmParams {
     const uint8_t *sfb;       // W scales, 128x4 layout
     uint16_t *d;              // BF16 output
     int64_t ldd;
+    int32_t d_vec16;          // 1: D and ldd allow 16-byte stores
     int32_t m;                // dense: rows of A (and D)
     int32_t n;                // columns of D (per group when grouped)
     int32_t k;

@@ -28,8 +28,9 @@ def _lib():
 def _rand(rows, cols, seed, scale=1.0):
     g = torch.Generator().manual_seed(seed)
     x = torch.randn(rows, cols, generator=g) * scale
-    idx = torch.randint(0, x.numel(), (max(1, x.numel() // 200),), generator=g)
-    x.view(-1)[idx] *= 30
+    if x.numel():
+        idx = torch.randint(0, x.numel(), (max(1, x.numel() // 200),), generator=g)
+        x.view(-1)[idx] *= 30
     return x.to(torch.bfloat16)
 
 
