@@ -220,6 +220,13 @@ NVFP4_API int64_t nvfp4_launch_count(void);
  * Meant for tests of the timeout path. */
 NVFP4_API long long nvfp4_set_wait_limit_cycles(long long cycles);
 
+/* Dense nvfp4_gemm calls with M >= 256 run on pairs of SMs sharing 256x256
+ * output tiles (less operand traffic from L2 per FLOP); smaller M and the
+ * grouped GEMM use one SM per 128x256 tile.  enable = 0 sends every dense
+ * call to the single-SM kernel (both give results within the same bound;
+ * used by tests to cover both).  Returns the previous setting. */
+NVFP4_API int32_t nvfp4_set_gemm_pairs(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ EXPORTED = (
     "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
-    "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles",
+    "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
 )
 
 
@@ -77,6 +77,7 @@ def lib() -> C.CDLL:
             "nvfp4_version": (i32, []),
             "nvfp4_launch_count": (i64, []),
             "nvfp4_set_wait_limit_cycles": (C.c_longlong, [C.c_longlong]),
+            "nvfp4_set_gemm_pairs": (i32, [i32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -275,3 +276,7 @@ def nvfp4_launch_count() -> int:
 
 def nvfp4_set_wait_limit_cycles(cycles: int) -> int:
     return int(lib().nvfp4_set_wait_limit_cycles(cycles))
+
+
+def nvfp4_set_gemm_pairs(enable: bool) -> bool:
+    return bool(lib().nvfp4_set_gemm_pairs(int(enable)))

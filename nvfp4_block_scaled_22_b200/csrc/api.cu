@@ -32,6 +32,7 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 long long g_timeout_cycles = kDefaultTimeoutCycles;
+bool g_use_pairs = true;
 
 nvfp4_status current_device(int *sms) {
     int dev = 0;
@@ -316,10 +317,11 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     if (st != NVFP4_OK) return st;
     st = get_encode();
     if (st != NVFP4_OK) return st;
+    const bool pair = groups == 0 && m >= kPairMinRows && sms >= 2 && g_use_pairs;
     CUtensorMap tmA, tmB;
     st = encode_codes_map(&tmA, A->codes, A->rows, k, kBM);
     if (st != NVFP4_OK) return st;
-    st = encode_codes_map(&tmB, W->codes, W->rows, k, kBN);
+    st = encode_codes_map(&tmB, W->codes, W->rows, k, pair ? 128 : kBN);
     if (st != NVFP4_OK) return st;
 
     GemmParams p;
@@ -340,6 +342,11 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
     p.status = reinterpret_cast<uint32_t *>(workspace);
     p.timeout_cycles = g_timeout_cycles;
+    if (pair) {
+        const int64_t pair_tiles = ceil_div(m, 256) * ceil_div(n, 256);
+        const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tiles, sms / 2));
+        return launched(launch_gemm_pair(tmA, tmB, p, clusters, static_cast<cudaStream_t>(stream)));
+    }
     const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, kBN);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, sms));
     return launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream)));
@@ -397,6 +404,14 @@ int64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_rela
 long long nvfp4_set_wait_limit_cycles(long long cycles) {
     long long prev = g_timeout_cycles;
     g_timeout_cycles = cycles > 0 ? cycles : kDefaultTimeoutCycles;
+    return prev;
+}
+
+// Test hook: route dense GEMMs of >= 256 rows to CTA pairs (1, default) or
+// to the single-CTA kernel (0).  Returns the previous setting.
+int32_t nvfp4_set_gemm_pairs(int32_t enable) {
+    const int32_t prev = g_use_pairs ? 1 : 0;
+    g_use_pairs = enable != 0;
     return prev;
 }
 

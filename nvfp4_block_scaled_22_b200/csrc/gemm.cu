@@ -72,7 +72,7 @@ struct Shared {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Shared *sh,
                                               const GemmParams &p) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -114,11 +114,6 @@ __device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, const GemmPa
     return t;
 }
 
-// Ragged or unaligned output columns: element stores (kept out of line so
-// the common full-tile path holds its 64 packed words in registers).
-__device__ __noinline__ void store_ragged(uint16_t *drow, const uint32_t *o, int ncol) {
-    for (int i = 0; i < ncol; ++i) drow[i] = (uint16_t)(o[i >> 1] >> (16 * (i & 1)));
-}
 
 }  // namespace
 
@@ -291,37 +286,51 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
             const uint64_t bdesc0 = smem_desc(smem_u32(smem) + kStageA, 16, 1024, 2);
             static_assert(kStageBytes % 16 == 0, "stage stride must be 16-byte granular");
+            // The tensor pipe queues very few MMAs, so everything between two
+            // MMA issues is on the critical path: per-stage bookkeeping below
+            // is incremental (no divisions), and the MMA waits once per pair.
+            const int last_nkb = kblocks - 4 * (ktiles - 1);
             uint32_t acc_phase = 0;
-            bool ok = true;
-            for (int g = 0; ok && g < total_k; ++g) {
-                const int stage = g & (kStages - 1);
-                const int kt = g % ktiles;
+            int stage = 0, kt = 0;
+            uint32_t stage_off = 0;                       // stage * kStageBytes / 16
+            uint32_t sfa = tmem + kAccCols;               // stage's TMEM scale columns
+            for (int g = 0; g < total_k; ++g) {
                 if ((g & 1) == 0) {
                     const int pj = g >> 1;
-                    if (!wait_or_abort(&sh->pair_ready[pj & 1], (uint32_t)(pj >> 1) & 1u, sh, p)) {
-                        ok = false;
+                    if (!wait_or_abort(&sh->pair_ready[pj & 1], (uint32_t)(pj >> 1) & 1u, sh, p))
                         break;
-                    }
                     tc_fence_after();
                 }
                 if (kt == 0) {   // first stage of a tile: the accumulator must be free
-                    if (!wait_or_abort(&sh->acc_empty, acc_phase ^ 1, sh, p)) { ok = false; break; }
+                    if (!wait_or_abort(&sh->acc_empty, acc_phase ^ 1, sh, p)) break;
                     tc_fence_after();
                 }
-                const int nkb = min(4, kblocks - 4 * kt);
-                const uint32_t sfa = tmem + kAccCols + (uint32_t)stage * kSfCols;
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    if (kb < nkb) {
-                        const uint64_t off = (uint64_t)(stage * (kStageBytes / 16) + 2 * kb);
-                        mma_nvf4(tmem, adesc0 + off, bdesc0 + off, kIdesc, sfa + 4 * kb,
-                                 sfa + 16 + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
-                    }
+                const uint32_t first = kt != 0 ? 1u : 0u;
+                if (kt != ktiles - 1 || last_nkb == 4) {
+                    mma_nvf4(tmem, adesc0 + stage_off, bdesc0 + stage_off, kIdesc, sfa, sfa + 16, first);
+                    mma_nvf4(tmem, adesc0 + stage_off + 2, bdesc0 + stage_off + 2, kIdesc, sfa + 4, sfa + 24, 1u);
+                    mma_nvf4(tmem, adesc0 + stage_off + 4, bdesc0 + stage_off + 4, kIdesc, sfa + 8, sfa + 32, 1u);
+                    mma_nvf4(tmem, adesc0 + stage_off + 6, bdesc0 + stage_off + 6, kIdesc, sfa + 12, sfa + 40, 1u);
+                } else {
+                    for (int kb = 0; kb < last_nkb; ++kb)
+                        mma_nvf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb, kIdesc,
+                                 sfa + 4 * kb, sfa + 16 + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
                 }
                 tc_commit(&sh->empty[stage]);
                 if (kt == ktiles - 1) {
                     tc_commit(&sh->acc_full);
                     acc_phase ^= 1;
+                    kt = 0;
+                } else {
+                    ++kt;
+                }
+                if (++stage == kStages) {
+                    stage = 0;
+                    stage_off = 0;
+                    sfa = tmem + kAccCols;
+                } else {
+                    stage_off += kStageBytes / 16;
+                    sfa += kSfCols;
                 }
             }
             // Wait for every issued MMA before TMEM can be released.
@@ -370,19 +379,13 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 }
             }
 
-            const int row = t.a_row0 + quarter * 32 + lane;
+            // One warp stores its 32 rows x 128 columns; a register transpose
+            // makes every store instruction cover one row's 128 bytes.
+            const int row0 = t.a_row0 + quarter * 32;
             const int col0 = t.nt * kBN + chalf * 128;
-            if (row < t.row_end && col0 < p.n) {
-                uint16_t *drow = p.d + (int64_t)row * p.ldd + col0;
-                if (p.d_vec16 && col0 + 128 <= p.n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(drow);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                } else {
-                    store_ragged(drow, o, min(128, p.n - col0));
-                }
-            }
+            if (row0 < t.row_end && col0 < p.n)
+                store_rows_coalesced(o, p.d + (int64_t)row0 * p.ldd + col0, p.ldd,
+                                     t.row_end - row0, min(128, p.n - col0), p.d_vec16 != 0, lane);
         }
     }
 

@@ -83,4 +83,11 @@ __global__ void k_dequantize(DequantParams p);
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t stream);
 
+// Dense GEMM on CTA pairs (256x256 tiles); tmB must use 128-row boxes.
+cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                             int clusters, cudaStream_t stream);
+
+// Dense GEMMs with at least this many rows run on CTA pairs.
+constexpr int64_t kPairMinRows = 256;
+
 }  // namespace nvfp4

@@ -115,6 +115,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of a phase (no suspend): true once it has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // after `limit_cycles` SM clocks (about a second at the default limit) and
 // returns false; the caller records NVFP4_ERR_TIMEOUT and unwinds.
@@ -291,6 +301,143 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const void *desc, int32_t x, 
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
                  :: "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+// ------------------------------------------------------ CTA pairs (2-SM)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Arrive (release, cluster scope) on an mbarrier given by its cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 :: "r"(cluster_addr) : "memory");
+}
+
+// try_wait with cluster-scope acquire, for barriers other CTAs arrive on.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                 :: "r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMA issued by the leader CTA: A rows from each CTA's shared memory
+// (M = 256 across the pair), B rows split by N between the two CTAs, scales
+// and accumulator at the same TMEM columns of both CTAs.
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem,
+                                              uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+           "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Arrive on the mbarrier at the same offset in every CTA of `cta_mask` once
+// all previously issued pair MMAs have finished.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;"
+        :: "r"(smem_u32(bar)), "h"(cta_mask) : "memory");
+}
+
+}  // namespace nvfp4
+
+
+namespace nvfp4 {
+
+// In-register transpose of a 32 x 32 matrix of 32-bit words held one row per
+// lane (lane l holds a[0..31] = row l): afterwards lane l holds column l, i.e.
+// a[r] = original row r, word l.  Five butterfly rounds of 16 shuffles; all
+// register indices are compile-time constants.
+__device__ __forceinline__ void warp_transpose32(uint32_t *a, int lane) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool hi = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if ((i & s) == 0) {
+                const uint32_t send = hi ? a[i] : a[i + s];
+                const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, s);
+                if (hi) a[i] = recv; else a[i + s] = recv;
+            }
+        }
+    }
+}
+
+// Store a warp's 32 rows x 128 BF16 columns (lane l holds row l as 64 packed
+// words) so that every store instruction writes one row's 128 contiguous
+// bytes.  Rows >= rows_left are skipped, columns >= ncol are masked.
+__device__ __forceinline__ void store_rows_coalesced(uint32_t (&o)[64], uint16_t *d, int64_t ldd,
+                                                     int rows_left, int ncol, bool aligned,
+                                                     int lane) {
+    warp_transpose32(o, lane);
+    warp_transpose32(o + 32, lane);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+        const int col = 64 * b + 2 * lane;           // this lane's column pair
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            if (r < rows_left) {
+                uint16_t *p = d + (int64_t)r * ldd + col;
+                const uint32_t w = o[32 * b + r];
+                if (aligned && col + 2 <= ncol) {
+                    *reinterpret_cast<uint32_t *>(p) = w;
+                } else {
+                    if (col < ncol) p[0] = (uint16_t)w;
+                    if (col + 1 < ncol) p[1] = (uint16_t)(w >> 16);
+                }
+            }
+        }
+    }
 }
 
 }  // namespace nvfp4

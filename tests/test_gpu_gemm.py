@@ -64,10 +64,17 @@ def test_tiny_linear():
     _check_full(inputs.tiny_operand("A"), inputs.tiny_operand("W"), "tiny")
 
 
+@pytest.fixture(params=[True, False], ids=["pairs", "single"])
+def pairs(request):
+    prev = nb.nvfp4_set_gemm_pairs(request.param)
+    yield request.param
+    nb.nvfp4_set_gemm_pairs(prev)
+
+
 @pytest.mark.parametrize("m,n,k", [(1, 1, 64), (7, 9, 64), (129, 300, 128), (128, 256, 320),
                                    (300, 513, 1088), (256, 512, 4096), (64, 1000, 256),
-                                   (1, 256, 5120)])
-def test_ragged_shapes(m, n, k):
+                                   (1, 256, 5120), (640, 384, 192), (257, 257, 320)])
+def test_ragged_shapes(m, n, k, pairs):
     _check_full(_rand(m, k, m + 7 * n + k), _rand(n, k, 3 * m + n + k, 0.02), f"{m}x{n}x{k}")
 
 
@@ -109,7 +116,7 @@ def ffn_weight():
 
 
 @pytest.mark.parametrize("m", inputs.FFN_M)
-def test_ffn_linear_full_size(m, ffn_weight):
+def test_ffn_linear_full_size(m, ffn_weight, pairs):
     qw, rw = ffn_weight
     qa, ra = _quant_both(inputs.ffn_activation(m), f"ffn A {m}")
     d = nb.nvfp4_gemm(qa, qw)
