@@ -304,6 +304,8 @@ def main():
                     help="skip the standalone 2^28 quantize measurement")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
+                    help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -324,6 +326,7 @@ def main():
     fp4_peak = bf16_tf * FP4_OVER_BF16
 
     wl = Workload(device)
+    wl.nb.nvfp4_set_gemm_pairs(args.gemm_kernel == "pair")
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -378,7 +381,9 @@ def main():
             "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed (256 MiB write) before every timed step",
-                       "weights": "pre-quantized once, outside the timed region"},
+                       "weights": "pre-quantized once, outside the timed region",
+                       "gemm_kernel": "cta_pair_256x256" if args.gemm_kernel == "pair"
+                       else "single_cta_128x256"},
             "roofline": {"kernel": "k_gemm_nvf4", "bound": "tensor",
                          "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak,

@@ -220,11 +220,12 @@ NVFP4_API int64_t nvfp4_launch_count(void);
  * Meant for tests of the timeout path. */
 NVFP4_API long long nvfp4_set_wait_limit_cycles(long long cycles);
 
-/* Dense nvfp4_gemm calls with M >= 256 run on pairs of SMs sharing 256x256
- * output tiles (less operand traffic from L2 per FLOP); smaller M and the
- * grouped GEMM use one SM per 128x256 tile.  enable = 0 sends every dense
- * call to the single-SM kernel (both give results within the same bound;
- * used by tests to cover both).  Returns the previous setting. */
+/* Kernel choice for dense nvfp4_gemm calls with M >= 256: enable = 1 runs
+ * them on pairs of SMs sharing 256x256 output tiles (half the operand
+ * traffic from L2 per SM), enable = 0 (the default, faster at the measured
+ * shapes) on one SM per 128x256 tile.  Smaller M and the grouped GEMM always
+ * use one SM per tile.  Both give results within the same bound.  Returns
+ * the previous setting. */
 NVFP4_API int32_t nvfp4_set_gemm_pairs(int32_t enable);
 
 #ifdef __cplusplus

@@ -32,7 +32,7 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 long long g_timeout_cycles = kDefaultTimeoutCycles;
-bool g_use_pairs = true;
+bool g_use_pairs = false;
 
 nvfp4_status current_device(int *sms) {
     int dev = 0;
@@ -407,8 +407,9 @@ long long nvfp4_set_wait_limit_cycles(long long cycles) {
     return prev;
 }
 
-// Test hook: route dense GEMMs of >= 256 rows to CTA pairs (1, default) or
-// to the single-CTA kernel (0).  Returns the previous setting.
+// Route dense GEMMs of >= 256 rows to CTA pairs (1) or to the single-CTA
+// kernel (0, default: faster at the measured shapes).  Returns the previous
+// setting.
 int32_t nvfp4_set_gemm_pairs(int32_t enable) {
     const int32_t prev = g_use_pairs ? 1 : 0;
     g_use_pairs = enable != 0;

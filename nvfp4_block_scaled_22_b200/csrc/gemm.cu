@@ -31,8 +31,7 @@
 //   warps 6-13 epilogue: two warps per TMEM lane quarter, 128 columns each;
 //              tcgen05.ld the accumulator, scale by alpha, round to BF16 in
 //              registers, hand the accumulator back at once, then store with
-//              row/column masks while the next tile's main loop runs.  One
-//              of them also warms L2 with the next tile's W operand.
+//              row/column masks while the next tile's main loop runs.
 // The grouped variant walks (group, M tile, N tile) with the group taken
 // from the device-side slot offsets, so no host synchronisation is needed.
 // Every mbarrier wait is bounded; a timeout records NVFP4_ERR_TIMEOUT, stops
@@ -365,19 +364,6 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh->acc_empty);    // accumulator free for the next tile
             acc_phase ^= 1;
-
-            if (warp == kFirstEpiWarp && lane == 0) {
-                // Warm L2 with the W rows (codes and scales) of this CTA's next tile.
-                const int next = tile + (int)gridDim.x;
-                if (next < tiles) {
-                    const TileInfo u = tile_info(next, mtiles, p, s_off, s_rows);
-                    for (int x = 0; x < p.k / 2; x += kBoxK / 2) tma_prefetch_l2_2d(&tmB, x, u.b_row0);
-                    const int ubrb = u.b_row0 / kBM;
-                    for (int h = 0; h < 2 && ubrb + h < p.b_row_blocks; ++h)
-                        bulk_prefetch_l2(p.sfb + (int64_t)(ubrb + h) * sf_rowblock_bytes,
-                                         (uint32_t)sf_rowblock_bytes);
-                }
-            }
 
             // One warp stores its 32 rows x 128 columns; a register transpose
             // makes every store instruction cover one row's 128 bytes.
