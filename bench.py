@@ -41,6 +41,22 @@ L2_FLUSH_BYTES = 256 << 20
 QUANT_BYTES_PER_VALUE_2PASS = 4.5625
 ENCODE_BYTES_PER_VALUE = 2.5625
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
+# DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
+# the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
+# Reported only while the kernel's sources hash to the profiled version.
+GEMM_TRAFFIC_BYTES = 87.4e6 + 293.3e6
+GEMM_TRAFFIC_SRC_SHA = "394c042151ea74c5"
+GEMM_SOURCES = ("gemm.cu", "kernels.h", "ptx.cuh")
+
+
+def gemm_traffic():
+    import hashlib
+    csrc = os.path.join(ROOT, "nvfp4_block_scaled_22_b200", "csrc")
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return GEMM_TRAFFIC_BYTES if h.hexdigest()[:16] == GEMM_TRAFFIC_SRC_SHA else None
 
 
 def env_rank():
@@ -389,7 +405,8 @@ def main():
                          "frac": gemm_tflops / fp4_peak,
                          "peak_source": f"{peak_src} bf16 burst {bf16_tf} TFLOP/s x "
                                         f"{FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
-                         "traffic": None, "ms_per_launch": gemm_avg},
+                         "traffic": gemm_traffic(), "ms_per_launch": gemm_avg,
+                         "algorithmic_flops_per_launch": flops},
             "quantize": {"workload": "quantize sweep, 2^28 BF16 values [65536 x 4096]",
                          "gbs_two_pass": gbs_2pass, "frac_two_pass": gbs_2pass / hbm_gbs,
                          "ms_two_pass": sweep_ms,
