@@ -152,6 +152,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t 
                                    int32_t global_supplied, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* Same quantization as nvfp4_quantize, for callers that cannot allocate
+ * device memory when they quantize: code recorded into a CUDA graph (device
+ * allocation cannot be captured), latency-critical paths that cannot afford
+ * the device synchronisation cudaMalloc implies, and host frameworks whose
+ * memory pool already owns the device.  (The pages have no counterpart to
+ * this entry point; it changes where scratch lives, not what is computed.)
+ * It takes no workspace: its scratch (status word plus up to 1024 per-block
+ * partial maxima, 4352 bytes) is a fixed device array inside the library
+ * that every GPU loading the library keeps until the process exits.  The
+ * scratch does not grow with the tensor, so every size nvfp4_quantize
+ * accepts is accepted here; a launch needing more partial slots than the
+ * array holds would be refused with NVFP4_ERR_WORKSPACE.
+ * - The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ * - All calls share the array and the status word is cleared by every call:
+ *   calls whose kernels can overlap on the GPU (unordered streams) race and
+ *   must not be issued.
+ * - Device-detected errors (non-finite input, amax out of range) are
+ *   reported in band: *out->global is set to NaN.
+ * Arguments and the other return codes are those of nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t ld, const nvfp4_tensor *out,
+                                              int32_t global_supplied, void *stream);
+
 /* ---- dequantize ------------------------------------------------------- */
 
 /* NVFP4 -> BF16:  y = bf16_rne(RN(e2m1(code) * d_b)),  d_b = RN(s_b / g).

@@ -34,6 +34,7 @@ EXPORTED = (
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
+    "nvfp4_quantize_noalloc",
 )
 
 
@@ -78,6 +79,7 @@ def lib() -> C.CDLL:
             "nvfp4_launch_count": (i64, []),
             "nvfp4_set_wait_limit_cycles": (C.c_longlong, [C.c_longlong]),
             "nvfp4_set_gemm_pairs": (i32, [i32]),
+            "nvfp4_quantize_noalloc": (C.c_int, [vp, i64, T, i32, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
