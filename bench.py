@@ -307,6 +307,191 @@ def run_reference(args):
     return 0
 
 
+
+# ------------------------------------------------- other workloads (rows)
+def _events(n):
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(n)]
+
+
+def _timed(fn, steps, warmup, flush=None):
+    """Median device time (ms) of fn() over `steps` runs, optional L2 flush
+    between runs outside the events."""
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        fn()
+    torch.cuda.synchronize()
+    evs = _events(steps)
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
+def workload_line(name, args, device):
+    """Measure one of the other scope rows; returns a JSON-able dict."""
+    from nvfp4_block_scaled_22_b200 import binding as nb
+    from nvfp4_block_scaled_22_b200 import inputs
+    hbm_gbs, bf16_tf, _, peak_src = measured_peaks()
+    fp4_peak = bf16_tf * FP4_OVER_BF16
+    ws = nb.Workspace(device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = flush_buf.zero_
+    line = {"impl": "ours", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "data": "synthetic", "scaling": "weak", "vs_baseline": None}
+
+    if name == "sweep":
+        rows = []
+        for n in inputs.SWEEP_SIZES:
+            x = inputs.sweep_tensor(n, device=device)
+            q = nb.NVFP4Tensor.empty(x.shape[0], x.shape[1], device=device)
+            big = 2 * n > 126e6
+            ms = _timed(lambda: nb.nvfp4_quantize(x, out=q, workspace=ws), args.steps, args.warmup,
+                        None if big else flush)
+            ms1 = _timed(lambda: nb.nvfp4_quantize(x, out=q, global_supplied=True, workspace=ws),
+                         args.steps, args.warmup, None if big else flush)
+            bpv = QUANT_BYTES_PER_VALUE_2PASS if big else ENCODE_BYTES_PER_VALUE
+            rows.append({"values": n, "ms": ms, "gbs": n * bpv / ms / 1e6,
+                         "bytes_per_value": bpv, "ms_supplied_scale": ms1,
+                         "gbs_supplied_scale": n * ENCODE_BYTES_PER_VALUE / ms1 / 1e6})
+            del x, q
+        top = rows[-1]
+        line.update({"metric": "NVFP4 quantize GB/s (2^28 values)", "value": top["gbs"],
+                     "unit": "GB/s", "higher_is_better": True, "ms_per_step": top["ms"],
+                     "config": {"workload": "quantize sweep 2^20 / 2^24 / 2^28 values"},
+                     "roofline": {"bound": "hbm", "achieved": top["gbs"], "peak": hbm_gbs,
+                                  "unit": "GB/s", "frac": top["gbs"] / hbm_gbs,
+                                  "peak_source": f"{peak_src} hbm_gbs"},
+                     "rows": rows})
+        return line
+
+    if name in ("ffn16", "ffn512"):
+        m = int(name[3:])
+        w = inputs.ffn_weight(device=device)
+        qw = nb.nvfp4_quantize(w, workspace=ws)
+        del w
+        a = inputs.ffn_activation(m, device=device)
+        qa = nb.NVFP4Tensor.empty(m, K, device=device)
+        d = torch.empty((m, N), dtype=torch.bfloat16, device=device)
+        qms = _timed(lambda: nb.nvfp4_quantize(a, out=qa, workspace=ws), args.steps, args.warmup, flush)
+        gms = _timed(lambda: nb.nvfp4_gemm(qa, qw, out=d, workspace=ws), args.steps, args.warmup, flush)
+        flops = 2.0 * m * N * K
+        wbytes = qw.nbytes() + qa.nbytes() + d.numel() * 2
+        gbs = wbytes / gms / 1e6
+        line.update({"metric": f"NVFP4 W4A4 linear M={m} TFLOP/s", "value": flops / (qms + gms) / 1e9,
+                     "unit": "TFLOP/s", "higher_is_better": True, "ms_per_step": qms + gms,
+                     "config": {"workload": f"ffn linear M={m} N={N} K={K}", "l2": "flushed"},
+                     "gemm_ms": gms, "quantize_ms": qms, "gemm_tflops": flops / gms / 1e9,
+                     "roofline": {"kernel": "k_gemm_nvf4", "bound": "hbm", "achieved": gbs,
+                                  "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                                  "algorithmic_bytes_per_launch": wbytes,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
+        return line
+
+    if name == "moe":
+        r = inputs.MoeRouting()
+        E, H, I = inputs.MOE_EXPERTS, inputs.MOE_HIDDEN, inputs.MOE_INTER
+        x = inputs.moe_activation(device=device)
+        slot = r.slot_offsets.to(device)
+        rows = r.rows.to(device)
+        gather = r.gather.to(device)
+        ident = torch.where(r.gather >= 0, torch.arange(r.padded_rows, dtype=torch.int32),
+                            torch.full_like(r.gather, -1)).to(device)
+        def stacked(which, n, k):
+            q = nb.NVFP4Tensor.empty(E * n, k, device=device)
+            g = torch.zeros(E, dtype=torch.float32, device=device)
+            sfb = nb.nvfp4_scales_bytes(n, k)
+            for e in range(E):
+                w = inputs.moe_expert_weight(which, e, device=device)
+                sub = nb.NVFP4Tensor(q.codes[e * n:(e + 1) * n], q.scales[e * sfb:(e + 1) * sfb],
+                                     g[e:e + 1], n, k, nb.SF_SWIZZLED)
+                nb.nvfp4_quantize(w, out=sub, workspace=ws)
+            return q, g
+        wu, gu = stacked("up", I, H)
+        wd, gd = stacked("down", H, I)
+        gx = torch.zeros(1, dtype=torch.float32, device=device)
+        qx = nb.NVFP4Tensor.empty(r.padded_rows, H, device=device, global_scale=gx)
+        hbuf = torch.empty((r.padded_rows, I), dtype=torch.bfloat16, device=device)
+        qh = nb.NVFP4Tensor.empty(r.padded_rows, I, device=device)
+        y = torch.empty((r.padded_rows, H), dtype=torch.bfloat16, device=device)
+        ev = {}
+
+        def step(mark=False):
+            nb.nvfp4_global_scale(x, out=gx, workspace=ws)
+            nb.nvfp4_quantize_gather(x, gather, out=qx, global_supplied=True, workspace=ws)
+            nb.nvfp4_grouped_gemm(slot, rows, qx, wu, gu, I, out=hbuf, workspace=ws)
+            nb.nvfp4_quantize_gather(hbuf, ident, out=qh, workspace=ws)
+            if mark:
+                ev["a"].record()
+            nb.nvfp4_grouped_gemm(slot, rows, qh, wd, gd, H, out=y, workspace=ws)
+            if mark:
+                ev["b"].record()
+
+        ms = _timed(step, args.steps, args.warmup, flush)
+        ev["a"], ev["b"] = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush()
+        step(mark=True)
+        torch.cuda.synchronize()
+        down_ms = ev["a"].elapsed_time(ev["b"])
+        st = nb.nvfp4_check_status(ws)
+        flops = 2.0 * r.real_rows * I * H * 2
+        down_bytes = wd.nbytes() + qh.nbytes() + r.real_rows * H * 2
+        gbs = down_bytes / down_ms / 1e6
+        line.update({"metric": "NVFP4 MoE expert block TFLOP/s (up + down grouped GEMMs)",
+                     "value": flops / ms / 1e9, "unit": "TFLOP/s", "higher_is_better": True,
+                     "ms_per_step": ms,
+                     "config": {"workload": f"moe {E} experts top-{inputs.MOE_TOPK} of "
+                                            f"{inputs.MOE_TOKENS} tokens, hidden {H}, inter {I}",
+                                "real_rows": r.real_rows, "padded_rows": r.padded_rows,
+                                "l2": "flushed"},
+                     "weights_bytes": wu.nbytes() + wd.nbytes(), "status": st,
+                     "roofline": {"kernel": "k_gemm_nvf4 (grouped, down projection)",
+                                  "bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s",
+                                  "frac": gbs / hbm_gbs, "ms_per_launch": down_ms,
+                                  "algorithmic_bytes_per_launch": down_bytes,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
+        return line
+
+    if name == "kv":
+        L, T = inputs.KV_LAYERS, inputs.KV_TOKENS
+        C = inputs.KV_HEADS * inputs.KV_HEAD_DIM
+        xs = [inputs.kv_tensor(l, kv, device=device).view(T, C) for l in range(L) for kv in (0, 1)]
+        qs = [nb.NVFP4Tensor.empty(T, C, nb.SF_LINEAR, device) for _ in xs]
+        y = torch.empty((T, C), dtype=torch.bfloat16, device=device)
+
+        def quant_all():
+            for x, q in zip(xs, qs):
+                nb.nvfp4_quantize(x, out=q, workspace=ws)
+
+        def deq_all():
+            for q in qs:
+                nb.nvfp4_dequantize(q, out=y)
+
+        qms = _timed(quant_all, args.steps, args.warmup)
+        dms = _timed(deq_all, args.steps, args.warmup)
+        st = nb.nvfp4_check_status(ws)
+        nvals = len(xs) * T * C
+        qgbs = nvals * QUANT_BYTES_PER_VALUE_2PASS / qms / 1e6
+        dgbs = nvals * (0.5625 + 2.0) / dms / 1e6
+        per_token = sum(q.nbytes() for q in qs) // T
+        line.update({"metric": "NVFP4 KV-cache quantize GB/s (32 layers x K,V, 128K tokens)",
+                     "value": qgbs, "unit": "GB/s", "higher_is_better": True, "ms_per_step": qms,
+                     "config": {"workload": "kv cache 32 x {K,V} x [131072 x 8 x 128]"},
+                     "bytes_per_token": per_token, "bytes_per_value": per_token / (2 * L * C),
+                     "dequantize_ms": dms, "dequantize_gbs": dgbs, "status": st,
+                     "roofline": {"kernel": "k_amax + k_encode", "bound": "hbm", "achieved": qgbs,
+                                  "peak": hbm_gbs, "unit": "GB/s", "frac": qgbs / hbm_gbs,
+                                  "bytes_per_value": QUANT_BYTES_PER_VALUE_2PASS,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
+        return line
+    raise ValueError(name)
+
+
 # -------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -320,6 +505,9 @@ def main():
                     help="skip the standalone 2^28 quantize measurement")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--workload", default="ffn8192",
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv"],
+                    help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")
     args = ap.parse_args()
@@ -331,6 +519,11 @@ def main():
     rank, local_rank, world = env_rank()
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
+    if args.workload != "ffn8192":
+        if world == 1:
+            line = workload_line(args.workload, args, device)
+            print(json.dumps(line), flush=True)
+            return 0
     dist = None
     if world > 1:
         import datetime

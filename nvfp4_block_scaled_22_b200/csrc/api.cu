@@ -147,8 +147,9 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
     p.partials = partials;
     p.n_partials = n_partials;
     p.status = status;
-    const int64_t tasks = ceil_div(out->rows, 128) * ceil_div(out->cols, 64);
-    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    const int64_t tasks = ceil_div(out->rows, 128) * 128 * ceil_div(ceil_div(out->cols / 16, 4) * 4, 32);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * 4), 8LL * sms);
     if (grid < 1) grid = 1;
     k_encode<<<grid, 256, 0, stream>>>(p);
     return launched(cudaGetLastError());
@@ -276,8 +277,9 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     p.cols = in->cols;
     p.y = static_cast<uint16_t *>(y);
     p.ld = ld;
-    const int64_t tasks = ceil_div(in->rows, 128) * ceil_div(in->cols, 64);
-    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    const int64_t tasks = in->rows * ceil_div(in->cols / 16, 32);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * 4), 8LL * sms);
     if (grid < 1) grid = 1;
     k_dequantize<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return launched(cudaGetLastError());

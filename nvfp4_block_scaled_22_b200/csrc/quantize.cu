@@ -14,10 +14,9 @@
 //   k_encode      : g (from partials or supplied) -> codes + scales.
 //   k_dequantize  : codes + scales + g -> BF16.
 //
-// Work split of k_encode/k_dequantize: one warp owns a 128-row x 64-column
-// tile; lane l handles rows l, l+32, l+64, l+96 of the tile, 4 blocks of 16
-// each.  Those 4x4 scale bytes are exactly one 16-byte row of the 512-byte
-// 128x4 scale tile, so the warp writes its scales as 512 contiguous bytes.
+// Work split of k_encode/k_dequantize: a warp takes one row's 512-value
+// segment, one 16-value block per lane, so every global access of a warp is
+// contiguous (see the comment above k_encode).
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -140,6 +139,35 @@ __global__ void k_finalize_g(const uint32_t *__restrict__ partials, int n, float
 }
 
 // --------------------------------------------------------------- k_encode
+// Exact shortcuts for the two per-block IEEE divisions, filled once per CTA
+// into shared memory:
+//  * div6[m] = RN((1 + m/128) / 6) for the 128 BF16 mantissas.  For a block
+//    amax a = (1 + m/128) * 2^k whose quotient stays a normal number,
+//    RN(a / 6) = div6[m] * 2^k exactly (scaling by a power of two commutes
+//    with rounding), applied as an exponent-field add; other amax values
+//    (zero, subnormal, tiny, non-finite) take the division itself.
+//  * inv_s[b] = RN(g / e4m3(b)) for the 127 non-negative finite E4M3 codes
+//    (inv_s[0] = 0 gives the zero-scale rule).
+struct EncodeTables {
+    float div6[128];
+    float inv_s[128];
+};
+
+__device__ __forceinline__ void fill_tables(EncodeTables &t, float g) {
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+        t.div6[i] = __fdiv_rn(1.0f + (float)i * 0.0078125f, 6.0f);
+        t.inv_s[i] = (i == 0 || i == 0x7F) ? 0.0f : __fdiv_rn(g, f32_from_e4m3((uint32_t)i));
+    }
+}
+
+// RN(a / 6) for a >= 0 given as f32 bits from a BF16 value.
+__device__ __forceinline__ float div6_rn(uint32_t bits, const EncodeTables &t) {
+    const uint32_t e = bits >> 23;                      // sign is clear
+    if (e >= 4u && e < 255u)
+        return __uint_as_float(__float_as_uint(t.div6[(bits >> 16) & 0x7Fu]) + ((e - 127u) << 23));
+    return __fdiv_rn(__uint_as_float(bits), 6.0f);
+}
+
 struct EncodeBlockOut {
     uint2 codes;
     uint32_t scale;
@@ -147,13 +175,13 @@ struct EncodeBlockOut {
 };
 
 // Quantize one 16-value block held in two 16-byte words.
-__device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g) {
+__device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g,
+                                                       const EncodeTables &tab) {
     uint32_t mw = amax_word(a, b);
     const uint32_t bits = halves_to_f32bits(mw);
-    float amax_b = __uint_as_float(bits);
-    float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g);
+    float t = __fmul_rn(div6_rn(bits, tab), g);
     uint32_t s = e4m3_from_f32(t);
-    float e = (s == 0u) ? 0.0f : __fdiv_rn(g, f32_from_e4m3(s));
+    float e = tab.inv_s[s & 0x7Fu];
     uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     float y[16];
 #pragma unroll
@@ -169,8 +197,35 @@ __device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g
     return o;
 }
 
+// Byte offset of scale (row r, scale column c) in either layout.
+__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sf_cols, int64_t col_tiles,
+                                             int32_t layout) {
+    if (layout == 1) return r * sf_cols + c;
+    return ((r >> 7) * col_tiles + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
+}
+
+// Work split: a task is one row and one 512-value segment of it; lane l
+// owns 16-value block l of the segment (two 16-byte loads, one 8-byte code
+// store), so a warp's loads and stores are contiguous.  The four scale
+// bytes of blocks 4j..4j+3 are contiguous in both scale layouts; lanes
+// 4j..4j+3 combine them with two shuffles and lane 4j stores the word.
+// Rows past the end of the last 128-row band (swizzled layout) and scale
+// columns past cols/16 up to the next multiple of 4 are written as zero.
+constexpr int kSegValues = 512;
+constexpr int kUnroll = 4;
+
+// Row of flat task t (tasks laid out row-major, segs per row) without a
+// 64-bit division: float reciprocal, then exact integer correction.
+__device__ __forceinline__ uint32_t task_row(uint32_t t, uint32_t segs, float inv) {
+    uint32_t r = __float2uint_rz((float)t * inv);
+    while (r * segs > t) --r;
+    while ((r + 1) * segs <= t) ++r;
+    return r;
+}
+
 __global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
     __shared__ uint32_t red[kThreads / 32];
+    __shared__ EncodeTables tab;
     float g;
     if (p.global_supplied) {
         g = *p.global;
@@ -178,82 +233,72 @@ __global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
         if (!global_from_partials(p.partials, p.n_partials, p.status, &g, red)) return;
         if (blockIdx.x == 0 && threadIdx.x == 0) *p.global = g;
     }
+    fill_tables(tab, g);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int64_t row_tiles = (p.rows + 127) / 128;
-    const int64_t col_tiles = (p.cols + 63) / 64;   // = padded scale columns / 4
-    const int64_t tasks = row_tiles * col_tiles;
-    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t sf_cols = p.cols / 16;
-    const bool codes16 = ((p.cols / 2) % 16) == 0;
-    for (int64_t t = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < tasks;
-         t += warps) {
-        const int64_t rt = t / col_tiles, ct = t - rt * col_tiles;
-        const int nb = (int)(sf_cols - ct * 4 < 4 ? sf_cols - ct * 4 : 4);  // valid blocks here
-        uint32_t sf_rows[4];
-        bool finite = true;
+    const int64_t sf_cols4 = (sf_cols + 3) / 4 * 4;               // padded scale columns
+    const int64_t col_tiles = sf_cols4 / 4;
+    const int64_t segs = (sf_cols4 + 31) / 32;                    // 32 blocks per segment
+    const int64_t rows_out = (p.layout == 0) ? (p.rows + 127) / 128 * 128 : p.rows;
+    const uint32_t tasks = (uint32_t)(rows_out * segs);        // < 2^32 (host-checked)
+    const uint32_t warps = gridDim.x * (kThreads / 32);
+    const float inv_segs = 1.0f / (float)segs;
+    bool finite = true;
+    for (uint32_t t0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t0 < tasks;
+         t0 += warps * kUnroll) {
+        uint4 va[kUnroll], vb[kUnroll];
+        int64_t rr[kUnroll], bb[kUnroll];
+        bool has[kUnroll];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t r = rt * 128 + q * 32 + lane;
-            uint32_t sfw = 0;
-            int64_t src = r;
-            if (r < p.rows && p.gather != nullptr) {
-                src = p.gather[r];
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t t = t0 + warps * u;
+            const uint32_t row = task_row(t, (uint32_t)segs, inv_segs);
+            rr[u] = row;
+            bb[u] = (int64_t)(t - row * (uint32_t)segs) * 32 + lane;   // scale column of this lane
+            int64_t src = rr[u];
+            has[u] = t < tasks && rr[u] < p.rows && bb[u] < sf_cols;
+            if (has[u] && p.gather != nullptr) {
+                src = p.gather[rr[u]];
                 if (src >= p.src_rows) {     // out-of-range map entry: zero row + status
                     set_status(p.status, ST_INVALID_ARG);
                     src = -1;
                 }
+                if (src < 0) has[u] = false;
             }
-            if (r < p.rows && src >= 0) {
-                const uint4 *xp =
-                    reinterpret_cast<const uint4 *>(p.x + src * p.ld + ct * 64);
-                uint8_t *cp = p.codes + r * (p.cols / 2) + ct * 32;
-                if (nb == 4) {
-                    uint4 v[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] = __ldg(xp + i);
-                    EncodeBlockOut o[4];
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        o[b] = encode_block(v[2 * b], v[2 * b + 1], g);
-                        finite &= o[b].finite;
-                    }
-                    if (codes16) {
-                        uint4 *c4 = reinterpret_cast<uint4 *>(cp);
-                        c4[0] = make_uint4(o[0].codes.x, o[0].codes.y, o[1].codes.x, o[1].codes.y);
-                        c4[1] = make_uint4(o[2].codes.x, o[2].codes.y, o[3].codes.x, o[3].codes.y);
-                    } else {
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) reinterpret_cast<uint2 *>(cp)[b] = o[b].codes;
-                    }
-                    sfw = o[0].scale | (o[1].scale << 8) | (o[2].scale << 16) | (o[3].scale << 24);
-                } else {
-                    for (int b = 0; b < nb; ++b) {
-                        EncodeBlockOut o = encode_block(__ldg(xp + 2 * b), __ldg(xp + 2 * b + 1), g);
-                        finite &= o.finite;
-                        reinterpret_cast<uint2 *>(cp)[b] = o.codes;
-                        sfw |= o.scale << (8 * b);
-                    }
-                }
-            } else if (r < p.rows) {  // gathered padding row: zero codes
-                uint8_t *cp = p.codes + r * (p.cols / 2) + ct * 32;
-                for (int b = 0; b < nb; ++b) reinterpret_cast<uint2 *>(cp)[b] = make_uint2(0, 0);
-            }
-            sf_rows[q] = sfw;
-            if (p.layout == 1 && r < p.rows) {  // linear [rows x cols/16]
-                uint8_t *sp = p.scales + r * sf_cols + ct * 4;
-                if (nb == 4 && (sf_cols % 4) == 0) {
-                    *reinterpret_cast<uint32_t *>(sp) = sfw;
-                } else {
-                    for (int b = 0; b < nb; ++b) sp[b] = (uint8_t)(sfw >> (8 * b));
-                }
+            if (has[u]) {
+                const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + src * p.ld + bb[u] * 16);
+                va[u] = __ldg(xp);
+                vb[u] = __ldg(xp + 1);
             }
         }
-        if (!finite) set_status(p.status, ST_NONFINITE);  // only reachable with a supplied g
-        if (p.layout == 0) {  // 128x4 tile: this lane's 16 bytes, padding = 0
-            uint4 *sp = reinterpret_cast<uint4 *>(p.scales + (rt * col_tiles + ct) * 512) + lane;
-            *sp = make_uint4(sf_rows[0], sf_rows[1], sf_rows[2], sf_rows[3]);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t t = t0 + warps * u;
+            if (t >= tasks) break;                                   // uniform across the warp
+            uint32_t s = 0;
+            if (has[u]) {
+                EncodeBlockOut o = encode_block(va[u], vb[u], g, tab);
+                finite &= o.finite;
+                s = o.scale;
+                *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;
+            } else if (rr[u] < p.rows && bb[u] < sf_cols) {          // gathered padding row
+                *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = make_uint2(0, 0);
+            }
+            uint32_t w = s << (8 * (lane & 3));
+            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+            if ((lane & 3) == 0 && bb[u] < sf_cols4 && (p.layout == 0 || bb[u] < sf_cols)) {
+                uint8_t *sp = p.scales + sf_offset(rr[u], bb[u], sf_cols, col_tiles, p.layout);
+                if (p.layout == 0 || ((sf_cols & 3) == 0 && bb[u] + 4 <= sf_cols)) {
+                    *reinterpret_cast<uint32_t *>(sp) = w;
+                } else {                                             // ragged linear row
+                    for (int j = 0; j < 4 && bb[u] + j < sf_cols; ++j) sp[j] = (uint8_t)(w >> (8 * j));
+                }
+            }
         }
     }
+    if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
 }
 
 // ----------------------------------------------------------- k_dequantize
@@ -275,35 +320,39 @@ __device__ __forceinline__ void decode_block(uint2 codes, float d, uint4 &o0, ui
 __global__ void __launch_bounds__(kThreads) k_dequantize(DequantParams p) {
     const float g = *p.global;
     const int lane = threadIdx.x & 31;
-    const int64_t row_tiles = (p.rows + 127) / 128;
-    const int64_t col_tiles = (p.cols + 63) / 64;
-    const int64_t tasks = row_tiles * col_tiles;
-    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t sf_cols = p.cols / 16;
-    for (int64_t t = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < tasks;
-         t += warps) {
-        const int64_t rt = t / col_tiles, ct = t - rt * col_tiles;
-        const int nb = (int)(sf_cols - ct * 4 < 4 ? sf_cols - ct * 4 : 4);
-        uint4 sf_tile = make_uint4(0, 0, 0, 0);
-        if (p.layout == 0)
-            sf_tile = __ldg(reinterpret_cast<const uint4 *>(p.scales + (rt * col_tiles + ct) * 512) + lane);
-        const uint32_t sfq[4] = {sf_tile.x, sf_tile.y, sf_tile.z, sf_tile.w};
+    const int64_t col_tiles = (sf_cols + 3) / 4;
+    const int64_t segs = (sf_cols + 31) / 32;
+    const uint32_t tasks = (uint32_t)(p.rows * segs);          // < 2^32 (host-checked)
+    const uint32_t warps = gridDim.x * (kThreads / 32);
+    const float inv_segs = 1.0f / (float)segs;
+    for (uint32_t t0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t0 < tasks;
+         t0 += warps * kUnroll) {
+        uint2 c[kUnroll];
+        uint32_t sb[kUnroll];
+        int64_t rr[kUnroll], bb[kUnroll];
+        bool has[kUnroll];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t r = rt * 128 + q * 32 + lane;
-            if (r >= p.rows) continue;
-            const uint8_t *cp = p.codes + r * (p.cols / 2) + ct * 32;
-            uint4 *yp = reinterpret_cast<uint4 *>(p.y + r * p.ld + ct * 64);
-            for (int b = 0; b < nb; ++b) {
-                uint32_t s = (p.layout == 0) ? (sfq[q] >> (8 * b)) & 0xFFu
-                                             : (uint32_t)p.scales[r * sf_cols + ct * 4 + b];
-                float d = __fdiv_rn(f32_from_e4m3(s), g);
-                uint2 c = __ldg(reinterpret_cast<const uint2 *>(cp) + b);
-                uint4 o0, o1;
-                decode_block(c, d, o0, o1);
-                yp[2 * b] = o0;
-                yp[2 * b + 1] = o1;
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t t = t0 + warps * u;
+            const uint32_t row = task_row(t, (uint32_t)segs, inv_segs);
+            rr[u] = row;
+            bb[u] = (int64_t)(t - row * (uint32_t)segs) * 32 + lane;
+            has[u] = t < tasks && bb[u] < sf_cols;
+            if (has[u]) {
+                c[u] = __ldg(reinterpret_cast<const uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8));
+                sb[u] = __ldg(p.scales + sf_offset(rr[u], bb[u], sf_cols, col_tiles, p.layout));
             }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (!has[u]) continue;
+            const float d = __fdiv_rn(f32_from_e4m3(sb[u]), g);
+            uint4 o0, o1;
+            decode_block(c[u], d, o0, o1);
+            uint4 *yp = reinterpret_cast<uint4 *>(p.y + rr[u] * p.ld + bb[u] * 16);
+            yp[0] = o0;
+            yp[1] = o1;
         }
     }
 }
