@@ -72,7 +72,8 @@ def test_up_projection_full_size(routing):
     qx = nb.NVFP4Tensor.empty(routing.padded_rows, H, device=DEV, global_scale=gx)
     nb.nvfp4_quantize_gather(x, routing.gather.to(DEV), out=qx, global_supplied=True)
     wu, gu, sfb = _stacked("up", I, H)
-    h = nb.nvfp4_grouped_gemm(routing.slot_offsets.to(DEV), routing.rows.to(DEV), qx, wu, gu, I)
+    h = torch.zeros((routing.padded_rows, I), dtype=torch.bfloat16, device=DEV)
+    nb.nvfp4_grouped_gemm(routing.slot_offsets.to(DEV), routing.rows.to(DEV), qx, wu, gu, I, out=h)
     assert nb.nvfp4_check_status() == 0
 
     xc = x.cpu()
@@ -105,7 +106,8 @@ def test_down_projection_full_size(routing):
                         torch.full_like(routing.gather, -1)).to(DEV)
     qh = nb.nvfp4_quantize_gather(hmid, ident)
     wd, gd, sfb = _stacked("down", H, I)
-    y = nb.nvfp4_grouped_gemm(routing.slot_offsets.to(DEV), routing.rows.to(DEV), qh, wd, gd, H)
+    y = torch.zeros((routing.padded_rows, H), dtype=torch.bfloat16, device=DEV)
+    nb.nvfp4_grouped_gemm(routing.slot_offsets.to(DEV), routing.rows.to(DEV), qh, wd, gd, H, out=y)
     assert nb.nvfp4_check_status() == 0
 
     hc = hmid.cpu()
