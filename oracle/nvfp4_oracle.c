@@ -22,6 +22,9 @@
  *       block amax mapped close to the FP4 maximum.
  *  [P5] "FP4 KV-cache quantization" (theddari.com), section "FP4 formats
  *       compared": 0.5625 bytes per value (4.5 bits) including scales.
+ *  [P2'] same pre-training page, section "Four stabilisation devices": the
+ *       Wgrad inputs are multiplied by a 16x16 Hadamard matrix and a random
+ *       +-1 sign vector before quantization.
  *  The FP32 evaluation order below is the convention the hot path is
  *  specified with: global g = 448*6/amax_tensor, block scale
  *  s = e4m3_rne(amax_block/6*g), code = e2m1_rne(x*g/s), with x*g/s taken as
@@ -367,4 +370,106 @@ int64_t nvo_dot_exact_i64(const uint8_t *a_codes, const uint8_t *a_sf, int a_lay
         acc += a2 * sa * w2 * sw;
     }
     return acc;
+}
+
+/* ------------------------------------------- random Hadamard transform */
+
+/* [P2'] 16x16 random Hadamard transform of one block.  READINGS (the page
+ * names the matrices only): y = (1/4) * H16 * diag(s) * x with H16 the
+ * Sylvester Hadamard matrix, H[i][j] = (-1)^popcount(i & j), scaled by 1/4 so
+ * that the transform is orthonormal; s_j = -1 where bit j of sign_mask is
+ * set.  FP32 evaluation: z_j = s_j x_j (exact), then the in-place fast
+ * Walsh-Hadamard butterfly with strides 1, 2, 4, 8 -- each pair (z_i, z_{i+h})
+ * becomes (RN(z_i + z_{i+h}), RN(z_i - z_{i+h})) -- then y_i = RN(z_i / 4). */
+void nvo_rht16(const float *x, uint32_t sign_mask, float *y)
+{
+    float z[16];
+    for (int j = 0; j < 16; ++j)
+        z[j] = ((sign_mask >> j) & 1u) ? -x[j] : x[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & h) == 0) {
+                float a = z[i], b = z[i + h];
+                z[i] = a + b;
+                z[i + h] = a - b;
+            }
+    for (int i = 0; i < 16; ++i)
+        y[i] = z[i] * 0.25f;
+}
+
+/* Inverse of nvo_rht16 in exact arithmetic: x = diag(s) * (1/4) * H16 * y
+ * (H16 is symmetric and H16 * H16 = 16 I).  Same butterfly, signs after. */
+void nvo_rht16_inverse(const float *y, uint32_t sign_mask, float *x)
+{
+    float z[16];
+    for (int j = 0; j < 16; ++j)
+        z[j] = y[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & h) == 0) {
+                float a = z[i], b = z[i + h];
+                z[i] = a + b;
+                z[i + h] = a - b;
+            }
+    for (int j = 0; j < 16; ++j) {
+        float v = z[j] * 0.25f;
+        x[j] = ((sign_mask >> j) & 1u) ? -v : v;
+    }
+}
+
+/* Two-level NVFP4 quantization of the transformed tensor: every 16-block
+ * of each row goes through nvo_rht16 first (FP32 values, not rounded back
+ * to BF16), then amax, g, block scales and codes follow the same steps as
+ * nvo_quantize on those FP32 values.  global_supplied = 1 uses *g_io. */
+int nvo_quantize_rht(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, uint32_t sign_mask,
+                     uint8_t *codes, uint8_t *scales, int layout, int global_supplied, float *g_io)
+{
+    if (cols % 16 != 0 || rows < 0 || cols < 0)
+        return NVO_ERR_SHAPE;
+    float g = *g_io;
+    if (!global_supplied) {
+        float m = 0.0f;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t b = 0; b < cols / 16; ++b) {
+                float in[16], y[16];
+                for (int i = 0; i < 16; ++i)
+                    in[i] = nvo_bf16_to_f32(x[r * ld + b * 16 + i]);
+                nvo_rht16(in, sign_mask, y);
+                for (int i = 0; i < 16; ++i) {
+                    float v = fabsf(y[i]);
+                    if (!isfinite(v))
+                        return NVO_ERR_NONFINITE;
+                    if (v > m)
+                        m = v;
+                }
+            }
+        int st = nvo_global_scale(m, &g);
+        *g_io = g;
+        if (st != NVO_OK)
+            return st;
+    }
+    memset(scales, 0, (size_t)nvo_scales_bytes(rows, cols, layout));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            float in[16], y[16];
+            for (int i = 0; i < 16; ++i)
+                in[i] = nvo_bf16_to_f32(x[r * ld + b * 16 + i]);
+            nvo_rht16(in, sign_mask, y);
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i)
+                if (fabsf(y[i]) > amax_b)
+                    amax_b = fabsf(y[i]);
+            float t = amax_b / 6.0f;
+            t = t * g;
+            uint8_t s = nvo_e4m3_rne_satfinite(t);
+            float e = (s == 0) ? 0.0f : g / nvo_e4m3_decode(s);
+            scales[nvo_sf_offset(r, b, rows, cols, layout)] = s;
+            uint8_t *cb = codes + r * (cols / 2) + b * 8;
+            for (int i = 0; i < 8; ++i) {
+                uint8_t c0 = nvo_e2m1_rne_satfinite(y[2 * i] * e);
+                uint8_t c1 = nvo_e2m1_rne_satfinite(y[2 * i + 1] * e);
+                cb[i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return NVO_OK;
 }

@@ -17,7 +17,7 @@ __all__ = [
     "lib", "bf16_bits", "bf16_to_f32", "f32_to_bf16", "e2m1_decode", "e2m1_rne",
     "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
     "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
-    "dot_exact_i64", "Quantized",
+    "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -52,6 +52,10 @@ def lib() -> C.CDLL:
                                     _i64, _i64, _p, _p, _i64, _p, _p]),
             "nvo_dot_exact_i64": (_i64, [_p, _p, C.c_int, _i64, _p, _p, C.c_int, _i64,
                                          _i64, _i64, _i64]),
+            "nvo_rht16": (None, [_p, C.c_uint32, _p]),
+            "nvo_rht16_inverse": (None, [_p, C.c_uint32, _p]),
+            "nvo_quantize_rht": (C.c_int, [_p, _i64, _i64, _i64, C.c_uint32, _p, _p, C.c_int,
+                                           C.c_int, C.POINTER(C.c_float)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -187,6 +191,33 @@ def dot_exact_i64(a: Quantized, w: Quantized, i: int, j: int) -> int:
     return int(lib().nvo_dot_exact_i64(_ptr(a.codes), _ptr(a.scales), a.layout, a.rows,
                                        _ptr(w.codes), _ptr(w.scales), w.layout, w.rows,
                                        a.cols, i, j))
+
+
+def rht16(x, sign_mask: int) -> np.ndarray:
+    """Random Hadamard transform of one 16-value block (float32)."""
+    x = np.ascontiguousarray(x, np.float32)
+    y = np.zeros(16, np.float32)
+    lib().nvo_rht16(_ptr(x), sign_mask, _ptr(y))
+    return y
+
+
+def rht16_inverse(y, sign_mask: int) -> np.ndarray:
+    y = np.ascontiguousarray(y, np.float32)
+    x = np.zeros(16, np.float32)
+    lib().nvo_rht16_inverse(_ptr(y), sign_mask, _ptr(x))
+    return x
+
+
+def quantize_rht(x, sign_mask: int, layout: int = SF_SWIZZLED, g=None) -> tuple[int, Quantized]:
+    """Quantize the random-Hadamard-transformed tensor (g given = supplied)."""
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    gv = C.c_float(0.0 if g is None else float(np.float32(g)))
+    st = lib().nvo_quantize_rht(_ptr(b), rows, cols, cols, sign_mask, _ptr(codes), _ptr(scales),
+                                layout, 0 if g is None else 1, C.byref(gv))
+    return st, Quantized(codes, scales, gv.value, rows, cols, layout)
 
 
 if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):
