@@ -44,8 +44,8 @@ FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
 # the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
 # Reported only while the kernel's sources hash to the profiled version.
-GEMM_TRAFFIC_BYTES = 87.4e6 + 293.3e6
-GEMM_TRAFFIC_SRC_SHA = "394c042151ea74c5"
+GEMM_TRAFFIC_BYTES = 86.6e6 + 292.3e6
+GEMM_TRAFFIC_SRC_SHA = "a6d927ba934dfbba"
 GEMM_SOURCES = ("gemm.cu", "kernels.h", "ptx.cuh")
 
 
@@ -489,6 +489,58 @@ def workload_line(name, args, device):
                                   "bytes_per_value": QUANT_BYTES_PER_VALUE_2PASS,
                                   "peak_source": f"{peak_src} hbm_gbs"}})
         return line
+    if name == "wgrad":
+        m = inputs.WGRAD_M
+        mask = inputs.rht_sign_mask(0)
+        dy_t = inputs.wgrad_grad_output_t(m, device=device)
+        x_t = inputs.wgrad_activation_t(m, device=device)
+        qa = nb.NVFP4Tensor.empty(N, m, device=device)
+        qw = nb.NVFP4Tensor.empty(K, m, device=device)
+        d = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+        ev = {k: torch.cuda.Event(enable_timing=True) for k in "abcd"}
+
+        def step(mark=False):
+            if mark:
+                ev["a"].record()
+            nb.nvfp4_quantize_rht(dy_t, mask, out=qa, workspace=ws)
+            if mark:
+                ev["b"].record()
+            nb.nvfp4_quantize_rht(x_t, mask, out=qw, workspace=ws)
+            if mark:
+                ev["c"].record()
+            nb.nvfp4_gemm(qa, qw, out=d, workspace=ws)
+            if mark:
+                ev["d"].record()
+
+        ms = _timed(step, args.steps, args.warmup, flush)
+        qa_ms, qw_ms, g_ms = [], [], []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush()
+            step(mark=True)
+            torch.cuda.synchronize()
+            qa_ms.append(ev["a"].elapsed_time(ev["b"]))
+            qw_ms.append(ev["b"].elapsed_time(ev["c"]))
+            g_ms.append(ev["c"].elapsed_time(ev["d"]))
+        qa_ms, qw_ms, g_ms = (statistics.median(v) for v in (qa_ms, qw_ms, g_ms))
+        st = nb.nvfp4_check_status(ws)
+        flops = 2.0 * N * K * m
+        qgbs = N * m * QUANT_BYTES_PER_VALUE_2PASS / qa_ms / 1e6
+        line.update({"metric": "NVFP4 Wgrad step TFLOP/s (RHT quantize of dY^T and X^T + GEMM)",
+                     "value": flops / ms / 1e9, "unit": "TFLOP/s", "higher_is_better": True,
+                     "ms_per_step": ms,
+                     "config": {"workload": f"wgrad dW = dY^T X, {N} x {K}, {m} tokens, "
+                                            "16x16 RHT on both operands", "sign_mask": mask,
+                                "l2": "flushed"},
+                     "quantize_rht_dy_ms": qa_ms, "quantize_rht_x_ms": qw_ms, "gemm_ms": g_ms,
+                     "quantize_rht_dy_gbs": qgbs,
+                     "quantize_rht_x_gbs": K * m * QUANT_BYTES_PER_VALUE_2PASS / qw_ms / 1e6,
+                     "gemm_tflops": flops / g_ms / 1e9, "status": st,
+                     "roofline": {"kernel": "k_amax_rht + k_encode_rht (dY^T)", "bound": "hbm",
+                                  "achieved": qgbs, "peak": hbm_gbs, "unit": "GB/s",
+                                  "frac": qgbs / hbm_gbs,
+                                  "bytes_per_value": QUANT_BYTES_PER_VALUE_2PASS,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
+        return line
     raise ValueError(name)
 
 
@@ -506,7 +558,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--workload", default="ffn8192",
-                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv"],
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")

@@ -152,6 +152,29 @@ NVFP4_API nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t 
                                    int32_t global_supplied, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* Quantize after a 16x16 random Hadamard transform of every 16-value block
+ * ("NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens", section
+ * "Four stabilisation devices": the Wgrad GEMM inputs are multiplied by a
+ * 16x16 Hadamard matrix and a random +-1 sign vector before quantization).
+ * Per block of 16 consecutive values along a row:
+ *   y = (1/4) * H16 * diag(s) * x,  H16[i][j] = (-1)^popcount(i & j),
+ *   s_j = -1 where bit j of sign_mask is set, else +1,
+ * evaluated in FP32 as an in-place butterfly with strides 1, 2, 4, 8 (each
+ * add/sub rounded to nearest even) and an exact-order multiply by 1/4.  The
+ * FP32 values y (not rounded to BF16) are then quantized as nvfp4_quantize
+ * quantizes x: g = RN(2688 / max|y|) unless supplied, s_b, codes.  The
+ * transform is orthogonal, so an NVFP4 GEMM of two operands transformed
+ * with the same sign_mask along the contraction axis approximates the
+ * product of the untransformed operands.
+ * sign_mask: the random sign vector drawn by the caller, bits 0..15
+ *   (NVFP4_ERR_INVALID_ARG if any higher bit is set).
+ * Other arguments, the workspace, the status word and the errors are those
+ * of nvfp4_quantize; an input whose transform overflows FP32 reports
+ * NVFP4_ERR_NONFINITE. */
+NVFP4_API nvfp4_status nvfp4_quantize_rht(const void *x, int64_t ld, uint32_t sign_mask,
+                                          const nvfp4_tensor *out, int32_t global_supplied,
+                                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* Same quantization as nvfp4_quantize, for callers that cannot allocate
  * device memory when they quantize: code recorded into a CUDA graph (device
  * allocation cannot be captured), latency-critical paths that cannot afford

@@ -34,7 +34,7 @@ EXPORTED = (
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
-    "nvfp4_quantize_noalloc",
+    "nvfp4_quantize_noalloc", "nvfp4_quantize_rht",
 )
 
 
@@ -80,6 +80,7 @@ def lib() -> C.CDLL:
             "nvfp4_set_wait_limit_cycles": (C.c_longlong, [C.c_longlong]),
             "nvfp4_set_gemm_pairs": (i32, [i32]),
             "nvfp4_quantize_noalloc": (C.c_int, [vp, i64, T, i32, vp]),
+            "nvfp4_quantize_rht": (C.c_int, [vp, i64, C.c_uint32, T, i32, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -191,6 +192,23 @@ def nvfp4_quantize(x: torch.Tensor, out: NVFP4Tensor | None = None, layout: int 
     t = out.c_struct()
     _check(lib().nvfp4_quantize(x.data_ptr(), x.stride(0), C.byref(t), int(global_supplied),
                                 ws.ptr, ws.nbytes, _stream(stream)), "nvfp4_quantize")
+    return out
+
+
+def nvfp4_quantize_rht(x: torch.Tensor, sign_mask: int, out: NVFP4Tensor | None = None,
+                       layout: int = SF_SWIZZLED, global_supplied: bool = False,
+                       workspace: Workspace | None = None, stream=None) -> NVFP4Tensor:
+    """Quantize after the 16x16 random Hadamard transform of every block
+    (``sign_mask`` bit j negates value j of each block before the transform)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out is None:
+        out = NVFP4Tensor.empty(rows, cols, layout, x.device)
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize_rht(x.data_ptr(), x.stride(0), sign_mask, C.byref(t),
+                                    int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
+           "nvfp4_quantize_rht")
     return out
 
 

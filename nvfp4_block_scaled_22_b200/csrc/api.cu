@@ -117,7 +117,7 @@ nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, i
 
 nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32_t *gather,
                         const nvfp4_tensor *out, int32_t global_supplied, void *ws,
-                        cudaStream_t stream, int sms) {
+                        cudaStream_t stream, int sms, bool rht = false, uint32_t rht_mask = 0) {
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kStatusBytes);
     int n_partials = 0;
@@ -126,8 +126,12 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
         int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(warps_needed, 8), 4 * sms),
                                           kMaxPartials);
         if (grid < 1) grid = 1;
-        k_amax<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), ld, out->rows,
-                                         out->cols, gather, src_rows, partials, status);
+        if (rht)
+            k_amax_rht<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), ld, out->rows,
+                                                 out->cols, rht_mask, partials);
+        else
+            k_amax<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), ld, out->rows,
+                                             out->cols, gather, src_rows, partials, status);
         nvfp4_status st = launched(cudaGetLastError());
         if (st != NVFP4_OK) return st;
         n_partials = grid;
@@ -147,11 +151,15 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
     p.partials = partials;
     p.n_partials = n_partials;
     p.status = status;
+    p.rht_mask = rht_mask;
     const int64_t tasks = ceil_div(out->rows, 128) * 128 * ceil_div(ceil_div(out->cols / 16, 4) * 4, 32);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
     int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * 4), 8LL * sms);
     if (grid < 1) grid = 1;
-    k_encode<<<grid, 256, 0, stream>>>(p);
+    if (rht)
+        k_encode_rht<<<grid, 256, 0, stream>>>(p);
+    else
+        k_encode<<<grid, 256, 0, stream>>>(p);
     return launched(cudaGetLastError());
 }
 
@@ -200,6 +208,28 @@ nvfp4_status nvfp4_quantize(const void *x, int64_t ld, const nvfp4_tensor *out,
     if (st != NVFP4_OK) return st;
     return run_encode(x, ld, out->rows, nullptr, out, global_supplied, workspace,
                       static_cast<cudaStream_t>(stream), sms);
+}
+
+nvfp4_status nvfp4_quantize_rht(const void *x, int64_t ld, uint32_t sign_mask,
+                                const nvfp4_tensor *out, int32_t global_supplied, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (sign_mask > 0xFFFFu) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    if (out->rows > 0 && out->cols > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < out->cols) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return run_encode(x, ld, out->rows, nullptr, out, global_supplied, workspace,
+                      static_cast<cudaStream_t>(stream), sms, true, sign_mask);
 }
 
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
@@ -342,6 +372,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.gw = gw;
     p.a_row_blocks = (int32_t)ceil_div(A->rows, 128);
     p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
+    p.n_fastest = (A->rows * (k / 2) > kL2SweepBytes && W->rows * (k / 2) <= kL2SweepBytes) ? 1 : 0;
     p.status = reinterpret_cast<uint32_t *>(workspace);
     p.timeout_cycles = g_timeout_cycles;
     if (pair) {

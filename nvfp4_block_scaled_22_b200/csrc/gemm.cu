@@ -90,11 +90,18 @@ struct TileInfo {
     int row_end;      // first row (exclusive) of real output rows for this tile
 };
 
-__device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, const GemmParams &p,
-                                              const int *s_off, const int *s_rows) {
+// Tile order: M fastest (the CTAs working at one time share a few W
+// column tiles and sweep all of A, which then has to stay in L2), or, when
+// A is too large for that and W is not, N fastest (they share a few A row
+// tiles and sweep all of W).
+__device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, int ntiles,
+                                              const GemmParams &p, const int *s_off,
+                                              const int *s_rows) {
     TileInfo t;
-    t.mt = tile % mtiles;
-    t.nt = tile / mtiles;
+    const int fast = p.n_fastest ? ntiles : mtiles;
+    const int q = tile / fast, r = tile - q * fast;
+    t.mt = p.n_fastest ? q : r;
+    t.nt = p.n_fastest ? r : q;
     t.a_row0 = t.mt * kBM;
     if (p.groups == 0) {
         t.group = 0;
@@ -191,7 +198,7 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             for (int s = 0; s < kStages; ++s) armed[s] = false;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-                const TileInfo t = tile_info(tile, mtiles, p, s_off, s_rows);
+                const TileInfo t = tile_info(tile, mtiles, ntiles, p, s_off, s_rows);
                 const int64_t sfa_base = (int64_t)(t.a_row0 / kBM) * sf_rowblock_bytes;
                 const int brb = t.b_row0 / kBM;
                 const int halves = (brb + 1 < p.b_row_blocks) ? 2 : 1;
@@ -344,27 +351,31 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const int chalf = (warp - kFirstEpiWarp) / 4;          // column half of the tile
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const TileInfo t = tile_info(tile, mtiles, p, s_off, s_rows);
+            // Only alpha is held across the accumulator loads; the tile's
+            // coordinates are derived again for the stores (fewer live
+            // registers next to the 64 output words).
+            const float alpha =
+                __frcp_rn(__fmul_rn(*p.ga, p.gw[tile_info(tile, mtiles, ntiles, p, s_off, s_rows).group]));
             if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
-            const float alpha = __frcp_rn(__fmul_rn(*p.ga, p.gw[t.group]));
             uint32_t o[64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) +
-                                       (uint32_t)(chalf * 128 + 32 * c), r);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                       (uint32_t)(chalf * 128 + 16 * c), r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    o[16 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                    __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                for (int i = 0; i < 8; ++i)
+                    o[8 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                   __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh->acc_empty);    // accumulator free for the next tile
             acc_phase ^= 1;
 
+            const TileInfo t = tile_info(tile, mtiles, ntiles, p, s_off, s_rows);
             // One warp stores its 32 rows x 128 columns; a register transpose
             // makes every store instruction cover one row's 128 bytes.
             const int row0 = t.a_row0 + quarter * 32;

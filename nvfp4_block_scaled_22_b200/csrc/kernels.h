@@ -21,6 +21,7 @@ struct EncodeParams {
     const uint32_t *partials;
     int32_t n_partials;
     uint32_t *status;
+    uint32_t rht_mask = 0;  // random Hadamard transform: sign bit j negates value j of a block
 };
 
 struct DequantParams {
@@ -69,6 +70,7 @@ struct GemmParams {
     const float *gw;          // W tensor scale(s) (device), one per group
     int32_t a_row_blocks;     // ceil(A rows / 128), bounds the grouped slots
     int32_t b_row_blocks;     // ceil(W rows / 128), bounds the SFB reads
+    int32_t n_fastest;        // tile order: 0 = M fastest, 1 = N fastest
     uint32_t *status;
     long long timeout_cycles;
 };
@@ -76,8 +78,11 @@ struct GemmParams {
 __global__ void k_amax(const uint16_t *x, int64_t ld, int64_t rows, int64_t cols,
                        const int32_t *gather, int64_t src_rows, uint32_t *partials,
                        uint32_t *status);
+__global__ void k_amax_rht(const uint16_t *x, int64_t ld, int64_t rows, int64_t cols,
+                           uint32_t rht_mask, uint32_t *partials);
 __global__ void k_finalize_g(const uint32_t *partials, int n, float *global, uint32_t *status);
 __global__ void k_encode(EncodeParams p);
+__global__ void k_encode_rht(EncodeParams p);
 __global__ void k_dequantize(DequantParams p);
 
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
@@ -86,6 +91,10 @@ cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const Ge
 // Dense GEMM on CTA pairs (256x256 tiles); tmB must use 128-row boxes.
 cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                              int clusters, cudaStream_t stream);
+
+// Tile order: N fastest when A's codes exceed this many bytes and W's do
+// not (the operand swept by the CTAs working at one time must stay in L2).
+constexpr int64_t kL2SweepBytes = 48ll << 20;
 
 // Dense GEMMs with at least this many rows run on CTA pairs.
 constexpr int64_t kPairMinRows = 256;

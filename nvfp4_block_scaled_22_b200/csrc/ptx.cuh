@@ -76,6 +76,31 @@ __device__ __forceinline__ uint32_t bf16x2_from_f32(float lo, float hi) {
     return r;
 }
 
+// Packed FP32 pair arithmetic (one instruction for both lanes), each lane
+// one IEEE operation rounded to nearest even, subnormals kept.
+#define NVFP4_F32X2_OP(name, op)                                                          \
+    __device__ __forceinline__ float2 name(float2 a, float2 b) {                         \
+        float2 d;                                                                        \
+        asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\t"                    \
+            "mov.b64 rb, {%4, %5};\n\t" op ".rn.f32x2 rd, ra, rb;\n\t"                    \
+            "mov.b64 {%0, %1}, rd;\n\t}"                                                 \
+            : "=f"(d.x), "=f"(d.y)                                                       \
+            : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));                                   \
+        return d;                                                                        \
+    }
+NVFP4_F32X2_OP(add_f32x2, "add")
+NVFP4_F32X2_OP(sub_f32x2, "sub")
+NVFP4_F32X2_OP(mul_f32x2, "mul")
+#undef NVFP4_F32X2_OP
+
+// max(|a|, |b|) with any NaN operand giving NaN (the sign of the result is
+// the xor of the operands' signs; callers clear it).
+__device__ __forceinline__ float absmax_nan(float a, float b) {
+    float d;
+    asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
 // Lane-wise unsigned 16-bit max of two packed pairs.
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
     uint32_t r;

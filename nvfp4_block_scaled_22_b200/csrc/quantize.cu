@@ -10,8 +10,10 @@
 //
 // Kernels
 //   k_amax        : per-CTA max|x| over whole rows (optionally gathered).
+//   k_amax_rht    : the same over the random-Hadamard-transformed blocks.
 //   k_finalize_g  : partial maxima -> g, error status (nvfp4_global_scale).
-//   k_encode      : g (from partials or supplied) -> codes + scales.
+//   k_encode      : g (from partials or supplied) -> codes + scales; the
+//                   kRht instance transforms each block first.
 //   k_dequantize  : codes + scales + g -> BF16.
 //
 // Work split of k_encode/k_dequantize: a warp takes one row's 512-value
@@ -57,6 +59,68 @@ __device__ __forceinline__ uint32_t block_reduce_max(uint32_t v, uint32_t *red) 
     return v;
 }
 
+// Random Hadamard transform of one 16-value block (same pre-training page,
+// section "Four stabilisation devices"): y = (1/4) H16 diag(s) x, H16 the
+// Sylvester Hadamard matrix, s_j = -1 where bit j of the mask is set.  The
+// sign flips act on the BF16 sign bits (exact); the four butterfly stages
+// run with strides 1, 2, 4, 8 in that order, each add/sub one FP32 RN
+// operation, then an RN multiply by 1/4 -- the evaluation order the
+// quantized result is specified with.
+//
+// Register layout: P[i] = (z_i, z_{i+8}).  Stages 1, 2 and 4 pair P[i]
+// with P[i+h] lane-wise (packed f32x2 add/sub); stage 8 pairs the two
+// lanes of each P[i].  Output y_i is P[i].x, y_{i+8} is P[i].y.
+struct SignFlips {
+    uint32_t w[8];   // XOR mask of BF16 word j (values 2j, 2j+1 of a block)
+};
+
+__device__ __forceinline__ SignFlips sign_flips(uint32_t mask) {
+    SignFlips f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        f.w[j] = (((mask >> (2 * j)) & 1u) << 15) | (((mask >> (2 * j + 1)) & 1u) << 31);
+    return f;
+}
+
+__device__ __forceinline__ void rht16(uint4 a, uint4 b, const SignFlips &f, float2 P[8]) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t v = w[j] ^ f.w[j], u = w[j + 4] ^ f.w[j + 4];
+        P[2 * j] = make_float2(__uint_as_float(v << 16), __uint_as_float(u << 16));
+        P[2 * j + 1] = make_float2(__uint_as_float(v & 0xFFFF0000u), __uint_as_float(u & 0xFFFF0000u));
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if ((i & h) == 0) {
+                const float2 u = P[i], v = P[i + h];
+                P[i] = add_f32x2(u, v);
+                P[i + h] = sub_f32x2(u, v);
+            }
+        }
+    }
+    const float2 q = make_float2(0.25f, 0.25f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float u = P[i].x, v = P[i].y;
+        P[i] = mul_f32x2(make_float2(__fadd_rn(u, v), __fsub_rn(u, v)), q);
+    }
+}
+
+// max |y_i| as f32 bits; Inf and NaN patterns compare above every finite one.
+__device__ __forceinline__ uint32_t abs_max_bits(const float2 P[8]) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = absmax_nan(P[i].x, P[i].y);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = absmax_nan(m[i], m[i + 4]);
+    m[0] = absmax_nan(m[0], m[2]);
+    m[1] = absmax_nan(m[1], m[3]);
+    return __float_as_uint(absmax_nan(m[0], m[1])) & 0x7FFFFFFFu;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- k_amax
@@ -97,6 +161,43 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint16_t *__restrict__ 
         }
     }
     uint32_t v = block_reduce_max(halves_to_f32bits(m), red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = v;
+}
+
+// ------------------------------------------------------------ k_amax_rht
+// One warp per row, one 16-value block per lane (a warp reads 1 KiB
+// contiguous per step); the block is transformed in registers and the max
+// of |y| over the CTA is written as f32 bits, the format k_amax writes.
+__global__ void __launch_bounds__(kThreads) k_amax_rht(const uint16_t *__restrict__ x, int64_t ld,
+                                                       int64_t rows, int64_t cols,
+                                                       uint32_t rht_mask,
+                                                       uint32_t *__restrict__ partials) {
+    __shared__ uint32_t red[kThreads / 32];
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t blocks = cols / 16;
+    const SignFlips f = sign_flips(rht_mask);
+    uint32_t m = 0;
+    for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(x + r * ld);
+        int64_t c = lane;
+        for (; c + 32 < blocks; c += 64) {
+            uint4 a0 = __ldg(p + 2 * c), b0 = __ldg(p + 2 * c + 1);
+            uint4 a1 = __ldg(p + 2 * c + 64), b1 = __ldg(p + 2 * c + 65);
+            float2 y[8];
+            rht16(a0, b0, f, y);
+            m = max(m, abs_max_bits(y));
+            rht16(a1, b1, f, y);
+            m = max(m, abs_max_bits(y));
+        }
+        if (c < blocks) {
+            float2 y[8];
+            rht16(__ldg(p + 2 * c), __ldg(p + 2 * c + 1), f, y);
+            m = max(m, abs_max_bits(y));
+        }
+    }
+    uint32_t v = block_reduce_max(m, red);
     if (threadIdx.x == 0) partials[blockIdx.x] = v;
 }
 
@@ -197,6 +298,27 @@ __device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g
     return o;
 }
 
+// Quantize one 16-value block after the random Hadamard transform: the
+// same steps on the FP32 values y (RN(amax_b / 6) by an IEEE division, as
+// amax_b is no longer a BF16 value).
+__device__ __forceinline__ EncodeBlockOut encode_block_rht(uint4 a, uint4 b, const SignFlips &f,
+                                                           float g, const EncodeTables &tab) {
+    float2 y[8];
+    rht16(a, b, f, y);
+    const uint32_t bits = abs_max_bits(y);
+    float t = __fmul_rn(__fdiv_rn(__uint_as_float(bits), 6.0f), g);
+    uint32_t s = e4m3_from_f32(t);
+    const float e = tab.inv_s[s & 0x7Fu];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = mul_f32x2(y[i], make_float2(e, e));
+    EncodeBlockOut o;   // y_i = y[i].x, y_{i+8} = y[i].y
+    o.codes.x = e2m1x4_from_f32(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
+    o.codes.y = e2m1x4_from_f32(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
+    o.scale = s;
+    o.finite = bits <= 0x7F7FFFFFu;
+    return o;
+}
+
 // Byte offset of scale (row r, scale column c) in either layout.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sf_cols, int64_t col_tiles,
                                              int32_t layout) {
@@ -211,7 +333,6 @@ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sf_co
 // 4j..4j+3 combine them with two shuffles and lane 4j stores the word.
 // Rows past the end of the last 128-row band (swizzled layout) and scale
 // columns past cols/16 up to the next multiple of 4 are written as zero.
-constexpr int kSegValues = 512;
 constexpr int kUnroll = 4;
 
 // Row of flat task t (tasks laid out row-major, segs per row) without a
@@ -223,7 +344,8 @@ __device__ __forceinline__ uint32_t task_row(uint32_t t, uint32_t segs, float in
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
+template <bool kRht>
+__device__ __forceinline__ void encode_body(const EncodeParams &p) {
     __shared__ uint32_t red[kThreads / 32];
     __shared__ EncodeTables tab;
     float g;
@@ -235,6 +357,7 @@ __global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
     }
     fill_tables(tab, g);
     __syncthreads();
+    const SignFlips flips = sign_flips(kRht ? p.rht_mask : 0u);
     const int lane = threadIdx.x & 31;
     const int64_t sf_cols = p.cols / 16;
     const int64_t sf_cols4 = (sf_cols + 3) / 4 * 4;               // padded scale columns
@@ -278,7 +401,8 @@ __global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
             if (t >= tasks) break;                                   // uniform across the warp
             uint32_t s = 0;
             if (has[u]) {
-                EncodeBlockOut o = encode_block(va[u], vb[u], g, tab);
+                EncodeBlockOut o = kRht ? encode_block_rht(va[u], vb[u], flips, g, tab)
+                                        : encode_block(va[u], vb[u], g, tab);
                 finite &= o.finite;
                 s = o.scale;
                 *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;
@@ -300,6 +424,10 @@ __global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
     }
     if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
 }
+
+__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) { encode_body<false>(p); }
+
+__global__ void __launch_bounds__(kThreads, 3) k_encode_rht(EncodeParams p) { encode_body<true>(p); }
 
 // ----------------------------------------------------------- k_dequantize
 __device__ __forceinline__ void decode_block(uint2 codes, float d, uint4 &o0, uint4 &o1) {

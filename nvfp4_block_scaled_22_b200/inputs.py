@@ -19,6 +19,11 @@ which ships weights here):
   N(0,1)), hidden 6144, expert intermediate 2048.
 * ``kv``        -- KV cache, 32 layers x {K,V} x [131072 tokens x 8 heads x
   128], N(0,1) with 5 of the 1024 (head, dim) channels x10.
+* ``wgrad``     -- weight-gradient GEMM inputs of the same FFN linear, laid
+  out with the token axis contiguous (the contraction axis of the Wgrad
+  GEMM): dY^T 20480 x M with N(0,1) * 2^-10 entries and 0.1% x50, X^T
+  5120 x M (the ffn activation, transposed); plus the random 16-bit sign
+  mask of the Hadamard transform applied to both before quantization.
 
 Every draw is keyed by ``seed_for(workload, stream)``; a tensor drawn on a
 given device type is the same on every call.  CPU and CUDA generators give
@@ -31,7 +36,7 @@ import math
 import torch
 
 SEED_BASE = 0x4E5646
-WORKLOADS = ("tiny", "sweep", "ffn", "moe", "kv")
+WORKLOADS = ("tiny", "sweep", "ffn", "moe", "kv", "wgrad")
 
 # The seven nonzero E2M1 magnitudes, used only to plant "exactly
 # representable" inputs in the sweep workload (the format's value list is
@@ -223,3 +228,30 @@ def kv_tensor(layer: int, kv: int, device="cpu", tokens: int = KV_TOKENS) -> tor
     x = _randn((tokens, KV_HEADS * KV_HEAD_DIM), g, device)
     x[:, kv_outlier_channels(layer, kv).to(device)] *= 10.0
     return x.view(tokens, KV_HEADS, KV_HEAD_DIM).to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------
+# wgrad: inputs of the weight-gradient GEMM dW = dY^T X of the FFN linear
+# --------------------------------------------------------------------------
+WGRAD_M = 8192
+
+
+def rht_sign_mask(stream: int = 0) -> int:
+    """The random +-1 sign vector of the 16x16 Hadamard transform as a
+    16-bit mask (bit j set = value j of a block negated), one per draw."""
+    g = _gen("wgrad", 100 + stream, "cpu")
+    return int(torch.randint(0, 1 << 16, (1,), generator=g).item())
+
+
+def wgrad_grad_output_t(m: int = WGRAD_M, device="cpu", n: int = FFN_N) -> torch.Tensor:
+    """dY^T [n x m] BF16: N(0,1) * 2^-10, 0.1% of the entries x50."""
+    g = _gen("wgrad", 1 + m, device)
+    x = _randn((n * m,), g, device) * 2.0 ** -10
+    idx = _pick(n * m, round(0.001 * n * m), g, device, replace=n * m > (1 << 22))
+    x[idx] *= 50.0
+    return x.view(n, m).to(torch.bfloat16)
+
+
+def wgrad_activation_t(m: int = WGRAD_M, device="cpu", k: int = FFN_K) -> torch.Tensor:
+    """X^T [k x m] BF16: the ffn activation of m tokens, transposed."""
+    return ffn_activation(m, device, k).t().contiguous()

@@ -64,6 +64,10 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     t = binding.CTensor(16, 16, 16, 4, 32, 0)
     assert lib.nvfp4_quantize(8, 32, t, 0, 16, 1 << 16, 0) == 2   # x misaligned
     assert lib.nvfp4_quantize(16, 32, t, 0, 16, 8, 0) == 6        # workspace too small
+    t = binding.CTensor(16, 16, 16, 4, 32, 0)
+    assert lib.nvfp4_quantize_rht(16, 32, 0x10000, t, 0, 16, 1 << 16, 0) == 1   # mask > 16 bits
+    t = binding.CTensor(16, 16, 16, 4, 24, 0)
+    assert lib.nvfp4_quantize_rht(16, 32, 0xFFFF, t, 0, 16, 1 << 16, 0) == 3    # cols % 16
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
