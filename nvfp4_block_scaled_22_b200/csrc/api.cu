@@ -152,14 +152,14 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
     p.n_partials = n_partials;
     p.status = status;
     p.rht_mask = rht_mask;
-    const int64_t tasks = ceil_div(out->rows, 128) * 128 * ceil_div(ceil_div(out->cols / 16, 4) * 4, 32);
+    const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * 4), 8LL * sms);
+    const bool narrow = tasks_are_groups(out->cols);
+    void (*kernel)(EncodeParams) = rht ? (narrow ? k_encode_rht_narrow : k_encode_rht)
+                                       : (narrow ? k_encode_narrow : k_encode);
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms);
     if (grid < 1) grid = 1;
-    if (rht)
-        k_encode_rht<<<grid, 256, 0, stream>>>(p);
-    else
-        k_encode<<<grid, 256, 0, stream>>>(p);
+    kernel<<<grid, 256, 0, stream>>>(p);
     return launched(cudaGetLastError());
 }
 
@@ -307,11 +307,13 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     p.cols = in->cols;
     p.y = static_cast<uint16_t *>(y);
     p.ld = ld;
-    const int64_t tasks = in->rows * ceil_div(in->cols / 16, 32);
+    const int64_t tasks = decode_tasks(in->rows, in->cols);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * 4), 8LL * sms);
+    const bool narrow = tasks_are_groups(in->cols);
+    void (*kernel)(DequantParams) = narrow ? k_dequantize_narrow : k_dequantize;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms);
     if (grid < 1) grid = 1;
-    k_dequantize<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return launched(cudaGetLastError());
 }
 

@@ -24,6 +24,32 @@ struct EncodeParams {
     uint32_t rht_mask = 0;  // random Hadamard transform: sign bit j negates value j of a block
 };
 
+// Quantize / dequantize work unit: one row and kChunkBlocks consecutive
+// 16-value blocks of it per warp task.
+constexpr int kChunkBlocks = 128;
+
+// Warp tasks of the encode kernel (rows padded to 128 in the swizzled
+// layout; scale columns padded to a multiple of 4): rows of at least
+// kChunkBlocks blocks split into chunks of kChunkBlocks, narrower rows into
+// 32-block groups.
+inline int64_t encode_tasks(int64_t rows, int64_t cols, int32_t layout) {
+    const int64_t rows_out = (layout == 0) ? (rows + 127) / 128 * 128 : rows;
+    const int64_t groups = ((cols / 16 + 3) / 4 * 4 + 31) / 32;
+    return rows_out * (groups >= kChunkBlocks / 32 ? (groups + 3) / 4 : groups);
+}
+
+// True when rows are split into 32-block groups (a warp then takes four
+// tasks per pass) rather than chunks.
+inline bool tasks_are_groups(int64_t cols) {
+    return ((cols / 16 + 3) / 4 * 4 + 31) / 32 < kChunkBlocks / 32;
+}
+
+// Warp tasks of the dequantize kernel (same split, unpadded).
+inline int64_t decode_tasks(int64_t rows, int64_t cols) {
+    const int64_t groups = (cols / 16 + 31) / 32;
+    return rows * (groups >= kChunkBlocks / 32 ? (groups + 3) / 4 : groups);
+}
+
 struct DequantParams {
     const uint8_t *codes;
     const uint8_t *scales;
@@ -82,8 +108,11 @@ __global__ void k_amax_rht(const uint16_t *x, int64_t ld, int64_t rows, int64_t 
                            uint32_t rht_mask, uint32_t *partials);
 __global__ void k_finalize_g(const uint32_t *partials, int n, float *global, uint32_t *status);
 __global__ void k_encode(EncodeParams p);
+__global__ void k_encode_narrow(EncodeParams p);
 __global__ void k_encode_rht(EncodeParams p);
+__global__ void k_encode_rht_narrow(EncodeParams p);
 __global__ void k_dequantize(DequantParams p);
+__global__ void k_dequantize_narrow(DequantParams p);
 
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t stream);

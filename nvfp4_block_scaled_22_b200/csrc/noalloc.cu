@@ -128,10 +128,13 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t ld, const 
     p.partials = partials;
     p.n_partials = n_partials;
     p.status = status;
-    const int64_t tasks = ceil_div64(out->rows, 128) * 128 * ceil_div64(ceil_div64(out->cols / 16, 4) * 4, 32);
+    const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(tasks, 8 * 4), 8LL * sms));
-    k_encode<<<grid, 256, 0, s>>>(p);
+    const bool narrow = tasks_are_groups(out->cols);
+    void (*kernel)(EncodeParams) = narrow ? k_encode_narrow : k_encode;
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div64(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms));
+    kernel<<<grid, 256, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     k_status_to_global<<<1, 32, 0, s>>>(status, out->global);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;

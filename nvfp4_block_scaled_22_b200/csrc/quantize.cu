@@ -70,15 +70,22 @@ __device__ __forceinline__ uint32_t block_reduce_max(uint32_t v, uint32_t *red) 
 // Register layout: P[i] = (z_i, z_{i+8}).  Stages 1, 2 and 4 pair P[i]
 // with P[i+h] lane-wise (packed f32x2 add/sub); stage 8 pairs the two
 // lanes of each P[i].  Output y_i is P[i].x, y_{i+8} is P[i].y.
+// Value 2j of a block is the low half of BF16 word j, value 2j + 1 the
+// high half.  As an FP32 bit pattern the low value is w << 16 and the high
+// one w & 0xFFFF0000; its sign flip is bit 31 of that pattern, applied to
+// the low value by adding 2^31 (mod 2^32, the same as flipping the bit) to
+// w * 2^16 and to the high value by an XOR before the mask.
 struct SignFlips {
-    uint32_t w[8];   // XOR mask of BF16 word j (values 2j, 2j+1 of a block)
+    uint32_t lo[8], hi[8];   // 0 or 0x80000000 for values 2j and 2j + 1
 };
 
 __device__ __forceinline__ SignFlips sign_flips(uint32_t mask) {
     SignFlips f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        f.w[j] = (((mask >> (2 * j)) & 1u) << 15) | (((mask >> (2 * j + 1)) & 1u) << 31);
+    for (int j = 0; j < 8; ++j) {
+        f.lo[j] = ((mask >> (2 * j)) & 1u) << 31;
+        f.hi[j] = ((mask >> (2 * j + 1)) & 1u) << 31;
+    }
     return f;
 }
 
@@ -86,9 +93,11 @@ __device__ __forceinline__ void rht16(uint4 a, uint4 b, const SignFlips &f, floa
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const uint32_t v = w[j] ^ f.w[j], u = w[j + 4] ^ f.w[j + 4];
-        P[2 * j] = make_float2(__uint_as_float(v << 16), __uint_as_float(u << 16));
-        P[2 * j + 1] = make_float2(__uint_as_float(v & 0xFFFF0000u), __uint_as_float(u & 0xFFFF0000u));
+        const uint32_t v = w[j], u = w[j + 4];
+        P[2 * j] = make_float2(__uint_as_float(v * 65536u + f.lo[j]),
+                               __uint_as_float(u * 65536u + f.lo[j + 4]));
+        P[2 * j + 1] = make_float2(__uint_as_float((v ^ f.hi[j]) & 0xFFFF0000u),
+                                   __uint_as_float((u ^ f.hi[j + 4]) & 0xFFFF0000u));
     }
 #pragma unroll
     for (int h = 1; h < 8; h <<= 1) {
@@ -298,15 +307,30 @@ __device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g
     return o;
 }
 
+// RN(a / 6) for an FP32 a >= 0.  While the quotient is a normal number
+// (a >= 1.5 * 2^-124) it is q = RN(a * RN(1/6)) corrected once with the
+// exact remainder a - 6q from a fused multiply-add (Markstein's FMA
+// correction step, "IA-64 and Elementary Functions", 2000); checked equal
+// to the IEEE division on every such input.  Smaller, non-finite and NaN
+// inputs take the division.
+__device__ __forceinline__ float div6_f32(float a) {
+    if (a >= 0x1.8p-124f && a <= 0x1.fffffep127f) {
+        const float c = 0x1.555556p-3f;     // RN(1/6)
+        const float q = __fmul_rn(a, c);
+        return __fmaf_rn(__fmaf_rn(-6.0f, q, a), c, q);
+    }
+    return __fdiv_rn(a, 6.0f);
+}
+
 // Quantize one 16-value block after the random Hadamard transform: the
-// same steps on the FP32 values y (RN(amax_b / 6) by an IEEE division, as
-// amax_b is no longer a BF16 value).
+// same steps on the FP32 values y (amax_b is no longer a BF16 value, so
+// RN(amax_b / 6) comes from div6_f32, not the BF16 table).
 __device__ __forceinline__ EncodeBlockOut encode_block_rht(uint4 a, uint4 b, const SignFlips &f,
                                                            float g, const EncodeTables &tab) {
     float2 y[8];
     rht16(a, b, f, y);
     const uint32_t bits = abs_max_bits(y);
-    float t = __fmul_rn(__fdiv_rn(__uint_as_float(bits), 6.0f), g);
+    float t = __fmul_rn(div6_f32(__uint_as_float(bits)), g);
     uint32_t s = e4m3_from_f32(t);
     const float e = tab.inv_s[s & 0x7Fu];
 #pragma unroll
@@ -326,14 +350,17 @@ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sf_co
     return ((r >> 7) * col_tiles + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
 }
 
-// Work split: a task is one row and one 512-value segment of it; lane l
-// owns 16-value block l of the segment (two 16-byte loads, one 8-byte code
-// store), so a warp's loads and stores are contiguous.  The four scale
-// bytes of blocks 4j..4j+3 are contiguous in both scale layouts; lanes
-// 4j..4j+3 combine them with two shuffles and lane 4j stores the word.
-// Rows past the end of the last 128-row band (swizzled layout) and scale
-// columns past cols/16 up to the next multiple of 4 are written as zero.
-constexpr int kUnroll = 4;
+// Work split: a task is one row and one chunk of kChunkBlocks = 128
+// consecutive 16-value blocks (2048 values) of it; lane l owns blocks
+// l, l + 32, l + 64, l + 96 of the chunk (two 16-byte loads and one 8-byte
+// code store each), so every load and store instruction of a warp is
+// contiguous, and the row's addresses are formed once per task.  The four
+// scale bytes of blocks 4i..4i+3 are contiguous in both scale layouts;
+// lanes 4i..4i+3 combine them with two shuffles and lane 4i stores the
+// word.  Rows past the end of the last 128-row band (swizzled layout) and
+// scale columns past cols/16 up to the next multiple of 4 are written as
+// zero.
+constexpr int kUnroll = kChunkBlocks / 32;
 
 // Row of flat task t (tasks laid out row-major, segs per row) without a
 // 64-bit division: float reciprocal, then exact integer correction.
@@ -344,7 +371,80 @@ __device__ __forceinline__ uint32_t task_row(uint32_t t, uint32_t segs, float in
     return r;
 }
 
+// The tasks a warp takes, t, t + stride, t + 2 stride, ..., as (row,
+// chunk) pairs of the row-major task grid (chunks per row): one division
+// for the first task, then an add with carry per step.
+struct TaskWalk {
+    uint32_t row, seg, segs, step_rows, step_segs;
+    __device__ __forceinline__ TaskWalk(uint32_t t, uint32_t stride, uint32_t segs_)
+        : row(t / segs_), seg(t - (t / segs_) * segs_), segs(segs_), step_rows(stride / segs_),
+          step_segs(stride - (stride / segs_) * segs_) {}
+    __device__ __forceinline__ void next() {
+        seg += step_segs;
+        row += step_rows;
+        if (seg >= segs) {
+            seg -= segs;
+            ++row;
+        }
+    }
+};
+
+// Shape constants of one encode launch.
+struct EncodeShape {
+    int64_t sf_cols, sf_cols4, col_tiles, rows_out, sf_step;
+};
+
+// Block column c of one row: quantize it (or write zero codes for a
+// gathered padding row), store its codes at cp, and let lanes 4i store the
+// scale word of blocks 4i..4i+3 at sp.  Every lane of the warp takes part
+// (two shuffles).
 template <bool kRht>
+__device__ __forceinline__ void emit_block(const EncodeParams &p, const EncodeShape &sh,
+                                           const SignFlips &flips, float g, const EncodeTables &tab,
+                                           bool real, bool load, int64_t c, uint4 a, uint4 b,
+                                           uint2 *cp, uint8_t *sp, int lane, bool &finite) {
+    uint32_t s = 0;
+    if (real && c < sh.sf_cols) {
+        if (load) {
+            EncodeBlockOut o = kRht ? encode_block_rht(a, b, flips, g, tab) : encode_block(a, b, g, tab);
+            finite &= o.finite;
+            s = o.scale;
+            *cp = o.codes;
+        } else {                                                      // gathered padding row
+            *cp = make_uint2(0, 0);
+        }
+    }
+    uint32_t word = s << (8 * (lane & 3));
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+    if ((lane & 3) == 0 && c < sh.sf_cols4 && (p.layout == 0 || c < sh.sf_cols)) {
+        if (p.layout == 0 || ((sh.sf_cols & 3) == 0 && c + 4 <= sh.sf_cols)) {
+            *reinterpret_cast<uint32_t *>(sp) = word;
+        } else {                                                      // ragged linear row
+            for (int i = 0; i < 4 && c + i < sh.sf_cols; ++i) sp[i] = (uint8_t)(word >> (8 * i));
+        }
+    }
+}
+
+// Source row of output row `row` (gathered or not); load = false for band
+// padding rows, gathered padding rows (-1) and invalid map entries.
+__device__ __forceinline__ int64_t source_row(const EncodeParams &p, int64_t row, bool &real,
+                                              bool &load) {
+    real = row < p.rows;
+    load = real;
+    int64_t src = row;
+    if (real && p.gather != nullptr) {
+        src = p.gather[row];
+        if (src >= p.src_rows) {             // out-of-range map entry: zero row + status
+            set_status(p.status, ST_INVALID_ARG);
+            src = -1;
+        }
+        load = src >= 0;
+    }
+    return load ? src : 0;
+}
+
+template <bool kRht, bool kNarrow>
 __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     __shared__ uint32_t red[kThreads / 32];
     __shared__ EncodeTables tab;
@@ -359,65 +459,102 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     __syncthreads();
     const SignFlips flips = sign_flips(kRht ? p.rht_mask : 0u);
     const int lane = threadIdx.x & 31;
-    const int64_t sf_cols = p.cols / 16;
-    const int64_t sf_cols4 = (sf_cols + 3) / 4 * 4;               // padded scale columns
-    const int64_t col_tiles = sf_cols4 / 4;
-    const int64_t segs = (sf_cols4 + 31) / 32;                    // 32 blocks per segment
-    const int64_t rows_out = (p.layout == 0) ? (p.rows + 127) / 128 * 128 : p.rows;
-    const uint32_t tasks = (uint32_t)(rows_out * segs);        // < 2^32 (host-checked)
+    EncodeShape sh;
+    sh.sf_cols = p.cols / 16;
+    sh.sf_cols4 = (sh.sf_cols + 3) / 4 * 4;                        // padded scale columns
+    sh.col_tiles = sh.sf_cols4 / 4;
+    sh.rows_out = (p.layout == 0) ? (p.rows + 127) / 128 * 128 : p.rows;
+    sh.sf_step = (p.layout == 0) ? 4096 : 32;                      // scale bytes per 32 blocks
+    const uint32_t groups = (uint32_t)((sh.sf_cols4 + 31) / 32);   // 32-block groups per row
     const uint32_t warps = gridDim.x * (kThreads / 32);
-    const float inv_segs = 1.0f / (float)segs;
+    const uint32_t warp_id = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    if (groups == 0) return;                                       // no columns
     bool finite = true;
-    for (uint32_t t0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t0 < tasks;
-         t0 += warps * kUnroll) {
-        uint4 va[kUnroll], vb[kUnroll];
-        int64_t rr[kUnroll], bb[kUnroll];
-        bool has[kUnroll];
+    if (!kNarrow) {
+        // Wide rows: a task is kChunkBlocks consecutive blocks of one row,
+        // lane l taking blocks l, l+32, l+64, l+96; addresses once per task.
+        const uint32_t chunks = (groups + kUnroll - 1) / kUnroll;
+        for (TaskWalk w(warp_id, warps, chunks); w.row < sh.rows_out; w.next()) {
+            const int64_t row = w.row;
+            const int64_t c0 = (int64_t)w.seg * kChunkBlocks + lane;   // this lane's first block
+            bool real, load;
+            const int64_t src = source_row(p, row, real, load);
+            const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + src * p.ld + c0 * 16);
+            uint4 va[kUnroll], vb[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t t = t0 + warps * u;
-            const uint32_t row = task_row(t, (uint32_t)segs, inv_segs);
-            rr[u] = row;
-            bb[u] = (int64_t)(t - row * (uint32_t)segs) * 32 + lane;   // scale column of this lane
-            int64_t src = rr[u];
-            has[u] = t < tasks && rr[u] < p.rows && bb[u] < sf_cols;
-            if (has[u] && p.gather != nullptr) {
-                src = p.gather[rr[u]];
-                if (src >= p.src_rows) {     // out-of-range map entry: zero row + status
-                    set_status(p.status, ST_INVALID_ARG);
-                    src = -1;
+            for (int j = 0; j < kUnroll; ++j) {
+                if (load && c0 + 32 * j < sh.sf_cols) {
+                    va[j] = __ldg(xp + 64 * j);
+                    vb[j] = __ldg(xp + 64 * j + 1);
                 }
-                if (src < 0) has[u] = false;
             }
-            if (has[u]) {
-                const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + src * p.ld + bb[u] * 16);
-                va[u] = __ldg(xp);
-                vb[u] = __ldg(xp + 1);
+            uint2 *cp = reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + c0 * 8);
+            uint8_t *sp = p.scales + sf_offset(row, c0, sh.sf_cols, sh.col_tiles, p.layout);
+#pragma unroll
+            for (int j = 0; j < kUnroll; ++j) {
+                if (c0 - lane + 32 * j >= sh.sf_cols4) break;           // uniform across the warp
+                emit_block<kRht>(p, sh, flips, g, tab, real, load, c0 + 32 * j, va[j], vb[j],
+                                 cp + 32 * j, sp + sh.sf_step * j, lane, finite);
             }
         }
+    } else {
+        // Narrow rows (fewer than 128 blocks): a task is one 32-block group
+        // of one row (lane l owns block l); a warp keeps kUnroll tasks in
+        // flight, tasks t0, t0 + warps, ... of the row-major task grid.
+        const uint32_t tasks = (uint32_t)(sh.rows_out * groups);   // < 2^32 (host-checked)
+        const float inv_groups = 1.0f / (float)groups;
+        for (uint32_t t0 = warp_id; t0 < tasks; t0 += warps * kUnroll) {
+            uint4 va[kUnroll], vb[kUnroll];
+            int64_t rr[kUnroll], bb[kUnroll];
+            bool has[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t t = t0 + warps * u;
-            if (t >= tasks) break;                                   // uniform across the warp
-            uint32_t s = 0;
-            if (has[u]) {
-                EncodeBlockOut o = kRht ? encode_block_rht(va[u], vb[u], flips, g, tab)
-                                        : encode_block(va[u], vb[u], g, tab);
-                finite &= o.finite;
-                s = o.scale;
-                *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;
-            } else if (rr[u] < p.rows && bb[u] < sf_cols) {          // gathered padding row
-                *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = make_uint2(0, 0);
+            for (int u = 0; u < kUnroll; ++u) {
+                const uint32_t t = t0 + warps * u;
+                const uint32_t row = task_row(t, groups, inv_groups);
+                rr[u] = row;
+                bb[u] = (int64_t)(t - row * groups) * 32 + lane;   // scale column of this lane
+                int64_t src = rr[u];
+                has[u] = t < tasks && rr[u] < p.rows && bb[u] < sh.sf_cols;
+                if (has[u] && p.gather != nullptr) {
+                    src = p.gather[rr[u]];
+                    if (src >= p.src_rows) {     // out-of-range map entry: zero row + status
+                        set_status(p.status, ST_INVALID_ARG);
+                        src = -1;
+                    }
+                    if (src < 0) has[u] = false;
+                }
+                if (has[u]) {
+                    const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + src * p.ld + bb[u] * 16);
+                    va[u] = __ldg(xp);
+                    vb[u] = __ldg(xp + 1);
+                }
             }
-            uint32_t w = s << (8 * (lane & 3));
-            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-            if ((lane & 3) == 0 && bb[u] < sf_cols4 && (p.layout == 0 || bb[u] < sf_cols)) {
-                uint8_t *sp = p.scales + sf_offset(rr[u], bb[u], sf_cols, col_tiles, p.layout);
-                if (p.layout == 0 || ((sf_cols & 3) == 0 && bb[u] + 4 <= sf_cols)) {
-                    *reinterpret_cast<uint32_t *>(sp) = w;
-                } else {                                             // ragged linear row
-                    for (int j = 0; j < 4 && bb[u] + j < sf_cols; ++j) sp[j] = (uint8_t)(w >> (8 * j));
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const uint32_t t = t0 + warps * u;
+                if (t >= tasks) break;                               // uniform across the warp
+                uint32_t s = 0;
+                if (has[u]) {
+                    EncodeBlockOut o = kRht ? encode_block_rht(va[u], vb[u], flips, g, tab)
+                                            : encode_block(va[u], vb[u], g, tab);
+                    finite &= o.finite;
+                    s = o.scale;
+                    *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;
+                } else if (rr[u] < p.rows && bb[u] < sh.sf_cols) {      // gathered padding row
+                    *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) =
+                        make_uint2(0, 0);
+                }
+                uint32_t w = s << (8 * (lane & 3));
+                w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+                w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+                if ((lane & 3) == 0 && bb[u] < sh.sf_cols4 && (p.layout == 0 || bb[u] < sh.sf_cols)) {
+                    uint8_t *sp = p.scales + sf_offset(rr[u], bb[u], sh.sf_cols, sh.col_tiles, p.layout);
+                    if (p.layout == 0 || ((sh.sf_cols & 3) == 0 && bb[u] + 4 <= sh.sf_cols)) {
+                        *reinterpret_cast<uint32_t *>(sp) = w;
+                    } else {                                         // ragged linear row
+                        for (int j = 0; j < 4 && bb[u] + j < sh.sf_cols; ++j)
+                            sp[j] = (uint8_t)(w >> (8 * j));
+                    }
                 }
             }
         }
@@ -425,9 +562,21 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
 }
 
-__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) { encode_body<false>(p); }
+// The host launches the *_narrow kernels for rows of fewer than
+// kChunkBlocks blocks (tasks_are_groups).
+__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) { encode_body<false, false>(p); }
 
-__global__ void __launch_bounds__(kThreads, 3) k_encode_rht(EncodeParams p) { encode_body<true>(p); }
+__global__ void __launch_bounds__(kThreads) k_encode_narrow(EncodeParams p) {
+    encode_body<false, true>(p);
+}
+
+__global__ void __launch_bounds__(kThreads, 3) k_encode_rht(EncodeParams p) {
+    encode_body<true, false>(p);
+}
+
+__global__ void __launch_bounds__(kThreads, 3) k_encode_rht_narrow(EncodeParams p) {
+    encode_body<true, true>(p);
+}
 
 // ----------------------------------------------------------- k_dequantize
 __device__ __forceinline__ void decode_block(uint2 codes, float d, uint4 &o0, uint4 &o1) {
@@ -445,44 +594,92 @@ __device__ __forceinline__ void decode_block(uint2 codes, float d, uint4 &o0, ui
     o1 = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
-__global__ void __launch_bounds__(kThreads) k_dequantize(DequantParams p) {
+template <bool kNarrow>
+__device__ __forceinline__ void dequantize_body(const DequantParams &p) {
+    // Wide rows: d = RN(f32(s) / g) for each of the 128 non-negative E4M3
+    // codes s (stored scales are never negative), one table per CTA; narrow
+    // rows divide per block.
+    __shared__ float dtab[128];
     const float g = *p.global;
+    if (!kNarrow) {
+        for (int i = threadIdx.x; i < 128; i += blockDim.x)
+            dtab[i] = __fdiv_rn(f32_from_e4m3((uint32_t)i), g);
+        __syncthreads();
+    }
     const int lane = threadIdx.x & 31;
     const int64_t sf_cols = p.cols / 16;
     const int64_t col_tiles = (sf_cols + 3) / 4;
-    const int64_t segs = (sf_cols + 31) / 32;
-    const uint32_t tasks = (uint32_t)(p.rows * segs);          // < 2^32 (host-checked)
+    const uint32_t groups = (uint32_t)((sf_cols + 31) / 32);
     const uint32_t warps = gridDim.x * (kThreads / 32);
-    const float inv_segs = 1.0f / (float)segs;
-    for (uint32_t t0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t0 < tasks;
-         t0 += warps * kUnroll) {
-        uint2 c[kUnroll];
-        uint32_t sb[kUnroll];
-        int64_t rr[kUnroll], bb[kUnroll];
-        bool has[kUnroll];
+    const uint32_t warp_id = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int64_t sf_step = (p.layout == 0) ? 4096 : 32;         // scale bytes per 32 blocks
+    if (groups == 0) return;                                      // no columns
+    if (!kNarrow) {
+        // Wide rows: kChunkBlocks blocks of one row per task (as in k_encode).
+        const uint32_t chunks = (groups + kUnroll - 1) / kUnroll;
+        for (TaskWalk w(warp_id, warps, chunks); w.row < p.rows; w.next()) {
+            const int64_t row = w.row;
+            const int64_t c0 = (int64_t)w.seg * kChunkBlocks + lane;
+            const uint2 *cp = reinterpret_cast<const uint2 *>(p.codes + row * (p.cols / 2) + c0 * 8);
+            const uint8_t *sp = p.scales + sf_offset(row, c0, sf_cols, col_tiles, p.layout);
+            uint2 c[kUnroll];
+            uint32_t sb[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t t = t0 + warps * u;
-            const uint32_t row = task_row(t, (uint32_t)segs, inv_segs);
-            rr[u] = row;
-            bb[u] = (int64_t)(t - row * (uint32_t)segs) * 32 + lane;
-            has[u] = t < tasks && bb[u] < sf_cols;
-            if (has[u]) {
-                c[u] = __ldg(reinterpret_cast<const uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8));
-                sb[u] = __ldg(p.scales + sf_offset(rr[u], bb[u], sf_cols, col_tiles, p.layout));
+            for (int j = 0; j < kUnroll; ++j) {
+                if (c0 + 32 * j < sf_cols) {
+                    c[j] = __ldg(cp + 32 * j);
+                    sb[j] = __ldg(sp + sf_step * j);
+                }
+            }
+            uint4 *yp = reinterpret_cast<uint4 *>(p.y + row * p.ld + c0 * 16);
+#pragma unroll
+            for (int j = 0; j < kUnroll; ++j) {
+                if (c0 + 32 * j >= sf_cols) continue;
+                uint4 o0, o1;
+                decode_block(c[j], dtab[sb[j] & 0x7Fu], o0, o1);
+                yp[64 * j] = o0;
+                yp[64 * j + 1] = o1;
             }
         }
+    } else {
+        // Narrow rows: one 32-block group per task, kUnroll tasks in flight.
+        const uint32_t tasks = (uint32_t)(p.rows * groups);       // < 2^32 (host-checked)
+        const float inv_groups = 1.0f / (float)groups;
+        for (uint32_t t0 = warp_id; t0 < tasks; t0 += warps * kUnroll) {
+            uint2 c[kUnroll];
+            uint32_t sb[kUnroll];
+            int64_t rr[kUnroll], bb[kUnroll];
+            bool has[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (!has[u]) continue;
-            const float d = __fdiv_rn(f32_from_e4m3(sb[u]), g);
-            uint4 o0, o1;
-            decode_block(c[u], d, o0, o1);
-            uint4 *yp = reinterpret_cast<uint4 *>(p.y + rr[u] * p.ld + bb[u] * 16);
-            yp[0] = o0;
-            yp[1] = o1;
+            for (int u = 0; u < kUnroll; ++u) {
+                const uint32_t t = t0 + warps * u;
+                const uint32_t row = task_row(t, groups, inv_groups);
+                rr[u] = row;
+                bb[u] = (int64_t)(t - row * groups) * 32 + lane;
+                has[u] = t < tasks && bb[u] < sf_cols;
+                if (has[u]) {
+                    c[u] = __ldg(reinterpret_cast<const uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8));
+                    sb[u] = __ldg(p.scales + sf_offset(rr[u], bb[u], sf_cols, col_tiles, p.layout));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (!has[u]) continue;
+                const float d = __fdiv_rn(f32_from_e4m3(sb[u]), g);
+                uint4 o0, o1;
+                decode_block(c[u], d, o0, o1);
+                uint4 *yp = reinterpret_cast<uint4 *>(p.y + rr[u] * p.ld + bb[u] * 16);
+                yp[0] = o0;
+                yp[1] = o1;
+            }
         }
     }
+}
+
+__global__ void __launch_bounds__(kThreads) k_dequantize(DequantParams p) { dequantize_body<false>(p); }
+
+__global__ void __launch_bounds__(kThreads) k_dequantize_narrow(DequantParams p) {
+    dequantize_body<true>(p);
 }
 
 }  // namespace nvfp4

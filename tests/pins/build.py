@@ -5,7 +5,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 LIB = os.path.join(HERE, "libpins.so")
-SRCS = [os.path.join(HERE, "exhaustive.c"), os.path.join(ROOT, "oracle", "nvfp4_oracle.c")]
+SRCS = [os.path.join(HERE, "exhaustive.c"), os.path.join(HERE, "kernel_shortcuts.c"),
+        os.path.join(ROOT, "oracle", "nvfp4_oracle.c")]
 
 
 def build():
