@@ -490,10 +490,13 @@ def workload_line(name, args, device):
                                   "peak_source": f"{peak_src} hbm_gbs"}})
         return line
     if name == "wgrad":
+        # dW = dY^T X from the forward layouts dY [M x N], X [M x K]: both
+        # operands quantized column-wise with the 16x16 Hadamard transform.
         m = inputs.WGRAD_M
         mask = inputs.rht_sign_mask(0)
         dy_t = inputs.wgrad_grad_output_t(m, device=device)
         x_t = inputs.wgrad_activation_t(m, device=device)
+        dy, x = dy_t.t().contiguous(), x_t.t().contiguous()
         qa = nb.NVFP4Tensor.empty(N, m, device=device)
         qw = nb.NVFP4Tensor.empty(K, m, device=device)
         d = torch.empty((N, K), dtype=torch.bfloat16, device=device)
@@ -502,10 +505,10 @@ def workload_line(name, args, device):
         def step(mark=False):
             if mark:
                 ev["a"].record()
-            nb.nvfp4_quantize_rht(dy_t, mask, out=qa, workspace=ws)
+            nb.nvfp4_quantize_t(dy, out=qa, sign_mask=mask, workspace=ws)
             if mark:
                 ev["b"].record()
-            nb.nvfp4_quantize_rht(x_t, mask, out=qw, workspace=ws)
+            nb.nvfp4_quantize_t(x, out=qw, sign_mask=mask, workspace=ws)
             if mark:
                 ev["c"].record()
             nb.nvfp4_gemm(qa, qw, out=d, workspace=ws)
@@ -522,20 +525,28 @@ def workload_line(name, args, device):
             qw_ms.append(ev["b"].elapsed_time(ev["c"]))
             g_ms.append(ev["c"].elapsed_time(ev["d"]))
         qa_ms, qw_ms, g_ms = (statistics.median(v) for v in (qa_ms, qw_ms, g_ms))
+        # the same operand quantized row-wise from an explicit dY^T
+        rw_ms = _timed(lambda: nb.nvfp4_quantize_rht(dy_t, mask, out=qa, workspace=ws),
+                       args.steps, args.warmup, flush)
+        # column-wise without the transform
+        cw_ms = _timed(lambda: nb.nvfp4_quantize_t(dy, out=qa, workspace=ws),
+                       args.steps, args.warmup, flush)
         st = nb.nvfp4_check_status(ws)
         flops = 2.0 * N * K * m
-        qgbs = N * m * QUANT_BYTES_PER_VALUE_2PASS / qa_ms / 1e6
-        line.update({"metric": "NVFP4 Wgrad step TFLOP/s (RHT quantize of dY^T and X^T + GEMM)",
+        nv = N * m
+        qgbs = nv * QUANT_BYTES_PER_VALUE_2PASS / qa_ms / 1e6
+        line.update({"metric": "NVFP4 Wgrad step TFLOP/s (column-wise RHT quantize of dY and X + GEMM)",
                      "value": flops / ms / 1e9, "unit": "TFLOP/s", "higher_is_better": True,
                      "ms_per_step": ms,
-                     "config": {"workload": f"wgrad dW = dY^T X, {N} x {K}, {m} tokens, "
+                     "config": {"workload": f"wgrad dW = dY^T X, {N} x {K}, {m} tokens, forward layouts, "
                                             "16x16 RHT on both operands", "sign_mask": mask,
                                 "l2": "flushed"},
-                     "quantize_rht_dy_ms": qa_ms, "quantize_rht_x_ms": qw_ms, "gemm_ms": g_ms,
-                     "quantize_rht_dy_gbs": qgbs,
-                     "quantize_rht_x_gbs": K * m * QUANT_BYTES_PER_VALUE_2PASS / qw_ms / 1e6,
+                     "quantize_t_rht_dy_ms": qa_ms, "quantize_t_rht_x_ms": qw_ms, "gemm_ms": g_ms,
+                     "quantize_t_rht_dy_gbs": qgbs,
+                     "quantize_t_dy_gbs": nv * QUANT_BYTES_PER_VALUE_2PASS / cw_ms / 1e6,
+                     "quantize_rht_rowwise_dy_t_gbs": nv * QUANT_BYTES_PER_VALUE_2PASS / rw_ms / 1e6,
                      "gemm_tflops": flops / g_ms / 1e9, "status": st,
-                     "roofline": {"kernel": "k_amax_rht + k_encode_rht (dY^T)", "bound": "hbm",
+                     "roofline": {"kernel": "k_amax_t_rht + k_encode_t_rht (dY)", "bound": "hbm",
                                   "achieved": qgbs, "peak": hbm_gbs, "unit": "GB/s",
                                   "frac": qgbs / hbm_gbs,
                                   "bytes_per_value": QUANT_BYTES_PER_VALUE_2PASS,

@@ -175,6 +175,25 @@ NVFP4_API nvfp4_status nvfp4_quantize_rht(const void *x, int64_t ld, uint32_t si
                                           const nvfp4_tensor *out, int32_t global_supplied,
                                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Column-wise quantization: out = NVFP4 of x^T, read straight from a
+ * row-major x without a BF16 transpose in memory.  The Dgrad and Wgrad GEMMs
+ * ("NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens", section
+ * "Four stabilisation devices": Fprop, Dgrad and Wgrad all in NVFP4)
+ * contract over the axes the forward pass keeps contiguous, and the
+ * block-scaled GEMM wants 16-value blocks along its contraction axis: for
+ * Wgrad dW = dY^T X both dY and X are quantized column-wise.
+ * x: BF16, out->cols rows x out->rows columns, row pitch ld elements.
+ *   out->cols % 16 == 0 (blocks of 16 rows of x); out->rows % 8 == 0
+ *   (NVFP4_ERR_SHAPE otherwise); x and ld 16-byte aligned.
+ * out: [out->rows x out->cols]; output row j is column j of x.  Codes,
+ *   scales and the tensor scale equal those of nvfp4_quantize (rht = 0) or
+ *   nvfp4_quantize_rht (rht = 1, sign_mask as there) applied to an explicit
+ *   BF16 copy of x^T.
+ * Workspace, status word, global_supplied and errors as nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t sign_mask,
+                                        const nvfp4_tensor *out, int32_t global_supplied,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
 /* Same quantization as nvfp4_quantize, for callers that cannot allocate
  * device memory when they quantize: code recorded into a CUDA graph (device
  * allocation cannot be captured), latency-critical paths that cannot afford

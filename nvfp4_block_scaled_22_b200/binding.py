@@ -34,7 +34,7 @@ EXPORTED = (
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
-    "nvfp4_quantize_noalloc", "nvfp4_quantize_rht",
+    "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t",
 )
 
 
@@ -81,6 +81,7 @@ def lib() -> C.CDLL:
             "nvfp4_set_gemm_pairs": (i32, [i32]),
             "nvfp4_quantize_noalloc": (C.c_int, [vp, i64, T, i32, vp]),
             "nvfp4_quantize_rht": (C.c_int, [vp, i64, C.c_uint32, T, i32, vp, sz, vp]),
+            "nvfp4_quantize_t": (C.c_int, [vp, i64, i32, C.c_uint32, T, i32, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -209,6 +210,24 @@ def nvfp4_quantize_rht(x: torch.Tensor, sign_mask: int, out: NVFP4Tensor | None 
     _check(lib().nvfp4_quantize_rht(x.data_ptr(), x.stride(0), sign_mask, C.byref(t),
                                     int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
            "nvfp4_quantize_rht")
+    return out
+
+
+def nvfp4_quantize_t(x: torch.Tensor, out: NVFP4Tensor | None = None, layout: int = SF_SWIZZLED,
+                     sign_mask: int | None = None, global_supplied: bool = False,
+                     workspace: Workspace | None = None, stream=None) -> NVFP4Tensor:
+    """NVFP4 of x^T from a row-major BF16 x (x.shape = (R, C) gives a C x R
+    tensor).  With ``sign_mask`` the blocks are Hadamard-transformed first."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows_x, cols_x = x.shape
+    if out is None:
+        out = NVFP4Tensor.empty(cols_x, rows_x, layout, x.device)
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    rht = 0 if sign_mask is None else 1
+    _check(lib().nvfp4_quantize_t(x.data_ptr(), x.stride(0), rht, sign_mask or 0, C.byref(t),
+                                  int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
+           "nvfp4_quantize_t")
     return out
 
 

@@ -232,6 +232,78 @@ nvfp4_status nvfp4_quantize_rht(const void *x, int64_t ld, uint32_t sign_mask,
                       static_cast<cudaStream_t>(stream), sms, true, sign_mask);
 }
 
+nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t sign_mask,
+                              const nvfp4_tensor *out, int32_t global_supplied, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    if (rht != 0 && rht != 1) return NVFP4_ERR_INVALID_ARG;
+    if (sign_mask > 0xFFFFu) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    const int64_t R = out->cols, C = out->rows;        // x is R x C
+    if (C % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (R > 0 && C > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < C) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
+    uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(C, 128) * 128 : C;
+    const int64_t tasks = transpose_tasks(R, rows_out);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    const int per_cta = kTransposeThreads / 32;
+    int n_partials = 0;
+    if (!global_supplied) {
+        if (rht) {
+            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(transpose_tasks(R, C), per_cta),
+                                                                8LL * sms), kMaxPartials);
+            if (grid < 1) grid = 1;
+            k_amax_t_rht<<<grid, kTransposeThreads, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C,
+                                                            sign_mask, partials);
+            n_partials = grid;
+        } else {
+            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(R, 8), 4 * sms), kMaxPartials);
+            if (grid < 1) grid = 1;
+            k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C, nullptr, R,
+                                        partials, status);
+            n_partials = grid;
+        }
+        st = launched(cudaGetLastError());
+        if (st != NVFP4_OK) return st;
+    }
+    EncodeParams p;
+    p.x = static_cast<const uint16_t *>(x);
+    p.ld = ld;
+    p.rows = C;
+    p.cols = R;
+    p.gather = nullptr;
+    p.src_rows = 0;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = out->global;
+    p.global_supplied = global_supplied;
+    p.partials = partials;
+    p.n_partials = n_partials;
+    p.status = status;
+    p.rht_mask = sign_mask;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, per_cta), 8LL * sms);
+    if (grid < 1) grid = 1;
+    if (rht)
+        k_encode_t_rht<<<grid, kTransposeThreads, 0, s>>>(p);
+    else
+        k_encode_t<<<grid, kTransposeThreads, 0, s>>>(p);
+    return launched(cudaGetLastError());
+}
+
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                                    const int32_t *d_gather, const nvfp4_tensor *out,
                                    int32_t global_supplied, void *workspace,

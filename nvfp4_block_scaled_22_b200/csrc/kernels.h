@@ -72,6 +72,18 @@ __global__ void k_encode(EncodeParams p);
 __global__ void k_encode_narrow(EncodeParams p);
 __global__ void k_encode_rht(EncodeParams p);
 __global__ void k_encode_rht_narrow(EncodeParams p);
+// Column-wise quantization (out = NVFP4 of x^T): p.rows = columns of x,
+// p.cols = rows of x (a multiple of 16), x is p.cols x p.rows with pitch
+// p.ld; 128 threads per CTA.
+constexpr int kTransposeThreads = 128;
+__global__ void k_amax_t_rht(const uint16_t *x, int64_t ld, int64_t R, int64_t C, uint32_t rht_mask,
+                             uint32_t *partials);
+__global__ void k_encode_t(EncodeParams p);
+__global__ void k_encode_t_rht(EncodeParams p);
+inline int64_t transpose_tasks(int64_t x_rows, int64_t out_rows_padded) {
+    return ((x_rows + 63) / 64) * ((out_rows_padded + 63) / 64);
+}
+
 __global__ void k_dequantize(DequantParams p);
 __global__ void k_dequantize_narrow(DequantParams p);
 

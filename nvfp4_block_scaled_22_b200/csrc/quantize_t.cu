@@ -1,0 +1,201 @@
+// Column-wise NVFP4 quantization: the NVFP4 tensor of x^T straight from a
+// row-major x, without a BF16 transpose in memory.
+//
+// The Dgrad and Wgrad GEMMs of a linear layer contract over the axes the
+// forward pass keeps contiguous ("NVFP4: how NVIDIA pre-trained a 12B model
+// on 10T tokens", section "Four stabilisation devices": Fprop, Dgrad and
+// Wgrad all run in NVFP4); the block-scaled GEMM wants both operands with
+// 16-value blocks along the contraction axis.  For x [R x C] this produces
+// out = NVFP4(x^T) [C x R]: output row j holds column j of x, blocked by 16
+// consecutive rows of x, with exactly the codes and scales that quantizing
+// an explicit BF16 x^T would give.
+//
+// Kernels
+//   k_amax_t_rht : tensor amax of the Hadamard-transformed column blocks
+//                  (the plain tensor amax of x^T is k_amax over x itself).
+//   k_encode_t   : codes + scales of x^T (kRht: of its transformed blocks).
+//
+// Work split: a warp task is a 64 x 64 tile of x (4 output blocks of 64
+// output rows).  The warp stages the tile in shared memory with coalesced
+// 16-byte loads (each instruction reads four 128-byte row pieces), then lane
+// l takes columns 2l and 2l + 1: a 32-bit shared read per tile row gives
+// both columns' values, two byte permutes per pair of rows regroup them
+// into each column's packed BF16 pairs, and the row-wise block encoder
+// does the rest.  Each lane stores 32 contiguous code bytes and one scale
+// word per output row.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "encode_common.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kTThreads = kTransposeThreads;   // 4 warps per CTA
+constexpr int kTile = 64;                 // tile rows (of x) and columns (of x)
+constexpr int kTileWords = kTile * kTile / 2;   // BF16 pairs per tile
+
+// Stage tile (tr, tc) of x in shared memory as [64 rows][32 words]; values
+// outside x read as zero.  Requires C % 8 == 0 (whole 16-byte pieces).
+__device__ __forceinline__ void load_tile(const uint16_t *__restrict__ x, int64_t ld, int64_t R,
+                                          int64_t C, int64_t r0, int64_t c0, uint32_t *tile,
+                                          int lane) {
+    const int pr = lane >> 3, pc = lane & 7;          // row within a 4-row step, 16-byte piece
+    uint4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int64_t r = r0 + pr + 4 * i, c = c0 + pc * 8;
+        v[i] = (r < R && c < C) ? __ldg(reinterpret_cast<const uint4 *>(x + r * ld + c))
+                                : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        reinterpret_cast<uint4 *>(tile)[(pr + 4 * i) * 8 + pc] = v[i];
+}
+
+// Rows 16k .. 16k+15 of the lane's two columns as the row-wise encoder's
+// packed input: a/b for column 2l, c/d for column 2l + 1 (value 2i in the
+// low half of word i).
+__device__ __forceinline__ void column_blocks(const uint32_t *tile, int k, int lane, uint4 &a,
+                                              uint4 &b, uint4 &c, uint4 &d) {
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t w0 = tile[(16 * k + 2 * i) * 32 + lane];       // row 2i:   (col 2l, col 2l+1)
+        const uint32_t w1 = tile[(16 * k + 2 * i + 1) * 32 + lane];   // row 2i+1
+        lo[i] = __byte_perm(w0, w1, 0x5410);                           // (row 2i, row 2i+1) of col 2l
+        hi[i] = __byte_perm(w0, w1, 0x7632);                           // same for col 2l + 1
+    }
+    a = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    b = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    c = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    d = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+}
+
+// Codes (up to four blocks) and the scale word of output row j at scale
+// column b0; rows in [C, rows_out) are band padding and get zero scales.
+// 16-byte code stores only where the row pitch R/2 keeps them aligned.
+__device__ __forceinline__ void store_row(const EncodeParams &p, int64_t j, int64_t C,
+                                          int64_t rows_out, int64_t R, int64_t b0, int nblk,
+                                          int64_t sf_cols, int64_t col_tiles, const uint2 (&cw)[4],
+                                          uint32_t sw) {
+    if (j >= rows_out) return;
+    if (j < C) {
+        uint8_t *cp = p.codes + j * (R / 2) + b0 * 8;
+        if (nblk == 4 && (R & 31) == 0) {
+            reinterpret_cast<uint4 *>(cp)[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+            reinterpret_cast<uint4 *>(cp)[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < nblk) reinterpret_cast<uint2 *>(cp)[k] = cw[k];
+        }
+    }
+    const uint32_t word = (j < C) ? sw : 0u;
+    uint8_t *sp = p.scales + sf_offset(j, b0, sf_cols, col_tiles, p.layout);
+    if (p.layout == 0 || ((sf_cols & 3) == 0 && b0 + 4 <= sf_cols)) {
+        *reinterpret_cast<uint32_t *>(sp) = word;
+    } else {                                                   // ragged linear row
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < nblk) sp[k] = (uint8_t)(word >> (8 * k));
+    }
+}
+
+}  // namespace
+
+// ----------------------------------------------------------- k_amax_t_rht
+// x is R x C (pitch ld); writes the CTA's max |y| as f32 bits.
+__global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__restrict__ x, int64_t ld,
+                                                          int64_t R, int64_t C, uint32_t rht_mask,
+                                                          uint32_t *__restrict__ partials) {
+    __shared__ uint32_t tiles[kTThreads / 32][kTileWords];
+    __shared__ uint32_t red[kTThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t rt = (uint32_t)((R + kTile - 1) / kTile), ct = (uint32_t)((C + kTile - 1) / kTile);
+    const uint32_t tasks = rt * ct;
+    const SignFlips f = sign_flips(rht_mask);
+    uint32_t m = 0;
+    for (uint32_t t = blockIdx.x * (kTThreads / 32) + warp; t < tasks;
+         t += gridDim.x * (kTThreads / 32)) {
+        const int64_t r0 = (int64_t)(t / ct) * kTile, c0 = (int64_t)(t % ct) * kTile;
+        load_tile(x, ld, R, C, r0, c0, tiles[warp], lane);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (r0 + 16 * k >= R) break;                               // uniform across the warp
+            uint4 a, b, c, d;
+            column_blocks(tiles[warp], k, lane, a, b, c, d);
+            float2 y[8];
+            rht16(a, b, f, y);                                         // zero columns stay zero
+            m = max(m, abs_max_bits(y));
+            rht16(c, d, f, y);
+            m = max(m, abs_max_bits(y));
+        }
+        __syncwarp();
+    }
+    const uint32_t v = block_reduce_max(m, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = v;
+}
+
+// -------------------------------------------------------------- k_encode_t
+template <bool kRht>
+__device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
+    __shared__ uint32_t tiles[kTThreads / 32][kTileWords];
+    __shared__ uint32_t red[kTThreads / 32];
+    __shared__ EncodeTables tab;
+    float g;
+    if (p.global_supplied) {
+        g = *p.global;
+    } else {
+        if (!global_from_partials(p.partials, p.n_partials, p.status, &g, red)) return;
+        if (blockIdx.x == 0 && threadIdx.x == 0) *p.global = g;
+    }
+    fill_tables(tab, g);
+    __syncthreads();
+    const SignFlips f = sign_flips(kRht ? p.rht_mask : 0u);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t R = p.cols, C = p.rows;
+    const int64_t sf_cols = R / 16, sf_cols4 = (sf_cols + 3) / 4 * 4, col_tiles = sf_cols4 / 4;
+    const int64_t rows_out = (p.layout == 0) ? (C + 127) / 128 * 128 : C;
+    const uint32_t rt = (uint32_t)((R + kTile - 1) / kTile);
+    const uint32_t ct = (uint32_t)((rows_out + kTile - 1) / kTile);
+    const uint32_t tasks = rt * ct;
+    bool finite = true;
+    for (uint32_t t = blockIdx.x * (kTThreads / 32) + warp; t < tasks;
+         t += gridDim.x * (kTThreads / 32)) {
+        const int64_t r0 = (int64_t)(t / ct) * kTile, c0 = (int64_t)(t % ct) * kTile;
+        load_tile(p.x, p.ld, R, C, r0, c0, tiles[warp], lane);
+        __syncwarp();
+        uint2 code0[4], code1[4];                  // columns 2l, 2l+1; blocks k = 0..3
+        uint32_t sw0 = 0, sw1 = 0;                 // their scale words
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            code0[k] = code1[k] = make_uint2(0, 0);
+            if (r0 + 16 * k >= R) continue;        // uniform across the warp
+            uint4 a, b, c, d;
+            column_blocks(tiles[warp], k, lane, a, b, c, d);
+            EncodeBlockOut o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
+            EncodeBlockOut o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
+            finite &= o0.finite && o1.finite;
+            code0[k] = o0.codes;
+            code1[k] = o1.codes;
+            sw0 |= o0.scale << (8 * k);
+            sw1 |= o1.scale << (8 * k);
+        }
+        const int64_t b0 = r0 / 16;                // first scale column of the tile
+        const int nblk = (sf_cols - b0 < 4) ? (int)(sf_cols - b0) : 4;
+        const int64_t j = c0 + 2 * lane;           // output rows j, j + 1
+        store_row(p, j, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code0, sw0);
+        store_row(p, j + 1, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code1, sw1);
+        __syncwarp();
+    }
+    if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
+}
+
+__global__ void __launch_bounds__(kTThreads) k_encode_t(EncodeParams p) { encode_t_body<false>(p); }
+
+__global__ void __launch_bounds__(kTThreads) k_encode_t_rht(EncodeParams p) { encode_t_body<true>(p); }
+
+}  // namespace nvfp4

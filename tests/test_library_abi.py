@@ -68,6 +68,10 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     assert lib.nvfp4_quantize_rht(16, 32, 0x10000, t, 0, 16, 1 << 16, 0) == 1   # mask > 16 bits
     t = binding.CTensor(16, 16, 16, 4, 24, 0)
     assert lib.nvfp4_quantize_rht(16, 32, 0xFFFF, t, 0, 16, 1 << 16, 0) == 3    # cols % 16
+    t = binding.CTensor(16, 16, 16, 12, 32, 0)
+    assert lib.nvfp4_quantize_t(16, 32, 0, 0, t, 0, 16, 1 << 16, 0) == 3        # x columns % 8
+    t = binding.CTensor(16, 16, 16, 16, 32, 0)
+    assert lib.nvfp4_quantize_t(16, 32, 2, 0, t, 0, 16, 1 << 16, 0) == 1        # rht flag
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
