@@ -266,18 +266,23 @@ nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t s
             int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(transpose_tasks(R, C), per_cta),
                                                                 8LL * sms), kMaxPartials);
             if (grid < 1) grid = 1;
-            k_amax_t_rht<<<grid, kTransposeThreads, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C,
-                                                            sign_mask, partials);
+            const uint16_t *xp = static_cast<const uint16_t *>(x);
+            int64_t ld_ = ld, R_ = R, C_ = C;
+            uint32_t mask_ = sign_mask;
+            uint32_t *part_ = partials;
+            void *args[] = {&xp, &ld_, &R_, &C_, &mask_, &part_};
+            st = launched(launch_transpose_kernel((const void *)k_amax_t_rht, grid, args, s));
+            if (st != NVFP4_OK) return st;
             n_partials = grid;
         } else {
             int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(R, 8), 4 * sms), kMaxPartials);
             if (grid < 1) grid = 1;
             k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C, nullptr, R,
                                         partials, status);
+            st = launched(cudaGetLastError());
+            if (st != NVFP4_OK) return st;
             n_partials = grid;
         }
-        st = launched(cudaGetLastError());
-        if (st != NVFP4_OK) return st;
     }
     EncodeParams p;
     p.x = static_cast<const uint16_t *>(x);
@@ -297,11 +302,9 @@ nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t s
     p.rht_mask = sign_mask;
     int grid = (int)std::min<int64_t>(ceil_div(tasks, per_cta), 8LL * sms);
     if (grid < 1) grid = 1;
-    if (rht)
-        k_encode_t_rht<<<grid, kTransposeThreads, 0, s>>>(p);
-    else
-        k_encode_t<<<grid, kTransposeThreads, 0, s>>>(p);
-    return launched(cudaGetLastError());
+    void *args[] = {&p};
+    return launched(launch_transpose_kernel(rht ? (const void *)k_encode_t_rht : (const void *)k_encode_t,
+                                            grid, args, s));
 }
 
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,

@@ -76,6 +76,8 @@ __global__ void k_encode_rht_narrow(EncodeParams p);
 // p.cols = rows of x (a multiple of 16), x is p.cols x p.rows with pitch
 // p.ld; 128 threads per CTA.
 constexpr int kTransposeThreads = 128;
+constexpr int kTransposeSmemBytes = (kTransposeThreads / 32) * 2 * 64 * 64 * 2;   // 64 KiB
+cudaError_t launch_transpose_kernel(const void *kernel, int grid, void **args, cudaStream_t stream);
 __global__ void k_amax_t_rht(const uint16_t *x, int64_t ld, int64_t R, int64_t C, uint32_t rht_mask,
                              uint32_t *partials);
 __global__ void k_encode_t(EncodeParams p);

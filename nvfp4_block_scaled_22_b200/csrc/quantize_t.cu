@@ -16,8 +16,9 @@
 //   k_encode_t   : codes + scales of x^T (kRht: of its transformed blocks).
 //
 // Work split: a warp task is a 64 x 64 tile of x (4 output blocks of 64
-// output rows).  The warp stages the tile in shared memory with coalesced
-// 16-byte loads (each instruction reads four 128-byte row pieces), then lane
+// output rows).  The warp copies the tile into shared memory with cp.async
+// (each instruction moves four 128-byte row pieces), double-buffered so the
+// next tile's copy overlaps the current tile's encode, then lane
 // l takes columns 2l and 2l + 1: a 32-bit shared read per tile row gives
 // both columns' values, two byte permutes per pair of rows regroup them
 // into each column's packed BF16 pairs, and the row-wise block encoder
@@ -36,22 +37,55 @@ constexpr int kTThreads = kTransposeThreads;   // 4 warps per CTA
 constexpr int kTile = 64;                 // tile rows (of x) and columns (of x)
 constexpr int kTileWords = kTile * kTile / 2;   // BF16 pairs per tile
 
-// Stage tile (tr, tc) of x in shared memory as [64 rows][32 words]; values
-// outside x read as zero.  Requires C % 8 == 0 (whole 16-byte pieces).
-__device__ __forceinline__ void load_tile(const uint16_t *__restrict__ x, int64_t ld, int64_t R,
-                                          int64_t C, int64_t r0, int64_t c0, uint32_t *tile,
-                                          int lane) {
+// Tile (r0, c0) of x copied asynchronously into shared memory as [64 rows]
+// [32 words] (cp.async, 16 bytes per lane per step, four 128-byte row
+// pieces per warp instruction); values outside x are zero-filled without a
+// global read.  Requires C % 8 == 0 (whole 16-byte pieces).
+__device__ __forceinline__ void issue_tile(const uint16_t *__restrict__ x, int64_t ld, int64_t R,
+                                           int64_t C, int64_t r0, int64_t c0, uint32_t *tile,
+                                           int lane) {
     const int pr = lane >> 3, pc = lane & 7;          // row within a 4-row step, 16-byte piece
-    uint4 v[16];
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(tile);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int64_t r = r0 + pr + 4 * i, c = c0 + pc * 8;
-        v[i] = (r < R && c < C) ? __ldg(reinterpret_cast<const uint4 *>(x + r * ld + c))
-                                : make_uint4(0, 0, 0, 0);
+        const bool in = r < R && c < C;
+        const void *src = in ? (const void *)(x + r * ld + c) : (const void *)x;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
+                     :: "r"(base + (uint32_t)(((pr + 4 * i) * 8 + pc) * 16)), "l"(src),
+                        "r"(in ? 16 : 0)
+                     : "memory");
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        reinterpret_cast<uint4 *>(tile)[(pr + 4 * i) * 8 + pc] = v[i];
+}
+
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
+// Wait until at most one committed group (the newest) is still in flight.
+__device__ __forceinline__ void async_wait_all_but_newest() {
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+}
+
+// Double-buffered walk over a warp's tiles t0, t0 + stride, ...: the copy of
+// the next tile runs while `work(tile_words, r0, c0)` handles the current one.
+template <typename Work>
+__device__ __forceinline__ void walk_tiles(const uint16_t *x, int64_t ld, int64_t R, int64_t C,
+                                           uint32_t t0, uint32_t stride, uint32_t tasks, uint32_t ct,
+                                           uint32_t *buf0, uint32_t *buf1, int lane, Work work) {
+    uint32_t t = t0;
+    if (t < tasks) issue_tile(x, ld, R, C, (int64_t)(t / ct) * kTile, (int64_t)(t % ct) * kTile, buf0, lane);
+    async_commit();
+    for (int i = 0; t < tasks; ++i, t += stride) {
+        uint32_t *cur = (i & 1) ? buf1 : buf0, *nxt = (i & 1) ? buf0 : buf1;
+        const uint32_t tn = t + stride;
+        if (tn < tasks)
+            issue_tile(x, ld, R, C, (int64_t)(tn / ct) * kTile, (int64_t)(tn % ct) * kTile, nxt, lane);
+        async_commit();
+        async_wait_all_but_newest();
+        __syncwarp();
+        work(cur, (int64_t)(t / ct) * kTile, (int64_t)(t % ct) * kTile);
+        __syncwarp();                            // cur is refilled two steps later
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
 // Rows 16k .. 16k+15 of the lane's two columns as the row-wise encoder's
@@ -106,35 +140,33 @@ __device__ __forceinline__ void store_row(const EncodeParams &p, int64_t j, int6
 }  // namespace
 
 // ----------------------------------------------------------- k_amax_t_rht
-// x is R x C (pitch ld); writes the CTA's max |y| as f32 bits.
+// x is R x C (pitch ld); writes the CTA's max |y| as f32 bits.  Dynamic
+// shared memory: two tile buffers per warp.
 __global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__restrict__ x, int64_t ld,
                                                           int64_t R, int64_t C, uint32_t rht_mask,
                                                           uint32_t *__restrict__ partials) {
-    __shared__ uint32_t tiles[kTThreads / 32][kTileWords];
+    extern __shared__ uint4 dyn_smem[];
     __shared__ uint32_t red[kTThreads / 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t *buf0 = reinterpret_cast<uint32_t *>(dyn_smem) + warp * 2 * kTileWords;
     const uint32_t rt = (uint32_t)((R + kTile - 1) / kTile), ct = (uint32_t)((C + kTile - 1) / kTile);
-    const uint32_t tasks = rt * ct;
     const SignFlips f = sign_flips(rht_mask);
     uint32_t m = 0;
-    for (uint32_t t = blockIdx.x * (kTThreads / 32) + warp; t < tasks;
-         t += gridDim.x * (kTThreads / 32)) {
-        const int64_t r0 = (int64_t)(t / ct) * kTile, c0 = (int64_t)(t % ct) * kTile;
-        load_tile(x, ld, R, C, r0, c0, tiles[warp], lane);
-        __syncwarp();
+    walk_tiles(x, ld, R, C, blockIdx.x * (kTThreads / 32) + warp, gridDim.x * (kTThreads / 32),
+               rt * ct, ct, buf0, buf0 + kTileWords, lane,
+               [&](const uint32_t *tile, int64_t r0, int64_t) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if (r0 + 16 * k >= R) break;                               // uniform across the warp
-            uint4 a, b, c, d;
-            column_blocks(tiles[warp], k, lane, a, b, c, d);
-            float2 y[8];
-            rht16(a, b, f, y);                                         // zero columns stay zero
-            m = max(m, abs_max_bits(y));
-            rht16(c, d, f, y);
-            m = max(m, abs_max_bits(y));
-        }
-        __syncwarp();
-    }
+                   for (int k = 0; k < 4; ++k) {
+                       if (r0 + 16 * k >= R) break;                    // uniform across the warp
+                       uint4 a, b, c, d;
+                       column_blocks(tile, k, lane, a, b, c, d);
+                       float2 y[8];
+                       rht16(a, b, f, y);                              // zero columns stay zero
+                       m = max(m, abs_max_bits(y));
+                       rht16(c, d, f, y);
+                       m = max(m, abs_max_bits(y));
+                   }
+               });
     const uint32_t v = block_reduce_max(m, red);
     if (threadIdx.x == 0) partials[blockIdx.x] = v;
 }
@@ -142,7 +174,7 @@ __global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__rest
 // -------------------------------------------------------------- k_encode_t
 template <bool kRht>
 __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
-    __shared__ uint32_t tiles[kTThreads / 32][kTileWords];
+    extern __shared__ uint4 dyn_smem[];
     __shared__ uint32_t red[kTThreads / 32];
     __shared__ EncodeTables tab;
     float g;
@@ -156,46 +188,64 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
     __syncthreads();
     const SignFlips f = sign_flips(kRht ? p.rht_mask : 0u);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t *buf0 = reinterpret_cast<uint32_t *>(dyn_smem) + warp * 2 * kTileWords;
     const int64_t R = p.cols, C = p.rows;
     const int64_t sf_cols = R / 16, sf_cols4 = (sf_cols + 3) / 4 * 4, col_tiles = sf_cols4 / 4;
     const int64_t rows_out = (p.layout == 0) ? (C + 127) / 128 * 128 : C;
     const uint32_t rt = (uint32_t)((R + kTile - 1) / kTile);
     const uint32_t ct = (uint32_t)((rows_out + kTile - 1) / kTile);
-    const uint32_t tasks = rt * ct;
     bool finite = true;
-    for (uint32_t t = blockIdx.x * (kTThreads / 32) + warp; t < tasks;
-         t += gridDim.x * (kTThreads / 32)) {
-        const int64_t r0 = (int64_t)(t / ct) * kTile, c0 = (int64_t)(t % ct) * kTile;
-        load_tile(p.x, p.ld, R, C, r0, c0, tiles[warp], lane);
-        __syncwarp();
-        uint2 code0[4], code1[4];                  // columns 2l, 2l+1; blocks k = 0..3
-        uint32_t sw0 = 0, sw1 = 0;                 // their scale words
+    walk_tiles(p.x, p.ld, R, C, blockIdx.x * (kTThreads / 32) + warp, gridDim.x * (kTThreads / 32),
+               rt * ct, ct, buf0, buf0 + kTileWords, lane,
+               [&](const uint32_t *tile, int64_t r0, int64_t c0) {
+                   uint2 code0[4], code1[4];           // columns 2l, 2l+1; blocks k = 0..3
+                   uint32_t sw0 = 0, sw1 = 0;          // their scale words
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            code0[k] = code1[k] = make_uint2(0, 0);
-            if (r0 + 16 * k >= R) continue;        // uniform across the warp
-            uint4 a, b, c, d;
-            column_blocks(tiles[warp], k, lane, a, b, c, d);
-            EncodeBlockOut o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
-            EncodeBlockOut o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
-            finite &= o0.finite && o1.finite;
-            code0[k] = o0.codes;
-            code1[k] = o1.codes;
-            sw0 |= o0.scale << (8 * k);
-            sw1 |= o1.scale << (8 * k);
-        }
-        const int64_t b0 = r0 / 16;                // first scale column of the tile
-        const int nblk = (sf_cols - b0 < 4) ? (int)(sf_cols - b0) : 4;
-        const int64_t j = c0 + 2 * lane;           // output rows j, j + 1
-        store_row(p, j, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code0, sw0);
-        store_row(p, j + 1, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code1, sw1);
-        __syncwarp();
-    }
+                   for (int k = 0; k < 4; ++k) {
+                       code0[k] = code1[k] = make_uint2(0, 0);
+                       if (r0 + 16 * k >= R) continue; // uniform across the warp
+                       uint4 a, b, c, d;
+                       column_blocks(tile, k, lane, a, b, c, d);
+                       EncodeBlockOut o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
+                       EncodeBlockOut o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
+                       finite &= o0.finite && o1.finite;
+                       code0[k] = o0.codes;
+                       code1[k] = o1.codes;
+                       sw0 |= o0.scale << (8 * k);
+                       sw1 |= o1.scale << (8 * k);
+                   }
+                   const int64_t b0 = r0 / 16;         // first scale column of the tile
+                   const int nblk = (sf_cols - b0 < 4) ? (int)(sf_cols - b0) : 4;
+                   const int64_t j = c0 + 2 * lane;    // output rows j, j + 1
+                   store_row(p, j, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code0, sw0);
+                   store_row(p, j + 1, C, rows_out, R, b0, nblk, sf_cols, col_tiles, code1, sw1);
+               });
     if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
 }
 
 __global__ void __launch_bounds__(kTThreads) k_encode_t(EncodeParams p) { encode_t_body<false>(p); }
 
 __global__ void __launch_bounds__(kTThreads) k_encode_t_rht(EncodeParams p) { encode_t_body<true>(p); }
+
+// Launch with the dynamic shared memory of two tile buffers per warp (the
+// size limit is raised once per device).
+cudaError_t launch_transpose_kernel(const void *kernel, int grid, void **args, cudaStream_t stream) {
+    static bool attr_set[64][3] = {};
+    const void *kernels[3] = {(const void *)k_amax_t_rht, (const void *)k_encode_t,
+                              (const void *)k_encode_t_rht};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int which = -1;
+    for (int i = 0; i < 3; ++i)
+        if (kernels[i] == kernel) which = i;
+    if (which < 0) return cudaErrorInvalidDeviceFunction;
+    if (dev < 0 || dev >= 64 || !attr_set[dev][which]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTransposeSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev][which] = true;
+    }
+    return cudaLaunchKernel(kernel, dim3(grid), dim3(kTThreads), args, kTransposeSmemBytes, stream);
+}
 
 }  // namespace nvfp4
