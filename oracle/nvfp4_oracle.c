@@ -24,7 +24,8 @@
  *       compared": 0.5625 bytes per value (4.5 bits) including scales.
  *  [P2'] same pre-training page, section "Four stabilisation devices": the
  *       Wgrad inputs are multiplied by a 16x16 Hadamard matrix and a random
- *       +-1 sign vector before quantization.
+ *       +-1 sign vector before quantization; weights use 16x16 (2D) blocks
+ *       so that the transposed weight holds the same quantized values.
  *  The FP32 evaluation order below is the convention the hot path is
  *  specified with: global g = 448*6/amax_tensor, block scale
  *  s = e4m3_rne(amax_block/6*g), code = e2m1_rne(x*g/s), with x*g/s taken as
@@ -469,6 +470,60 @@ int nvo_quantize_rht(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, 
                 uint8_t c0 = nvo_e2m1_rne_satfinite(y[2 * i] * e);
                 uint8_t c1 = nvo_e2m1_rne_satfinite(y[2 * i + 1] * e);
                 cb[i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return NVO_OK;
+}
+
+/* ------------------------------------------------------ 2D (16x16) blocks */
+
+/* [P2'] 2D block scaling of a weight: one E4M3 scale per 16x16 block (16
+ * rows x 16 columns), so that W and W^T are quantized identically.
+ * READINGS: the block amax is max |x| over the block's values (a partial
+ * block at the bottom edge covers the rows present); s, e and the codes
+ * follow the 1D steps with that amax; the result is stored as an ordinary
+ * NVFP4 tensor (1x16 scale positions along each row) whose scale entry for
+ * row r, scale column b is the scale of block (r / 16, b).  g comes from the
+ * plain tensor amax (or is supplied). */
+int nvo_quantize_2d(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes,
+                    uint8_t *scales, int layout, int global_supplied, float *g_io)
+{
+    if (cols % 16 != 0 || rows < 0 || cols < 0)
+        return NVO_ERR_SHAPE;
+    float g = *g_io;
+    if (!global_supplied) {
+        float amax;
+        int st = nvo_tensor_amax(x, rows, cols, ld, &amax);
+        if (st != NVO_OK)
+            return st;
+        st = nvo_global_scale(amax, &g);
+        *g_io = g;
+        if (st != NVO_OK)
+            return st;
+    }
+    memset(scales, 0, (size_t)nvo_scales_bytes(rows, cols, layout));
+    for (int64_t a = 0; a * 16 < rows; ++a)
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            const int64_t r_end = (a * 16 + 16 < rows) ? a * 16 + 16 : rows;
+            float amax_b = 0.0f;
+            for (int64_t r = a * 16; r < r_end; ++r)
+                for (int i = 0; i < 16; ++i) {
+                    float v = fabsf(nvo_bf16_to_f32(x[r * ld + b * 16 + i]));
+                    if (v > amax_b)
+                        amax_b = v;
+                }
+            float t = amax_b / 6.0f;
+            t = t * g;
+            uint8_t s = nvo_e4m3_rne_satfinite(t);
+            float e = (s == 0) ? 0.0f : g / nvo_e4m3_decode(s);
+            for (int64_t r = a * 16; r < r_end; ++r) {
+                scales[nvo_sf_offset(r, b, rows, cols, layout)] = s;
+                uint8_t *cb = codes + r * (cols / 2) + b * 8;
+                for (int i = 0; i < 8; ++i) {
+                    uint8_t c0 = nvo_e2m1_rne_satfinite(nvo_bf16_to_f32(x[r * ld + b * 16 + 2 * i]) * e);
+                    uint8_t c1 = nvo_e2m1_rne_satfinite(nvo_bf16_to_f32(x[r * ld + b * 16 + 2 * i + 1]) * e);
+                    cb[i] = (uint8_t)(c0 | (c1 << 4));
+                }
             }
         }
     return NVO_OK;

@@ -17,7 +17,7 @@ __all__ = [
     "lib", "bf16_bits", "bf16_to_f32", "f32_to_bf16", "e2m1_decode", "e2m1_rne",
     "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
     "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
-    "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht",
+    "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -56,6 +56,8 @@ def lib() -> C.CDLL:
             "nvo_rht16_inverse": (None, [_p, C.c_uint32, _p]),
             "nvo_quantize_rht": (C.c_int, [_p, _i64, _i64, _i64, C.c_uint32, _p, _p, C.c_int,
                                            C.c_int, C.POINTER(C.c_float)]),
+            "nvo_quantize_2d": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int, C.c_int,
+                                          C.POINTER(C.c_float)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -217,6 +219,18 @@ def quantize_rht(x, sign_mask: int, layout: int = SF_SWIZZLED, g=None) -> tuple[
     gv = C.c_float(0.0 if g is None else float(np.float32(g)))
     st = lib().nvo_quantize_rht(_ptr(b), rows, cols, cols, sign_mask, _ptr(codes), _ptr(scales),
                                 layout, 0 if g is None else 1, C.byref(gv))
+    return st, Quantized(codes, scales, gv.value, rows, cols, layout)
+
+
+def quantize_2d(x, layout: int = SF_SWIZZLED, g=None) -> tuple[int, Quantized]:
+    """Quantize with one scale per 16x16 block (g given = supplied)."""
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    gv = C.c_float(0.0 if g is None else float(np.float32(g)))
+    st = lib().nvo_quantize_2d(_ptr(b), rows, cols, cols, _ptr(codes), _ptr(scales), layout,
+                               0 if g is None else 1, C.byref(gv))
     return st, Quantized(codes, scales, gv.value, rows, cols, layout)
 
 
