@@ -194,6 +194,25 @@ NVFP4_API nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, 
                                         const nvfp4_tensor *out, int32_t global_supplied,
                                         void *workspace, size_t workspace_bytes, void *stream);
 
+/* 2D (16x16 block) quantization of a weight ("NVFP4: how NVIDIA pre-trained
+ * a 12B model on 10T tokens", section "Four stabilisation devices": weights
+ * use 16x16 blocks so that W and W^T hold the same quantized values, which
+ * the Fprop and Dgrad GEMMs then share).
+ * One E4M3 scale per block of 16 rows x 16 columns of w, from the block's
+ * amax (a partial block at the bottom edge covers the rows present); the
+ * codes of each value follow the 1D steps under that scale.  g as in
+ * nvfp4_quantize (plain tensor amax, or supplied in *out->global).
+ * w: BF16 out->rows x out->cols, pitch ld, 16-byte aligned.
+ * out: W's NVFP4 tensor (16 rows of a group share each scale entry).
+ * out_t: NULL, or W^T's NVFP4 tensor [out->cols x out->rows] (requires
+ *   out->rows % 16 == 0 and out->cols % 8 == 0): the same quantized values
+ *   transposed, scales of block (a, b) at row k, column a for every k in
+ *   column group b; its tensor scale receives the same g.
+ * Workspace, status word and errors as nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_quantize_2d(const void *w, int64_t ld, const nvfp4_tensor *out,
+                                         const nvfp4_tensor *out_t, int32_t global_supplied,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
 /* Same quantization as nvfp4_quantize, for callers that cannot allocate
  * device memory when they quantize: code recorded into a CUDA graph (device
  * allocation cannot be captured), latency-critical paths that cannot afford

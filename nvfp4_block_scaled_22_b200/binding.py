@@ -34,7 +34,7 @@ EXPORTED = (
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
-    "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t",
+    "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
 )
 
 
@@ -82,6 +82,7 @@ def lib() -> C.CDLL:
             "nvfp4_quantize_noalloc": (C.c_int, [vp, i64, T, i32, vp]),
             "nvfp4_quantize_rht": (C.c_int, [vp, i64, C.c_uint32, T, i32, vp, sz, vp]),
             "nvfp4_quantize_t": (C.c_int, [vp, i64, i32, C.c_uint32, T, i32, vp, sz, vp]),
+            "nvfp4_quantize_2d": (C.c_int, [vp, i64, T, T, i32, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -229,6 +230,27 @@ def nvfp4_quantize_t(x: torch.Tensor, out: NVFP4Tensor | None = None, layout: in
                                   int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
            "nvfp4_quantize_t")
     return out
+
+
+def nvfp4_quantize_2d(w: torch.Tensor, out: NVFP4Tensor | None = None,
+                      out_t: NVFP4Tensor | None = None, transposed: bool = False,
+                      layout: int = SF_SWIZZLED, global_supplied: bool = False,
+                      workspace: Workspace | None = None, stream=None):
+    """16x16-block quantization of a BF16 weight; with ``transposed`` (or an
+    ``out_t``) also returns W^T's NVFP4 tensor holding the same values."""
+    assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.stride(1) == 1
+    rows, cols = w.shape
+    if out is None:
+        out = NVFP4Tensor.empty(rows, cols, layout, w.device)
+    if out_t is None and transposed:
+        out_t = NVFP4Tensor.empty(cols, rows, layout, w.device)
+    ws = workspace or default_workspace(w.device)
+    t = out.c_struct()
+    tt = out_t.c_struct() if out_t is not None else None
+    _check(lib().nvfp4_quantize_2d(w.data_ptr(), w.stride(0), C.byref(t),
+                                   C.byref(tt) if tt is not None else None, int(global_supplied),
+                                   ws.ptr, ws.nbytes, _stream(stream)), "nvfp4_quantize_2d")
+    return (out, out_t) if out_t is not None else out
 
 
 def nvfp4_global_scale(x: torch.Tensor, out: torch.Tensor | None = None,

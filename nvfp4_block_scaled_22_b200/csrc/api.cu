@@ -307,6 +307,87 @@ nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t s
                                             grid, args, s));
 }
 
+nvfp4_status nvfp4_quantize_2d(const void *w, int64_t ld, const nvfp4_tensor *out,
+                               const nvfp4_tensor *out_t, int32_t global_supplied, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    const int64_t R = out->rows, C = out->cols;
+    if (out_t != nullptr) {
+        st = check_tensor(out_t);
+        if (st != NVFP4_OK) return st;
+        if (out_t->rows != C || out_t->cols != R) return NVFP4_ERR_SHAPE;
+        if (R % 16 != 0) return NVFP4_ERR_SHAPE;
+    }
+    if (R > 0 && C > 0) {
+        if (w == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(w) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < C) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, R, C, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
+    uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    int n_partials = 0;
+    if (!global_supplied) {
+        int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(R, 8), 4 * sms), kMaxPartials);
+        if (grid < 1) grid = 1;
+        k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(w), ld, R, C, nullptr, R, partials,
+                                    status);
+        st = launched(cudaGetLastError());
+        if (st != NVFP4_OK) return st;
+        n_partials = grid;
+    } else if (out_t != nullptr && out_t->global != out->global) {
+        if (cudaMemcpyAsync(out_t->global, out->global, sizeof(float), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+    }
+    EncodeParams p;
+    p.x = static_cast<const uint16_t *>(w);
+    p.ld = ld;
+    p.rows = R;
+    p.cols = C;
+    p.gather = nullptr;
+    p.src_rows = 0;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = out->global;
+    p.global_supplied = global_supplied;
+    p.partials = partials;
+    p.n_partials = n_partials;
+    p.status = status;
+    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(R, 128) * 128 : R;
+    const int64_t tasks = ceil_div(rows_out, 16) * ceil_div(ceil_div(C / 16, 4) * 4, 16);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    if (grid < 1) grid = 1;
+    k_encode_2d<<<grid, 256, 0, s>>>(p);
+    st = launched(cudaGetLastError());
+    if (st != NVFP4_OK || out_t == nullptr) return st;
+    // W^T: column-wise with 16x16 blocks (x = W is R x C; out_t is C x R)
+    EncodeParams q = p;
+    q.rows = C;
+    q.cols = R;
+    q.codes = static_cast<uint8_t *>(out_t->codes);
+    q.scales = static_cast<uint8_t *>(out_t->scales);
+    q.layout = out_t->sf_layout;
+    q.global = out_t->global;
+    const int64_t rows_out_t = (out_t->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(C, 128) * 128 : C;
+    const int64_t tasks_t = transpose_tasks(R, rows_out_t);
+    if (tasks_t >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    int grid_t = (int)std::min<int64_t>(ceil_div(tasks_t, kTransposeThreads / 32), 8LL * sms);
+    if (grid_t < 1) grid_t = 1;
+    void *args[] = {&q};
+    return launched(launch_transpose_kernel((const void *)k_encode_t_2d, grid_t, args, s));
+}
+
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                                    const int32_t *d_gather, const nvfp4_tensor *out,
                                    int32_t global_supplied, void *workspace,

@@ -183,27 +183,47 @@ struct EncodeBlockOut {
     bool finite;
 };
 
-// Quantize one 16-value block held in two 16-byte words.
-__device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g,
-                                                       const EncodeTables &tab) {
-    uint32_t mw = amax_word(a, b);
-    const uint32_t bits = halves_to_f32bits(mw);
-    float t = __fmul_rn(div6_rn(bits, tab), g);
-    uint32_t s = e4m3_from_f32(t);
-    float e = tab.inv_s[s & 0x7Fu];
-    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float y[16];
+// Block scale code for a block amax given as the f32 bits of a BF16 value
+// (sign clear): s = e4m3(RN(RN(amax / 6) * g)).
+__device__ __forceinline__ uint32_t scale_code(uint32_t amax_bits, float g, const EncodeTables &tab) {
+    return e4m3_from_f32(__fmul_rn(div6_rn(amax_bits, tab), g));
+}
+
+// E2M1 codes of eight BF16 values (packed pairs, value 2i low) times e.
+__device__ __forceinline__ uint32_t encode8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float e) {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+    float y[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
         y[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), e);
         y[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), e);
     }
+    return e2m1x4_from_f32(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+}
+
+// Quantize one 16-value block held in two 16-byte words with the block
+// amax `bits` (its own, or that of the 16x16 block it belongs to).
+__device__ __forceinline__ EncodeBlockOut encode_block_amax(uint4 a, uint4 b, uint32_t bits, float g,
+                                                            const EncodeTables &tab) {
+    const uint32_t s = scale_code(bits, g, tab);
+    const float e = tab.inv_s[s & 0x7Fu];
     EncodeBlockOut o;
-    o.codes.x = e2m1x4_from_f32(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-    o.codes.y = e2m1x4_from_f32(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+    o.codes.x = encode8(a.x, a.y, a.z, a.w, e);
+    o.codes.y = encode8(b.x, b.y, b.z, b.w, e);
     o.scale = s;
     o.finite = bits <= 0x7F7FFFFFu;
     return o;
+}
+
+// max |x| of a 16-value BF16 block as f32 bits (Inf/NaN above every finite).
+__device__ __forceinline__ uint32_t block_amax_bits(uint4 a, uint4 b) {
+    return halves_to_f32bits(amax_word(a, b));
+}
+
+// Quantize one 16-value block held in two 16-byte words.
+__device__ __forceinline__ EncodeBlockOut encode_block(uint4 a, uint4 b, float g,
+                                                       const EncodeTables &tab) {
+    return encode_block_amax(a, b, block_amax_bits(a, b), g, tab);
 }
 
 // RN(a / 6) for an FP32 a >= 0.  While the quotient is a normal number

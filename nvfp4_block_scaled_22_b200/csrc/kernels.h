@@ -82,6 +82,9 @@ __global__ void k_amax_t_rht(const uint16_t *x, int64_t ld, int64_t R, int64_t C
                              uint32_t *partials);
 __global__ void k_encode_t(EncodeParams p);
 __global__ void k_encode_t_rht(EncodeParams p);
+__global__ void k_encode_t_2d(EncodeParams p);
+// 2D (16x16 block) row-wise encode: 256 threads; tasks of 16 rows x 256 columns.
+__global__ void k_encode_2d(EncodeParams p);
 inline int64_t transpose_tasks(int64_t x_rows, int64_t out_rows_padded) {
     return ((x_rows + 63) / 64) * ((out_rows_padded + 63) / 64);
 }

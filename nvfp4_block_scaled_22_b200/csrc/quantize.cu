@@ -340,6 +340,79 @@ __global__ void __launch_bounds__(kThreads, 3) k_encode_rht_narrow(EncodeParams 
     encode_body<true, true>(p);
 }
 
+// ------------------------------------------------------------ k_encode_2d
+// 2D weight blocks ("NVFP4: how NVIDIA pre-trained a 12B model on 10T
+// tokens", section "Four stabilisation devices"): one scale per 16 rows x
+// 16 columns.  A warp task is one 16-row group x 256 columns; lane l holds
+// columns 8l..8l+7 of all 16 rows (each load instruction reads 512
+// contiguous bytes of one row), lanes 2m and 2m+1 share a block and combine
+// their maxima with one shuffle, and each code store writes 128 contiguous
+// bytes of one row.  Every row of the group gets the block's scale.
+__global__ void __launch_bounds__(kThreads) k_encode_2d(EncodeParams p) {
+    __shared__ uint32_t red[kThreads / 32];
+    __shared__ EncodeTables tab;
+    float g;
+    if (p.global_supplied) {
+        g = *p.global;
+    } else {
+        if (!global_from_partials(p.partials, p.n_partials, p.status, &g, red)) return;
+        if (blockIdx.x == 0 && threadIdx.x == 0) *p.global = g;
+    }
+    fill_tables(tab, g);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t sf_cols = p.cols / 16, sf_cols4 = (sf_cols + 3) / 4 * 4, col_tiles = sf_cols4 / 4;
+    const int64_t rows_out = (p.layout == 0) ? (p.rows + 127) / 128 * 128 : p.rows;
+    const uint32_t chunks = (uint32_t)((sf_cols4 + 15) / 16);          // 16 blocks per task
+    const uint32_t tasks = (uint32_t)((rows_out + 15) / 16) * chunks;
+    bool finite = true;
+    for (uint32_t t = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); t < tasks;
+         t += gridDim.x * (kThreads / 32)) {
+        const int64_t r0 = (int64_t)(t / chunks) * 16;
+        const int64_t blk = (int64_t)(t % chunks) * 16 + (lane >> 1);   // this lane's block column
+        const int64_t c0 = blk * 16 + (lane & 1) * 8;                   // its first element column
+        const bool col_ok = blk < sf_cols;
+        uint4 v[16];
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            v[i] = (col_ok && r0 + i < p.rows)
+                       ? __ldg(reinterpret_cast<const uint4 *>(p.x + (r0 + i) * p.ld + c0))
+                       : make_uint4(0, 0, 0, 0);
+            m = max_u16x2(m, amax_word(v[i], v[i]));
+        }
+        uint32_t bits = halves_to_f32bits(m);
+        bits = max(bits, __shfl_xor_sync(0xFFFFFFFFu, bits, 1));
+        const uint32_t s = scale_code(bits, g, tab);
+        const float e = tab.inv_s[s & 0x7Fu];
+        finite &= bits <= 0x7F7FFFFFu;
+        if (col_ok) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (r0 + i < p.rows)
+                    *reinterpret_cast<uint32_t *>(p.codes + (r0 + i) * (p.cols / 2) + c0 / 2) =
+                        encode8(v[i].x, v[i].y, v[i].z, v[i].w, e);
+        }
+        // scale word of blocks blk..blk+3 (lanes 8q, 8q+2, 8q+4, 8q+6)
+        uint32_t word = s;
+        word |= __shfl_down_sync(0xFFFFFFFFu, s, 2) << 8;
+        word |= __shfl_down_sync(0xFFFFFFFFu, s, 4) << 16;
+        word |= __shfl_down_sync(0xFFFFFFFFu, s, 6) << 24;
+        if ((lane & 7) == 0 && blk < sf_cols4 && (p.layout == 0 || blk < sf_cols)) {
+            for (int i = 0; i < 16 && r0 + i < rows_out; ++i) {
+                const uint32_t wr = (r0 + i < p.rows) ? word : 0u;  // band padding rows: zero
+                uint8_t *sp = p.scales + sf_offset(r0 + i, blk, sf_cols, col_tiles, p.layout);
+                if (p.layout == 0 || ((sf_cols & 3) == 0 && blk + 4 <= sf_cols)) {
+                    *reinterpret_cast<uint32_t *>(sp) = wr;
+                } else {                                               // ragged linear row
+                    for (int j = 0; j < 4 && blk + j < sf_cols; ++j) sp[j] = (uint8_t)(wr >> (8 * j));
+                }
+            }
+        }
+    }
+    if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
+}
+
 // ----------------------------------------------------------- k_dequantize
 __device__ __forceinline__ void decode_block(uint2 codes, float d, uint4 &o0, uint4 &o1) {
     uint32_t out[8];

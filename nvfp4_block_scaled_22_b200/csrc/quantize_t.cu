@@ -172,7 +172,9 @@ __global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__rest
 }
 
 // -------------------------------------------------------------- k_encode_t
-template <bool kRht>
+// kTwoD: one scale per 16x16 block of x (16 rows x 16 columns, the 2D
+// weight blocks), so the output is the 2D quantization of x^T.
+template <bool kRht, bool kTwoD>
 __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
     extern __shared__ uint4 dyn_smem[];
     __shared__ uint32_t red[kTThreads / 32];
@@ -206,8 +208,19 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
                        if (r0 + 16 * k >= R) continue; // uniform across the warp
                        uint4 a, b, c, d;
                        column_blocks(tile, k, lane, a, b, c, d);
-                       EncodeBlockOut o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
-                       EncodeBlockOut o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
+                       EncodeBlockOut o0, o1;
+                       if (kTwoD) {
+                           // lanes 8m..8m+7 hold columns 16m..16m+15: one 16x16 block
+                           uint32_t m = max(block_amax_bits(a, b), block_amax_bits(c, d));
+                           m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                           m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                           m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                           o0 = encode_block_amax(a, b, m, g, tab);
+                           o1 = encode_block_amax(c, d, m, g, tab);
+                       } else {
+                           o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
+                           o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
+                       }
                        finite &= o0.finite && o1.finite;
                        code0[k] = o0.codes;
                        code1[k] = o1.codes;
@@ -223,21 +236,29 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
     if (!finite) set_status(p.status, ST_NONFINITE);   // only reachable with a supplied g
 }
 
-__global__ void __launch_bounds__(kTThreads) k_encode_t(EncodeParams p) { encode_t_body<false>(p); }
+__global__ void __launch_bounds__(kTThreads) k_encode_t(EncodeParams p) {
+    encode_t_body<false, false>(p);
+}
 
-__global__ void __launch_bounds__(kTThreads) k_encode_t_rht(EncodeParams p) { encode_t_body<true>(p); }
+__global__ void __launch_bounds__(kTThreads) k_encode_t_rht(EncodeParams p) {
+    encode_t_body<true, false>(p);
+}
+
+__global__ void __launch_bounds__(kTThreads) k_encode_t_2d(EncodeParams p) {
+    encode_t_body<false, true>(p);
+}
 
 // Launch with the dynamic shared memory of two tile buffers per warp (the
 // size limit is raised once per device).
 cudaError_t launch_transpose_kernel(const void *kernel, int grid, void **args, cudaStream_t stream) {
-    static bool attr_set[64][3] = {};
-    const void *kernels[3] = {(const void *)k_amax_t_rht, (const void *)k_encode_t,
-                              (const void *)k_encode_t_rht};
+    static bool attr_set[64][4] = {};
+    const void *kernels[4] = {(const void *)k_amax_t_rht, (const void *)k_encode_t,
+                              (const void *)k_encode_t_rht, (const void *)k_encode_t_2d};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int which = -1;
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 4; ++i)
         if (kernels[i] == kernel) which = i;
     if (which < 0) return cudaErrorInvalidDeviceFunction;
     if (dev < 0 || dev >= 64 || !attr_set[dev][which]) {

@@ -72,6 +72,11 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     assert lib.nvfp4_quantize_t(16, 32, 0, 0, t, 0, 16, 1 << 16, 0) == 3        # x columns % 8
     t = binding.CTensor(16, 16, 16, 16, 32, 0)
     assert lib.nvfp4_quantize_t(16, 32, 2, 0, t, 0, 16, 1 << 16, 0) == 1        # rht flag
+    t = binding.CTensor(16, 16, 16, 40, 32, 0)
+    tt = binding.CTensor(16, 16, 16, 32, 40, 0)
+    assert lib.nvfp4_quantize_2d(16, 32, t, tt, 0, 16, 1 << 16, 0) == 3         # rows % 16 with W^T
+    tt = binding.CTensor(16, 16, 16, 32, 48, 0)
+    assert lib.nvfp4_quantize_2d(16, 32, t, tt, 0, 16, 1 << 16, 0) == 3         # W^T shape
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
