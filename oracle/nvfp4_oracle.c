@@ -25,7 +25,11 @@
  *  [P2'] same pre-training page, section "Four stabilisation devices": the
  *       Wgrad inputs are multiplied by a 16x16 Hadamard matrix and a random
  *       +-1 sign vector before quantization; weights use 16x16 (2D) blocks
- *       so that the transposed weight holds the same quantized values.
+ *       so that the transposed weight holds the same quantized values;
+ *       gradients are rounded stochastically (a value 0.7 of the way from
+ *       one grid point to the next goes up with probability 0.7).
+ *  [PX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
+ *       1, 2, 3" (SC 2011): the Philox4x32-10 counter-based generator.
  *  The FP32 evaluation order below is the convention the hot path is
  *  specified with: global g = 448*6/amax_tensor, block scale
  *  s = e4m3_rne(amax_block/6*g), code = e2m1_rne(x*g/s), with x*g/s taken as
@@ -524,6 +528,141 @@ int nvo_quantize_2d(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, u
                     uint8_t c1 = nvo_e2m1_rne_satfinite(nvo_bf16_to_f32(x[r * ld + b * 16 + 2 * i + 1]) * e);
                     cb[i] = (uint8_t)(c0 | (c1 << 4));
                 }
+            }
+        }
+    return NVO_OK;
+}
+
+/* ---------------------------------------------- counter-based random bits */
+
+/* [PX] Philox4x32-10: ten rounds on a 128-bit counter under a 64-bit key.
+ * A round multiplies words 0 and 2 by 0xD2511F53 and 0xCD9E8D57 (full
+ * 64-bit products), then sets (c0, c1, c2, c3) = (hi(c2*M1) ^ c1 ^ k0,
+ * lo(c2*M1), hi(c0*M0) ^ c3 ^ k1, lo(c0*M0)); the key gains the Weyl
+ * constants 0x9E3779B9 and 0xBB67AE85 after every round. */
+void nvo_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    uint32_t c[4] = {ctr_in[0], ctr_in[1], ctr_in[2], ctr_in[3]};
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+        uint32_t n0 = (uint32_t)(p1 >> 32) ^ c[1] ^ k0;
+        uint32_t n1 = (uint32_t)p1;
+        uint32_t n2 = (uint32_t)(p0 >> 32) ^ c[3] ^ k1;
+        uint32_t n3 = (uint32_t)p0;
+        c[0] = n0; c[1] = n1; c[2] = n2; c[3] = n3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    for (int i = 0; i < 4; ++i)
+        out[i] = c[i];
+}
+
+/* ----------------------------------------------------- stochastic rounding */
+
+/* [P2'] Stochastic rounding onto the E2M1 grid.  READINGS: |y| >= 6
+ * saturates to 6; otherwise with lo <= |y| < hi the neighbouring grid
+ * values, |y| rounds up to hi with probability (|y| - lo) / (hi - lo),
+ * decided by a 16-bit uniform draw u (up iff u / 2^16 < that fraction, so
+ * the probability is ceil(2^16 * fraction) / 2^16); grid values stay put;
+ * the sign is copied from y (as in the round-to-nearest encode).  Returns
+ * the 4-bit code. */
+uint8_t nvo_e2m1_sr(float y, uint32_t u16)
+{
+    static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    uint8_t sign = signbit(y) ? 8 : 0;
+    double a = fabs((double)y);
+    if (a >= 6.0)
+        return sign | 7;
+    int k = 0;
+    while (k < 7 && grid[k + 1] <= a)
+        ++k;                                   /* grid[k] <= a < grid[k + 1] */
+    double frac = (a - grid[k]) / (grid[k + 1] - grid[k]);
+    int up = ((double)u16 / 65536.0) < frac;
+    return sign | (uint8_t)(k + up);
+}
+
+/* Random 16-bit draws of the 16 values of output block (row r, block b) of
+ * an R x C NVFP4 tensor, for the caller's 64-bit seed.  READING (the pages
+ * fix no generator): block index n = r * (C / 16) + b; Philox4x32-10 with
+ * counter (lo32(n), hi32(n), j, 0), j = 0, 1, and key (lo32(seed),
+ * hi32(seed)); value 8j + 2w takes the low 16 bits of word w of draw j,
+ * value 8j + 2w + 1 its high 16 bits. */
+void nvo_sr_block_draws(uint64_t seed, int64_t r, int64_t b, int64_t cols, uint32_t u[16])
+{
+    uint64_t n = (uint64_t)r * (uint64_t)(cols / 16) + (uint64_t)b;
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (uint32_t j = 0; j < 2; ++j) {
+        uint32_t ctr[4] = {(uint32_t)n, (uint32_t)(n >> 32), j, 0u}, w[4];
+        nvo_philox4x32_10(ctr, key, w);
+        for (int i = 0; i < 4; ++i) {
+            u[8 * j + 2 * i] = w[i] & 0xFFFFu;
+            u[8 * j + 2 * i + 1] = w[i] >> 16;
+        }
+    }
+}
+
+/* Two-level quantization with stochastic rounding of the codes (the block
+ * scales and g as in nvo_quantize; rht = 1 transforms every block first as
+ * in nvo_quantize_rht). */
+int nvo_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int rht,
+                    uint32_t sign_mask, uint64_t seed, uint8_t *codes, uint8_t *scales, int layout,
+                    int global_supplied, float *g_io)
+{
+    if (cols % 16 != 0 || rows < 0 || cols < 0)
+        return NVO_ERR_SHAPE;
+    float g = *g_io;
+    if (!global_supplied) {
+        float m = 0.0f;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t b = 0; b < cols / 16; ++b) {
+                float in[16], y[16];
+                for (int i = 0; i < 16; ++i)
+                    in[i] = nvo_bf16_to_f32(x[r * ld + b * 16 + i]);
+                if (rht)
+                    nvo_rht16(in, sign_mask, y);
+                else
+                    memcpy(y, in, sizeof y);
+                for (int i = 0; i < 16; ++i) {
+                    float v = fabsf(y[i]);
+                    if (!isfinite(v))
+                        return NVO_ERR_NONFINITE;
+                    if (v > m)
+                        m = v;
+                }
+            }
+        int st = nvo_global_scale(m, &g);
+        *g_io = g;
+        if (st != NVO_OK)
+            return st;
+    }
+    memset(scales, 0, (size_t)nvo_scales_bytes(rows, cols, layout));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            float in[16], y[16];
+            uint32_t u[16];
+            for (int i = 0; i < 16; ++i)
+                in[i] = nvo_bf16_to_f32(x[r * ld + b * 16 + i]);
+            if (rht)
+                nvo_rht16(in, sign_mask, y);
+            else
+                memcpy(y, in, sizeof y);
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i)
+                if (fabsf(y[i]) > amax_b)
+                    amax_b = fabsf(y[i]);
+            float t = amax_b / 6.0f;
+            t = t * g;
+            uint8_t s = nvo_e4m3_rne_satfinite(t);
+            float e = (s == 0) ? 0.0f : g / nvo_e4m3_decode(s);
+            scales[nvo_sf_offset(r, b, rows, cols, layout)] = s;
+            nvo_sr_block_draws(seed, r, b, cols, u);
+            uint8_t *cb = codes + r * (cols / 2) + b * 8;
+            for (int i = 0; i < 8; ++i) {
+                uint8_t c0 = nvo_e2m1_sr(y[2 * i] * e, u[2 * i]);
+                uint8_t c1 = nvo_e2m1_sr(y[2 * i + 1] * e, u[2 * i + 1]);
+                cb[i] = (uint8_t)(c0 | (c1 << 4));
             }
         }
     return NVO_OK;

@@ -18,6 +18,7 @@ __all__ = [
     "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
     "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
     "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
+    "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -58,6 +59,11 @@ def lib() -> C.CDLL:
                                            C.c_int, C.POINTER(C.c_float)]),
             "nvo_quantize_2d": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int, C.c_int,
                                           C.POINTER(C.c_float)]),
+            "nvo_philox4x32_10": (None, [_p, _p, _p]),
+            "nvo_e2m1_sr": (C.c_uint8, [C.c_float, C.c_uint32]),
+            "nvo_sr_block_draws": (None, [C.c_uint64, _i64, _i64, _i64, _p]),
+            "nvo_quantize_sr": (C.c_int, [_p, _i64, _i64, _i64, C.c_int, C.c_uint32, C.c_uint64, _p,
+                                          _p, C.c_int, C.c_int, C.POINTER(C.c_float)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -230,6 +236,38 @@ def quantize_2d(x, layout: int = SF_SWIZZLED, g=None) -> tuple[int, Quantized]:
     scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
     gv = C.c_float(0.0 if g is None else float(np.float32(g)))
     st = lib().nvo_quantize_2d(_ptr(b), rows, cols, cols, _ptr(codes), _ptr(scales), layout,
+                               0 if g is None else 1, C.byref(gv))
+    return st, Quantized(codes, scales, gv.value, rows, cols, layout)
+
+
+def philox4x32_10(ctr, key) -> list[int]:
+    c = np.ascontiguousarray(ctr, np.uint32)
+    k = np.ascontiguousarray(key, np.uint32)
+    out = np.zeros(4, np.uint32)
+    lib().nvo_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return [int(v) for v in out]
+
+
+def e2m1_sr(y: float, u16: int) -> int:
+    return int(lib().nvo_e2m1_sr(float(np.float32(y)), u16))
+
+
+def sr_block_draws(seed: int, r: int, b: int, cols: int) -> np.ndarray:
+    u = np.zeros(16, np.uint32)
+    lib().nvo_sr_block_draws(seed, r, b, cols, _ptr(u))
+    return u
+
+
+def quantize_sr(x, seed: int, layout: int = SF_SWIZZLED, sign_mask=None, g=None):
+    """Quantize with stochastically rounded codes (optionally after the
+    Hadamard transform).  Returns (status, tensor)."""
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    gv = C.c_float(0.0 if g is None else float(np.float32(g)))
+    st = lib().nvo_quantize_sr(_ptr(b), rows, cols, cols, 0 if sign_mask is None else 1,
+                               sign_mask or 0, seed, _ptr(codes), _ptr(scales), layout,
                                0 if g is None else 1, C.byref(gv))
     return st, Quantized(codes, scales, gv.value, rows, cols, layout)
 
