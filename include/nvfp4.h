@@ -213,6 +213,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_2d(const void *w, int64_t ld, const nvfp4_
                                          const nvfp4_tensor *out_t, int32_t global_supplied,
                                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* Quantization with stochastically rounded codes, for gradients ("NVFP4:
+ * how NVIDIA pre-trained a 12B model on 10T tokens", section "Four
+ * stabilisation devices": gradients are rounded stochastically -- a value
+ * 0.7 of the way to the next grid point goes up with probability 0.7).
+ * Scales and g are those of the round-to-nearest path; each value y = x*e
+ * (after the optional transform) goes to the E2M1 grid point above it with
+ * probability (|y| - lo) / (hi - lo), decided by a 16-bit draw u (up iff
+ * u / 2^16 < that fraction; grid values stay, |y| >= 6 saturates, the sign
+ * is kept).  Draws: Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011) keyed by `seed`, counter
+ * (lo32(n), hi32(n), j, 0) for output block n = row * (cols / 16) + block
+ * column and j = 0, 1; value 8j + 2w uses the low 16 bits of word w of draw
+ * j, value 8j + 2w + 1 the high 16 bits.  The same seed gives the same
+ * codes on every call.
+ * transposed: 0 = row-wise (x is out->rows x out->cols, as nvfp4_quantize),
+ *   1 = column-wise (x is out->cols x out->rows, as nvfp4_quantize_t).
+ * rht, sign_mask: apply the random Hadamard transform first (as
+ *   nvfp4_quantize_rht); rht = 0 ignores sign_mask.
+ * Other arguments, workspace and errors as nvfp4_quantize / _t. */
+NVFP4_API nvfp4_status nvfp4_quantize_sr(const void *x, int64_t ld, int32_t transposed, int32_t rht,
+                                         uint32_t sign_mask, uint64_t seed, const nvfp4_tensor *out,
+                                         int32_t global_supplied, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
 /* Same quantization as nvfp4_quantize, for callers that cannot allocate
  * device memory when they quantize: code recorded into a CUDA graph (device
  * allocation cannot be captured), latency-critical paths that cannot afford

@@ -35,6 +35,7 @@ EXPORTED = (
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
+    "nvfp4_quantize_sr",
 )
 
 
@@ -83,6 +84,8 @@ def lib() -> C.CDLL:
             "nvfp4_quantize_rht": (C.c_int, [vp, i64, C.c_uint32, T, i32, vp, sz, vp]),
             "nvfp4_quantize_t": (C.c_int, [vp, i64, i32, C.c_uint32, T, i32, vp, sz, vp]),
             "nvfp4_quantize_2d": (C.c_int, [vp, i64, T, T, i32, vp, sz, vp]),
+            "nvfp4_quantize_sr": (C.c_int, [vp, i64, i32, i32, C.c_uint32, C.c_uint64, T, i32, vp,
+                                            sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -251,6 +254,27 @@ def nvfp4_quantize_2d(w: torch.Tensor, out: NVFP4Tensor | None = None,
                                    C.byref(tt) if tt is not None else None, int(global_supplied),
                                    ws.ptr, ws.nbytes, _stream(stream)), "nvfp4_quantize_2d")
     return (out, out_t) if out_t is not None else out
+
+
+def nvfp4_quantize_sr(x: torch.Tensor, seed: int, out: NVFP4Tensor | None = None,
+                      transposed: bool = False, sign_mask: int | None = None,
+                      layout: int = SF_SWIZZLED, global_supplied: bool = False,
+                      workspace: Workspace | None = None, stream=None) -> NVFP4Tensor:
+    """Quantize with stochastically rounded codes (Philox draws keyed by
+    ``seed``); ``transposed`` gives NVFP4 of x^T, ``sign_mask`` applies the
+    Hadamard transform first."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out is None:
+        out = (NVFP4Tensor.empty(cols, rows, layout, x.device) if transposed
+               else NVFP4Tensor.empty(rows, cols, layout, x.device))
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize_sr(x.data_ptr(), x.stride(0), int(transposed),
+                                   0 if sign_mask is None else 1, sign_mask or 0, seed, C.byref(t),
+                                   int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
+           "nvfp4_quantize_sr")
+    return out
 
 
 def nvfp4_global_scale(x: torch.Tensor, out: torch.Tensor | None = None,

@@ -117,7 +117,8 @@ nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, i
 
 nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32_t *gather,
                         const nvfp4_tensor *out, int32_t global_supplied, void *ws,
-                        cudaStream_t stream, int sms, bool rht = false, uint32_t rht_mask = 0) {
+                        cudaStream_t stream, int sms, bool rht = false, uint32_t rht_mask = 0,
+                        bool sr = false, uint64_t sr_seed = 0) {
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
     uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kStatusBytes);
     int n_partials = 0;
@@ -152,15 +153,97 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
     p.n_partials = n_partials;
     p.status = status;
     p.rht_mask = rht_mask;
+    p.sr_seed = sr_seed;
     const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
     const bool narrow = tasks_are_groups(out->cols);
-    void (*kernel)(EncodeParams) = rht ? (narrow ? k_encode_rht_narrow : k_encode_rht)
-                                       : (narrow ? k_encode_narrow : k_encode);
+    void (*kernel)(EncodeParams) =
+        sr ? (rht ? (narrow ? k_encode_rht_sr_narrow : k_encode_rht_sr)
+                  : (narrow ? k_encode_sr_narrow : k_encode_sr))
+           : (rht ? (narrow ? k_encode_rht_narrow : k_encode_rht)
+                  : (narrow ? k_encode_narrow : k_encode));
     int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms);
     if (grid < 1) grid = 1;
     kernel<<<grid, 256, 0, stream>>>(p);
     return launched(cudaGetLastError());
+}
+
+// Column-wise quantize (out = NVFP4 of x^T); arguments already validated.
+nvfp4_status run_encode_t(const void *x, int64_t ld, bool rht, uint32_t sign_mask, bool sr,
+                          uint64_t sr_seed, const nvfp4_tensor *out, int32_t global_supplied,
+                          void *workspace, cudaStream_t s, int sms) {
+    nvfp4_status st = NVFP4_OK;
+    const int64_t R = out->cols, C = out->rows;        // x is R x C
+    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
+    uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(C, 128) * 128 : C;
+    const int64_t tasks = transpose_tasks(R, rows_out);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    const int per_cta = kTransposeThreads / 32;
+    int n_partials = 0;
+    if (!global_supplied) {
+        if (rht) {
+            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(transpose_tasks(R, C), per_cta),
+                                                                8LL * sms), kMaxPartials);
+            if (grid < 1) grid = 1;
+            const uint16_t *xp = static_cast<const uint16_t *>(x);
+            int64_t ld_ = ld, R_ = R, C_ = C;
+            uint32_t mask_ = sign_mask;
+            uint32_t *part_ = partials;
+            void *args[] = {&xp, &ld_, &R_, &C_, &mask_, &part_};
+            st = launched(launch_transpose_kernel((const void *)k_amax_t_rht, grid, args, s));
+            if (st != NVFP4_OK) return st;
+            n_partials = grid;
+        } else {
+            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(R, 8), 4 * sms), kMaxPartials);
+            if (grid < 1) grid = 1;
+            k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C, nullptr, R,
+                                        partials, status);
+            st = launched(cudaGetLastError());
+            if (st != NVFP4_OK) return st;
+            n_partials = grid;
+        }
+    }
+    EncodeParams p;
+    p.x = static_cast<const uint16_t *>(x);
+    p.ld = ld;
+    p.rows = C;
+    p.cols = R;
+    p.gather = nullptr;
+    p.src_rows = 0;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = out->global;
+    p.global_supplied = global_supplied;
+    p.partials = partials;
+    p.n_partials = n_partials;
+    p.status = status;
+    p.rht_mask = sign_mask;
+    p.sr_seed = sr_seed;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, per_cta), 8LL * sms);
+    if (grid < 1) grid = 1;
+    const void *kernel = sr ? (rht ? (const void *)k_encode_t_rht_sr : (const void *)k_encode_t_sr)
+                            : (rht ? (const void *)k_encode_t_rht : (const void *)k_encode_t);
+    void *args[] = {&p};
+    return launched(launch_transpose_kernel(kernel, grid, args, s));
+}
+
+// Shared argument checks of the column-wise entry points.
+nvfp4_status check_transposed(const void *x, int64_t ld, const nvfp4_tensor *out,
+                              int32_t global_supplied, void *workspace, size_t workspace_bytes) {
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
+    const int64_t R = out->cols, C = out->rows;
+    if (C % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (R > 0 && C > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < C) return NVFP4_ERR_SHAPE;
+    }
+    return check_workspace(workspace, workspace_bytes,
+                           nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
 }
 
 }  // namespace
@@ -237,74 +320,46 @@ nvfp4_status nvfp4_quantize_t(const void *x, int64_t ld, int32_t rht, uint32_t s
                               size_t workspace_bytes, void *stream) {
     if (rht != 0 && rht != 1) return NVFP4_ERR_INVALID_ARG;
     if (sign_mask > 0xFFFFu) return NVFP4_ERR_INVALID_ARG;
-    nvfp4_status st = check_tensor(out);
+    nvfp4_status st = check_transposed(x, ld, out, global_supplied, workspace, workspace_bytes);
     if (st != NVFP4_OK) return st;
-    if (global_supplied != 0 && global_supplied != 1) return NVFP4_ERR_INVALID_ARG;
-    const int64_t R = out->cols, C = out->rows;        // x is R x C
-    if (C % 8 != 0) return NVFP4_ERR_SHAPE;
-    if (R > 0 && C > 0) {
-        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
-        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
-        if (ld < C) return NVFP4_ERR_SHAPE;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return run_encode_t(x, ld, rht != 0, sign_mask, false, 0, out, global_supplied, workspace,
+                        static_cast<cudaStream_t>(stream), sms);
+}
+
+nvfp4_status nvfp4_quantize_sr(const void *x, int64_t ld, int32_t transposed, int32_t rht,
+                               uint32_t sign_mask, uint64_t seed, const nvfp4_tensor *out,
+                               int32_t global_supplied, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    if ((transposed != 0 && transposed != 1) || (rht != 0 && rht != 1)) return NVFP4_ERR_INVALID_ARG;
+    if (sign_mask > 0xFFFFu) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st;
+    if (transposed) {
+        st = check_transposed(x, ld, out, global_supplied, workspace, workspace_bytes);
+    } else {
+        st = check_tensor(out);
+        if (st == NVFP4_OK && global_supplied != 0 && global_supplied != 1) st = NVFP4_ERR_INVALID_ARG;
+        if (st == NVFP4_OK && out->rows > 0 && out->cols > 0) {
+            if (x == nullptr) st = NVFP4_ERR_INVALID_ARG;
+            else if (!aligned16(x) || ld % 8 != 0) st = NVFP4_ERR_ALIGNMENT;
+            else if (ld < out->cols) st = NVFP4_ERR_SHAPE;
+        }
+        if (st == NVFP4_OK)
+            st = check_workspace(workspace, workspace_bytes,
+                                 nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
     }
-    st = check_workspace(workspace, workspace_bytes,
-                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, out->rows, out->cols, 0, 0));
     if (st != NVFP4_OK) return st;
     int sms = 0;
     st = current_device(&sms);
     if (st != NVFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
-    uint32_t *partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
-    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(C, 128) * 128 : C;
-    const int64_t tasks = transpose_tasks(R, rows_out);
-    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    const int per_cta = kTransposeThreads / 32;
-    int n_partials = 0;
-    if (!global_supplied) {
-        if (rht) {
-            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(transpose_tasks(R, C), per_cta),
-                                                                8LL * sms), kMaxPartials);
-            if (grid < 1) grid = 1;
-            const uint16_t *xp = static_cast<const uint16_t *>(x);
-            int64_t ld_ = ld, R_ = R, C_ = C;
-            uint32_t mask_ = sign_mask;
-            uint32_t *part_ = partials;
-            void *args[] = {&xp, &ld_, &R_, &C_, &mask_, &part_};
-            st = launched(launch_transpose_kernel((const void *)k_amax_t_rht, grid, args, s));
-            if (st != NVFP4_OK) return st;
-            n_partials = grid;
-        } else {
-            int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(R, 8), 4 * sms), kMaxPartials);
-            if (grid < 1) grid = 1;
-            k_amax<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(x), ld, R, C, nullptr, R,
-                                        partials, status);
-            st = launched(cudaGetLastError());
-            if (st != NVFP4_OK) return st;
-            n_partials = grid;
-        }
-    }
-    EncodeParams p;
-    p.x = static_cast<const uint16_t *>(x);
-    p.ld = ld;
-    p.rows = C;
-    p.cols = R;
-    p.gather = nullptr;
-    p.src_rows = 0;
-    p.codes = static_cast<uint8_t *>(out->codes);
-    p.scales = static_cast<uint8_t *>(out->scales);
-    p.layout = out->sf_layout;
-    p.global = out->global;
-    p.global_supplied = global_supplied;
-    p.partials = partials;
-    p.n_partials = n_partials;
-    p.status = status;
-    p.rht_mask = sign_mask;
-    int grid = (int)std::min<int64_t>(ceil_div(tasks, per_cta), 8LL * sms);
-    if (grid < 1) grid = 1;
-    void *args[] = {&p};
-    return launched(launch_transpose_kernel(rht ? (const void *)k_encode_t_rht : (const void *)k_encode_t,
-                                            grid, args, s));
+    if (transposed)
+        return run_encode_t(x, ld, rht != 0, sign_mask, true, seed, out, global_supplied, workspace, s,
+                            sms);
+    return run_encode(x, ld, out->rows, nullptr, out, global_supplied, workspace, s, sms, rht != 0,
+                      sign_mask, true, seed);
 }
 
 nvfp4_status nvfp4_quantize_2d(const void *w, int64_t ld, const nvfp4_tensor *out,

@@ -262,6 +262,124 @@ __device__ __forceinline__ EncodeBlockOut encode_block_rht(uint4 a, uint4 b, con
     return o;
 }
 
+// ------------------------------------------------------ stochastic rounding
+// Gradients are rounded stochastically ("NVFP4: how NVIDIA pre-trained a 12B
+// model on 10T tokens", section "Four stabilisation devices"): a value goes
+// up to the next E2M1 grid point with probability equal to its fractional
+// distance.  Random bits: Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011) keyed by the
+// caller's 64-bit seed, counter (lo32(n), hi32(n), j, 0) for output block n
+// = row * (cols / 16) + block column and draws j = 0, 1; value 8j + 2w takes
+// the low 16 bits of word w of draw j, value 8j + 2w + 1 the high 16 bits.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t lo0 = c.x * 0xD2511F53u, hi0 = __umulhi(c.x, 0xD2511F53u);
+        const uint32_t lo1 = c.z * 0xCD9E8D57u, hi1 = __umulhi(c.z, 0xCD9E8D57u);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// Stochastic E2M1 code of y with a 16-bit draw u: |y| >= 6 saturates;
+// otherwise lo <= |y| < hi (neighbouring grid values) and the code of hi
+// is taken iff u / 2^16 < (|y| - lo) / (hi - lo).  Every step is exact:
+// the grid spacing is 0.5, 1 or 2 and |y| - lo is a Sterbenz difference.
+__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t u) {
+    const uint32_t sign = (__float_as_uint(y) >> 28) & 8u;
+    const float a = fabsf(y);
+    if (a >= 6.0f) return sign | 7u;
+    uint32_t k;
+    float frac;
+    if (a < 2.0f) {                                // spacing 0.5: codes 0..4
+        const float f = floorf(__fmul_rn(a, 2.0f));
+        k = (uint32_t)f;
+        frac = __fsub_rn(__fmul_rn(a, 2.0f), f);
+    } else if (a < 4.0f) {                         // spacing 1: codes 4..6
+        const float f = floorf(a);
+        k = 2u + (uint32_t)f;
+        frac = __fsub_rn(a, f);
+    } else {                                       // spacing 2: codes 6..7
+        k = 6u;
+        frac = __fmul_rn(__fsub_rn(a, 4.0f), 0.5f);
+    }
+    return sign | (k + (__fmul_rn((float)u, 0x1p-16f) < frac ? 1u : 0u));
+}
+
+// Codes of 16 values y (already multiplied by the block factor), value i
+// of the block in y[i], stochastically rounded with the draws of block n.
+__device__ __forceinline__ uint2 encode16_sr(const float y[16], uint64_t seed, uint64_t n) {
+    uint32_t w[8];
+#pragma unroll
+    for (uint32_t j = 0; j < 2; ++j) {
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)n, (uint32_t)(n >> 32), j, 0u),
+                                      (uint32_t)seed, (uint32_t)(seed >> 32));
+        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = e2m1_sr(y[8 * j + 2 * i], rw[i] & 0xFFFFu);
+            const uint32_t hi = e2m1_sr(y[8 * j + 2 * i + 1], rw[i] >> 16);
+            w[4 * j + i] = lo | (hi << 4);       // byte 4j + i of the block
+        }
+    }
+    return make_uint2(w[0] | (w[1] << 8) | (w[2] << 16) | (w[3] << 24),
+                      w[4] | (w[5] << 8) | (w[6] << 16) | (w[7] << 24));
+}
+
+// Stochastically rounded encode of a BF16 block (scale as encode_block).
+__device__ __forceinline__ EncodeBlockOut encode_block_sr(uint4 a, uint4 b, float g,
+                                                          const EncodeTables &tab, uint64_t seed,
+                                                          uint64_t n) {
+    const uint32_t bits = block_amax_bits(a, b);
+    const uint32_t s = scale_code(bits, g, tab);
+    const float e = tab.inv_s[s & 0x7Fu];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        y[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), e);
+        y[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), e);
+    }
+    EncodeBlockOut o;
+    o.codes = encode16_sr(y, seed, n);
+    o.scale = s;
+    o.finite = bits <= 0x7F7FFFFFu;
+    return o;
+}
+
+// Stochastically rounded encode after the random Hadamard transform.
+__device__ __forceinline__ EncodeBlockOut encode_block_rht_sr(uint4 a, uint4 b, const SignFlips &f,
+                                                              float g, const EncodeTables &tab,
+                                                              uint64_t seed, uint64_t n) {
+    float2 P[8];
+    rht16(a, b, f, P);
+    const uint32_t bits = abs_max_bits(P);
+    const uint32_t s = e4m3_from_f32(__fmul_rn(div6_f32(__uint_as_float(bits)), g));
+    const float e = tab.inv_s[s & 0x7Fu];
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {                  // P[i] = (y_i, y_{i+8})
+        y[i] = __fmul_rn(P[i].x, e);
+        y[i + 8] = __fmul_rn(P[i].y, e);
+    }
+    EncodeBlockOut o;
+    o.codes = encode16_sr(y, seed, n);
+    o.scale = s;
+    o.finite = bits <= 0x7F7FFFFFu;
+    return o;
+}
+
+// The block encoder selected by the compile-time options.
+template <bool kRht, bool kSR>
+__device__ __forceinline__ EncodeBlockOut encode_any(uint4 a, uint4 b, const SignFlips &f, float g,
+                                                     const EncodeTables &tab, uint64_t seed,
+                                                     uint64_t n) {
+    if (kSR) return kRht ? encode_block_rht_sr(a, b, f, g, tab, seed, n) : encode_block_sr(a, b, g, tab, seed, n);
+    return kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
+}
+
 // Byte offset of scale (row r, scale column c) in either layout.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t sf_cols, int64_t col_tiles,
                                              int32_t layout) {

@@ -24,6 +24,7 @@ struct EncodeParams {
     int32_t n_partials;
     uint32_t *status;
     uint32_t rht_mask = 0;  // random Hadamard transform: sign bit j negates value j of a block
+    uint64_t sr_seed = 0;   // stochastic rounding: Philox key
 };
 
 // Quantize / dequantize work unit: one row and kChunkBlocks consecutive
@@ -72,6 +73,10 @@ __global__ void k_encode(EncodeParams p);
 __global__ void k_encode_narrow(EncodeParams p);
 __global__ void k_encode_rht(EncodeParams p);
 __global__ void k_encode_rht_narrow(EncodeParams p);
+__global__ void k_encode_sr(EncodeParams p);
+__global__ void k_encode_sr_narrow(EncodeParams p);
+__global__ void k_encode_rht_sr(EncodeParams p);
+__global__ void k_encode_rht_sr_narrow(EncodeParams p);
 // Column-wise quantization (out = NVFP4 of x^T): p.rows = columns of x,
 // p.cols = rows of x (a multiple of 16), x is p.cols x p.rows with pitch
 // p.ld; 128 threads per CTA.
@@ -83,6 +88,8 @@ __global__ void k_amax_t_rht(const uint16_t *x, int64_t ld, int64_t R, int64_t C
 __global__ void k_encode_t(EncodeParams p);
 __global__ void k_encode_t_rht(EncodeParams p);
 __global__ void k_encode_t_2d(EncodeParams p);
+__global__ void k_encode_t_sr(EncodeParams p);
+__global__ void k_encode_t_rht_sr(EncodeParams p);
 // 2D (16x16 block) row-wise encode: 256 threads; tasks of 16 rows x 256 columns.
 __global__ void k_encode_2d(EncodeParams p);
 inline int64_t transpose_tasks(int64_t x_rows, int64_t out_rows_padded) {

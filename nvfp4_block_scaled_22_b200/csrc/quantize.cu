@@ -160,15 +160,16 @@ struct EncodeShape {
 // gathered padding row), store its codes at cp, and let lanes 4i store the
 // scale word of blocks 4i..4i+3 at sp.  Every lane of the warp takes part
 // (two shuffles).
-template <bool kRht>
+template <bool kRht, bool kSR>
 __device__ __forceinline__ void emit_block(const EncodeParams &p, const EncodeShape &sh,
                                            const SignFlips &flips, float g, const EncodeTables &tab,
-                                           bool real, bool load, int64_t c, uint4 a, uint4 b,
-                                           uint2 *cp, uint8_t *sp, int lane, bool &finite) {
+                                           bool real, bool load, int64_t row, int64_t c, uint4 a,
+                                           uint4 b, uint2 *cp, uint8_t *sp, int lane, bool &finite) {
     uint32_t s = 0;
     if (real && c < sh.sf_cols) {
         if (load) {
-            EncodeBlockOut o = kRht ? encode_block_rht(a, b, flips, g, tab) : encode_block(a, b, g, tab);
+            EncodeBlockOut o = encode_any<kRht, kSR>(a, b, flips, g, tab, p.sr_seed,
+                                                     (uint64_t)row * (uint64_t)sh.sf_cols + (uint64_t)c);
             finite &= o.finite;
             s = o.scale;
             *cp = o.codes;
@@ -206,7 +207,7 @@ __device__ __forceinline__ int64_t source_row(const EncodeParams &p, int64_t row
     return load ? src : 0;
 }
 
-template <bool kRht, bool kNarrow>
+template <bool kRht, bool kNarrow, bool kSR>
 __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     __shared__ uint32_t red[kThreads / 32];
     __shared__ EncodeTables tab;
@@ -255,8 +256,8 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
 #pragma unroll
             for (int j = 0; j < kUnroll; ++j) {
                 if (c0 - lane + 32 * j >= sh.sf_cols4) break;           // uniform across the warp
-                emit_block<kRht>(p, sh, flips, g, tab, real, load, c0 + 32 * j, va[j], vb[j],
-                                 cp + 32 * j, sp + sh.sf_step * j, lane, finite);
+                emit_block<kRht, kSR>(p, sh, flips, g, tab, real, load, row, c0 + 32 * j, va[j],
+                                      vb[j], cp + 32 * j, sp + sh.sf_step * j, lane, finite);
             }
         }
     } else {
@@ -297,8 +298,9 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
                 if (t >= tasks) break;                               // uniform across the warp
                 uint32_t s = 0;
                 if (has[u]) {
-                    EncodeBlockOut o = kRht ? encode_block_rht(va[u], vb[u], flips, g, tab)
-                                            : encode_block(va[u], vb[u], g, tab);
+                    EncodeBlockOut o = encode_any<kRht, kSR>(
+                        va[u], vb[u], flips, g, tab, p.sr_seed,
+                        (uint64_t)rr[u] * (uint64_t)sh.sf_cols + (uint64_t)bb[u]);
                     finite &= o.finite;
                     s = o.scale;
                     *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;
@@ -326,18 +328,37 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
 
 // The host launches the *_narrow kernels for rows of fewer than
 // kChunkBlocks blocks (tasks_are_groups).
-__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) { encode_body<false, false>(p); }
+__global__ void __launch_bounds__(kThreads) k_encode(EncodeParams p) {
+    encode_body<false, false, false>(p);
+}
 
 __global__ void __launch_bounds__(kThreads) k_encode_narrow(EncodeParams p) {
-    encode_body<false, true>(p);
+    encode_body<false, true, false>(p);
 }
 
 __global__ void __launch_bounds__(kThreads, 3) k_encode_rht(EncodeParams p) {
-    encode_body<true, false>(p);
+    encode_body<true, false, false>(p);
 }
 
 __global__ void __launch_bounds__(kThreads, 3) k_encode_rht_narrow(EncodeParams p) {
-    encode_body<true, true>(p);
+    encode_body<true, true, false>(p);
+}
+
+// Stochastically rounded codes (p.sr_seed), with or without the transform.
+__global__ void __launch_bounds__(kThreads) k_encode_sr(EncodeParams p) {
+    encode_body<false, false, true>(p);
+}
+
+__global__ void __launch_bounds__(kThreads) k_encode_sr_narrow(EncodeParams p) {
+    encode_body<false, true, true>(p);
+}
+
+__global__ void __launch_bounds__(kThreads) k_encode_rht_sr(EncodeParams p) {
+    encode_body<true, false, true>(p);
+}
+
+__global__ void __launch_bounds__(kThreads) k_encode_rht_sr_narrow(EncodeParams p) {
+    encode_body<true, true, true>(p);
 }
 
 // ------------------------------------------------------------ k_encode_2d

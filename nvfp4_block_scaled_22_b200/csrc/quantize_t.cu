@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__rest
 // -------------------------------------------------------------- k_encode_t
 // kTwoD: one scale per 16x16 block of x (16 rows x 16 columns, the 2D
 // weight blocks), so the output is the 2D quantization of x^T.
-template <bool kRht, bool kTwoD>
+template <bool kRht, bool kTwoD, bool kSR>
 __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
     extern __shared__ uint4 dyn_smem[];
     __shared__ uint32_t red[kTThreads / 32];
@@ -218,8 +218,11 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
                            o0 = encode_block_amax(a, b, m, g, tab);
                            o1 = encode_block_amax(c, d, m, g, tab);
                        } else {
-                           o0 = kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
-                           o1 = kRht ? encode_block_rht(c, d, f, g, tab) : encode_block(c, d, g, tab);
+                           // output block n = output row * (R / 16) + block column
+                           const uint64_t n0 = (uint64_t)(c0 + 2 * lane) * (uint64_t)sf_cols +
+                                               (uint64_t)(r0 / 16 + k);
+                           o0 = encode_any<kRht, kSR>(a, b, f, g, tab, p.sr_seed, n0);
+                           o1 = encode_any<kRht, kSR>(c, d, f, g, tab, p.sr_seed, n0 + (uint64_t)sf_cols);
                        }
                        finite &= o0.finite && o1.finite;
                        code0[k] = o0.codes;
@@ -237,28 +240,38 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
 }
 
 __global__ void __launch_bounds__(kTThreads) k_encode_t(EncodeParams p) {
-    encode_t_body<false, false>(p);
+    encode_t_body<false, false, false>(p);
 }
 
 __global__ void __launch_bounds__(kTThreads) k_encode_t_rht(EncodeParams p) {
-    encode_t_body<true, false>(p);
+    encode_t_body<true, false, false>(p);
 }
 
 __global__ void __launch_bounds__(kTThreads) k_encode_t_2d(EncodeParams p) {
-    encode_t_body<false, true>(p);
+    encode_t_body<false, true, false>(p);
+}
+
+__global__ void __launch_bounds__(kTThreads) k_encode_t_sr(EncodeParams p) {
+    encode_t_body<false, false, true>(p);
+}
+
+__global__ void __launch_bounds__(kTThreads) k_encode_t_rht_sr(EncodeParams p) {
+    encode_t_body<true, false, true>(p);
 }
 
 // Launch with the dynamic shared memory of two tile buffers per warp (the
 // size limit is raised once per device).
 cudaError_t launch_transpose_kernel(const void *kernel, int grid, void **args, cudaStream_t stream) {
-    static bool attr_set[64][4] = {};
-    const void *kernels[4] = {(const void *)k_amax_t_rht, (const void *)k_encode_t,
-                              (const void *)k_encode_t_rht, (const void *)k_encode_t_2d};
+    constexpr int kKernels = 6;
+    static bool attr_set[64][kKernels] = {};
+    const void *kernels[kKernels] = {(const void *)k_amax_t_rht, (const void *)k_encode_t,
+                                     (const void *)k_encode_t_rht, (const void *)k_encode_t_2d,
+                                     (const void *)k_encode_t_sr, (const void *)k_encode_t_rht_sr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int which = -1;
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kKernels; ++i)
         if (kernels[i] == kernel) which = i;
     if (which < 0) return cudaErrorInvalidDeviceFunction;
     if (dev < 0 || dev >= 64 || !attr_set[dev][which]) {

@@ -77,6 +77,11 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     assert lib.nvfp4_quantize_2d(16, 32, t, tt, 0, 16, 1 << 16, 0) == 3         # rows % 16 with W^T
     tt = binding.CTensor(16, 16, 16, 32, 48, 0)
     assert lib.nvfp4_quantize_2d(16, 32, t, tt, 0, 16, 1 << 16, 0) == 3         # W^T shape
+    t = binding.CTensor(16, 16, 16, 16, 32, 0)
+    assert lib.nvfp4_quantize_sr(16, 32, 2, 0, 0, 1, t, 0, 16, 1 << 16, 0) == 1  # transposed flag
+    assert lib.nvfp4_quantize_sr(16, 32, 0, 0, 1 << 16, 1, t, 0, 16, 1 << 16, 0) == 1   # mask
+    t = binding.CTensor(16, 16, 16, 12, 32, 0)
+    assert lib.nvfp4_quantize_sr(16, 32, 1, 0, 0, 1, t, 0, 16, 1 << 16, 0) == 3  # x columns % 8
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
