@@ -552,6 +552,73 @@ def workload_line(name, args, device):
                                   "bytes_per_value": QUANT_BYTES_PER_VALUE_2PASS,
                                   "peak_source": f"{peak_src} hbm_gbs"}})
         return line
+    if name == "train":
+        # One NVFP4 linear layer of the ffn, forward and backward, in the
+        # recipe's roles: Fprop Y = X W^T; Dgrad dX = dY W (dY stochastically
+        # rounded, W^T from the 2D blocks); Wgrad dW = dY^T X (both operands
+        # column-wise with the Hadamard transform, dY stochastically rounded).
+        m = inputs.WGRAD_M
+        mask = inputs.rht_sign_mask(0)
+        w = inputs.ffn_weight(device=device)                      # N x K
+        x = inputs.ffn_activation(m, device=device)                # M x K
+        dy = inputs.wgrad_grad_output_t(m, device=device).t().contiguous()   # M x N
+        qw = nb.NVFP4Tensor.empty(N, K, device=device)
+        qwt = nb.NVFP4Tensor.empty(K, N, device=device)
+        qx = nb.NVFP4Tensor.empty(m, K, device=device)
+        qdy = nb.NVFP4Tensor.empty(m, N, device=device)
+        qdyt = nb.NVFP4Tensor.empty(N, m, device=device)
+        qxt = nb.NVFP4Tensor.empty(K, m, device=device)
+        y = torch.empty((m, N), dtype=torch.bfloat16, device=device)
+        dx = torch.empty((m, K), dtype=torch.bfloat16, device=device)
+        dw = torch.empty((N, K), dtype=torch.bfloat16, device=device)
+        names = ["quantize_2d_w", "quantize_x", "fprop_gemm", "quantize_sr_dy", "dgrad_gemm",
+                 "quantize_t_sr_rht_dy", "quantize_t_rht_x", "wgrad_gemm"]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        seed = [0]
+
+        def step(mark=False):
+            seed[0] += 1
+            ops = [lambda: nb.nvfp4_quantize_2d(w, out=qw, out_t=qwt, workspace=ws),
+                   lambda: nb.nvfp4_quantize(x, out=qx, workspace=ws),
+                   lambda: nb.nvfp4_gemm(qx, qw, out=y, workspace=ws),
+                   lambda: nb.nvfp4_quantize_sr(dy, 2 * seed[0], out=qdy, workspace=ws),
+                   lambda: nb.nvfp4_gemm(qdy, qwt, out=dx, workspace=ws),
+                   lambda: nb.nvfp4_quantize_sr(dy, 2 * seed[0] + 1, out=qdyt, transposed=True,
+                                                sign_mask=mask, workspace=ws),
+                   lambda: nb.nvfp4_quantize_t(x, out=qxt, sign_mask=mask, workspace=ws),
+                   lambda: nb.nvfp4_gemm(qdyt, qxt, out=dw, workspace=ws)]
+            for i, op in enumerate(ops):
+                if mark:
+                    ev[i].record()
+                op()
+            if mark:
+                ev[-1].record()
+
+        ms = _timed(step, args.steps, args.warmup, flush)
+        parts = {n: [] for n in names}
+        for _ in range(max(3, min(args.steps, 10))):
+            flush()
+            step(mark=True)
+            torch.cuda.synchronize()
+            for i, n in enumerate(names):
+                parts[n].append(ev[i].elapsed_time(ev[i + 1]))
+        parts = {n: statistics.median(v) for n, v in parts.items()}
+        st = nb.nvfp4_check_status(ws)
+        flops = 3 * 2.0 * m * N * K
+        gemm_ms = parts["fprop_gemm"] + parts["dgrad_gemm"] + parts["wgrad_gemm"]
+        q_ms = ms - gemm_ms
+        line.update({"metric": "NVFP4 linear-layer training step TFLOP/s (Fprop + Dgrad + Wgrad)",
+                     "value": flops / ms / 1e9, "unit": "TFLOP/s", "higher_is_better": True,
+                     "ms_per_step": ms,
+                     "config": {"workload": f"ffn linear {N} x {K}, {m} tokens: 2D-block W, SR "
+                                            "gradients, RHT on the Wgrad operands", "l2": "flushed"},
+                     "phase_ms": parts, "gemm_tflops": flops / gemm_ms / 1e9, "status": st,
+                     "roofline": {"kernel": "k_gemm_nvf4 (three GEMMs)", "bound": "tensor",
+                                  "achieved": flops / gemm_ms / 1e9, "peak": fp4_peak,
+                                  "unit": "TFLOP/s", "frac": flops / gemm_ms / 1e9 / fp4_peak,
+                                  "quantize_share": q_ms / ms,
+                                  "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g}"}})
+        return line
     raise ValueError(name)
 
 
@@ -569,7 +636,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--workload", default="ffn8192",
-                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad"],
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")

@@ -585,7 +585,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.gw = gw;
     p.a_row_blocks = (int32_t)ceil_div(A->rows, 128);
     p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
-    p.n_fastest = (A->rows * (k / 2) > kL2SweepBytes && W->rows * (k / 2) <= kL2SweepBytes) ? 1 : 0;
+    p.n_fastest = (A->rows * (k / 2) > kL2SweepBytes && A->rows > W->rows) ? 1 : 0;
     p.status = reinterpret_cast<uint32_t *>(workspace);
     p.timeout_cycles = g_timeout_cycles;
     if (pair) {

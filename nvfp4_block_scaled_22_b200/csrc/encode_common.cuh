@@ -285,44 +285,51 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 
 // Stochastic E2M1 code of y with a 16-bit draw u: |y| >= 6 saturates;
 // otherwise lo <= |y| < hi (neighbouring grid values) and the code of hi
-// is taken iff u / 2^16 < (|y| - lo) / (hi - lo).  Every step is exact:
-// the grid spacing is 0.5, 1 or 2 and |y| - lo is a Sterbenz difference.
+// is taken iff u / 2^16 < (|y| - lo) / (hi - lo).  Evaluated on the FP32
+// bit pattern, exactly: for |y| in [1, 6) the grid keeps one mantissa bit,
+// so lo is |y| with its lower 22 mantissa bits cleared, its code is
+// (exponent - 126) * 2 + top mantissa bit, and the fraction is those 22
+// bits / 2^22 (u / 2^16 < f  <=>  u * 64 < bits); on [0.5, 1) lo = 0.5 and
+// the fraction is the 23 mantissa bits / 2^23; below 0.5 lo = 0 and the
+// fraction is 2|y| (compared as u < |y| * 2^17, exact in FP32).
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t u) {
-    const uint32_t sign = (__float_as_uint(y) >> 28) & 8u;
-    const float a = fabsf(y);
-    if (a >= 6.0f) return sign | 7u;
-    uint32_t k;
-    float frac;
-    if (a < 2.0f) {                                // spacing 0.5: codes 0..4
-        const float f = floorf(__fmul_rn(a, 2.0f));
-        k = (uint32_t)f;
-        frac = __fsub_rn(__fmul_rn(a, 2.0f), f);
-    } else if (a < 4.0f) {                         // spacing 1: codes 4..6
-        const float f = floorf(a);
-        k = 2u + (uint32_t)f;
-        frac = __fsub_rn(a, f);
-    } else {                                       // spacing 2: codes 6..7
-        k = 6u;
-        frac = __fmul_rn(__fsub_rn(a, 4.0f), 0.5f);
-    }
-    return sign | (k + (__fmul_rn((float)u, 0x1p-16f) < frac ? 1u : 0u));
+    const uint32_t bits = __float_as_uint(y);
+    const uint32_t sign = (bits >> 28) & 8u;
+    const uint32_t mag = bits & 0x7FFFFFFFu;
+    const uint32_t e = mag >> 23, m = mag & 0x7FFFFFu;
+    // selects, not branches: the lanes of a warp hold values of every range
+    const bool ge1 = e >= 127u;
+    const uint32_t code_n = ge1 ? (((e - 126u) << 1) | (m >> 22)) : 1u;       // [0.5, 6)
+    const bool up_n = (u << (ge1 ? 6 : 7)) < (m & (ge1 ? 0x3FFFFFu : 0x7FFFFFu));
+    const bool up_s = (float)u < __fmul_rn(__uint_as_float(mag), 131072.0f);   // [0, 0.5)
+    const uint32_t code = (e >= 126u) ? code_n + (up_n ? 1u : 0u) : (up_s ? 1u : 0u);
+    return sign | (mag >= 0x40C00000u ? 7u : code);                          // |y| >= 6
+}
+
+// The two Philox draws of output block n (see above).
+struct BlockDraws {
+    uint4 d0, d1;
+};
+
+__device__ __forceinline__ BlockDraws block_draws(uint64_t seed, uint64_t n) {
+    BlockDraws r;
+    r.d0 = philox4x32_10(make_uint4((uint32_t)n, (uint32_t)(n >> 32), 0u, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+    r.d1 = philox4x32_10(make_uint4((uint32_t)n, (uint32_t)(n >> 32), 1u, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+    return r;
 }
 
 // Codes of 16 values y (already multiplied by the block factor), value i
-// of the block in y[i], stochastically rounded with the draws of block n.
-__device__ __forceinline__ uint2 encode16_sr(const float y[16], uint64_t seed, uint64_t n) {
+// of the block in y[i], stochastically rounded with the block's draws.
+__device__ __forceinline__ uint2 encode16_sr(const float y[16], const BlockDraws &r) {
+    const uint32_t rw[8] = {r.d0.x, r.d0.y, r.d0.z, r.d0.w, r.d1.x, r.d1.y, r.d1.z, r.d1.w};
     uint32_t w[8];
 #pragma unroll
-    for (uint32_t j = 0; j < 2; ++j) {
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)n, (uint32_t)(n >> 32), j, 0u),
-                                      (uint32_t)seed, (uint32_t)(seed >> 32));
-        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = e2m1_sr(y[8 * j + 2 * i], rw[i] & 0xFFFFu);
-            const uint32_t hi = e2m1_sr(y[8 * j + 2 * i + 1], rw[i] >> 16);
-            w[4 * j + i] = lo | (hi << 4);       // byte 4j + i of the block
-        }
+    for (int i = 0; i < 8; ++i) {                  // byte i of the block: values 2i, 2i + 1
+        const uint32_t lo = e2m1_sr(y[2 * i], rw[i] & 0xFFFFu);
+        const uint32_t hi = e2m1_sr(y[2 * i + 1], rw[i] >> 16);
+        w[i] = lo | (hi << 4);
     }
     return make_uint2(w[0] | (w[1] << 8) | (w[2] << 16) | (w[3] << 24),
                       w[4] | (w[5] << 8) | (w[6] << 16) | (w[7] << 24));
@@ -330,8 +337,8 @@ __device__ __forceinline__ uint2 encode16_sr(const float y[16], uint64_t seed, u
 
 // Stochastically rounded encode of a BF16 block (scale as encode_block).
 __device__ __forceinline__ EncodeBlockOut encode_block_sr(uint4 a, uint4 b, float g,
-                                                          const EncodeTables &tab, uint64_t seed,
-                                                          uint64_t n) {
+                                                          const EncodeTables &tab,
+                                                          const BlockDraws &r) {
     const uint32_t bits = block_amax_bits(a, b);
     const uint32_t s = scale_code(bits, g, tab);
     const float e = tab.inv_s[s & 0x7Fu];
@@ -343,7 +350,7 @@ __device__ __forceinline__ EncodeBlockOut encode_block_sr(uint4 a, uint4 b, floa
         y[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), e);
     }
     EncodeBlockOut o;
-    o.codes = encode16_sr(y, seed, n);
+    o.codes = encode16_sr(y, r);
     o.scale = s;
     o.finite = bits <= 0x7F7FFFFFu;
     return o;
@@ -352,7 +359,7 @@ __device__ __forceinline__ EncodeBlockOut encode_block_sr(uint4 a, uint4 b, floa
 // Stochastically rounded encode after the random Hadamard transform.
 __device__ __forceinline__ EncodeBlockOut encode_block_rht_sr(uint4 a, uint4 b, const SignFlips &f,
                                                               float g, const EncodeTables &tab,
-                                                              uint64_t seed, uint64_t n) {
+                                                              const BlockDraws &r) {
     float2 P[8];
     rht16(a, b, f, P);
     const uint32_t bits = abs_max_bits(P);
@@ -365,18 +372,18 @@ __device__ __forceinline__ EncodeBlockOut encode_block_rht_sr(uint4 a, uint4 b, 
         y[i + 8] = __fmul_rn(P[i].y, e);
     }
     EncodeBlockOut o;
-    o.codes = encode16_sr(y, seed, n);
+    o.codes = encode16_sr(y, r);
     o.scale = s;
     o.finite = bits <= 0x7F7FFFFFu;
     return o;
 }
 
-// The block encoder selected by the compile-time options.
+// The block encoder selected by the compile-time options (r: the block's
+// draws, used with kSR only).
 template <bool kRht, bool kSR>
 __device__ __forceinline__ EncodeBlockOut encode_any(uint4 a, uint4 b, const SignFlips &f, float g,
-                                                     const EncodeTables &tab, uint64_t seed,
-                                                     uint64_t n) {
-    if (kSR) return kRht ? encode_block_rht_sr(a, b, f, g, tab, seed, n) : encode_block_sr(a, b, g, tab, seed, n);
+                                                     const EncodeTables &tab, const BlockDraws &r) {
+    if (kSR) return kRht ? encode_block_rht_sr(a, b, f, g, tab, r) : encode_block_sr(a, b, g, tab, r);
     return kRht ? encode_block_rht(a, b, f, g, tab) : encode_block(a, b, g, tab);
 }
 

@@ -92,8 +92,8 @@ struct TileInfo {
 
 // Tile order: M fastest (the CTAs working at one time share a few W
 // column tiles and sweep all of A, which then has to stay in L2), or, when
-// A is too large for that and W is not, N fastest (they share a few A row
-// tiles and sweep all of W).
+// A is large and W is the smaller operand, N fastest (they share a few A
+// row tiles and sweep all of W).
 __device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, int ntiles,
                                               const GemmParams &p, const int *s_off,
                                               const int *s_rows) {

@@ -55,8 +55,9 @@ cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const Ge
 cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                              int clusters, cudaStream_t stream);
 
-// Tile order: N fastest when A's codes exceed this many bytes and W's do
-// not (the operand swept by the CTAs working at one time must stay in L2).
+// Tile order: the CTAs working at one time sweep one operand, which must
+// stay in L2.  M fastest sweeps A; when A's codes exceed this many bytes
+// and W is the smaller operand, N fastest sweeps W instead.
 constexpr int64_t kL2SweepBytes = 48ll << 20;
 
 // Dense GEMMs with at least this many rows run on CTA pairs.

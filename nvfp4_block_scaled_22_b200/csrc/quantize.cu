@@ -163,13 +163,13 @@ struct EncodeShape {
 template <bool kRht, bool kSR>
 __device__ __forceinline__ void emit_block(const EncodeParams &p, const EncodeShape &sh,
                                            const SignFlips &flips, float g, const EncodeTables &tab,
-                                           bool real, bool load, int64_t row, int64_t c, uint4 a,
-                                           uint4 b, uint2 *cp, uint8_t *sp, int lane, bool &finite) {
+                                           bool real, bool load, int64_t c, uint4 a, uint4 b,
+                                           const BlockDraws &r, uint2 *cp, uint8_t *sp, int lane,
+                                           bool &finite) {
     uint32_t s = 0;
     if (real && c < sh.sf_cols) {
         if (load) {
-            EncodeBlockOut o = encode_any<kRht, kSR>(a, b, flips, g, tab, p.sr_seed,
-                                                     (uint64_t)row * (uint64_t)sh.sf_cols + (uint64_t)c);
+            EncodeBlockOut o = encode_any<kRht, kSR>(a, b, flips, g, tab, r);
             finite &= o.finite;
             s = o.scale;
             *cp = o.codes;
@@ -251,13 +251,22 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
                     vb[j] = __ldg(xp + 64 * j + 1);
                 }
             }
+            // stochastic rounding: all draws of the task first (independent
+            // Philox chains, so their latencies overlap)
+            BlockDraws rnd[kUnroll];
+            if (kSR) {
+#pragma unroll
+                for (int j = 0; j < kUnroll; ++j)
+                    rnd[j] = block_draws(p.sr_seed, (uint64_t)row * (uint64_t)sh.sf_cols +
+                                                        (uint64_t)(c0 + 32 * j));
+            }
             uint2 *cp = reinterpret_cast<uint2 *>(p.codes + row * (p.cols / 2) + c0 * 8);
             uint8_t *sp = p.scales + sf_offset(row, c0, sh.sf_cols, sh.col_tiles, p.layout);
 #pragma unroll
             for (int j = 0; j < kUnroll; ++j) {
                 if (c0 - lane + 32 * j >= sh.sf_cols4) break;           // uniform across the warp
-                emit_block<kRht, kSR>(p, sh, flips, g, tab, real, load, row, c0 + 32 * j, va[j],
-                                      vb[j], cp + 32 * j, sp + sh.sf_step * j, lane, finite);
+                emit_block<kRht, kSR>(p, sh, flips, g, tab, real, load, c0 + 32 * j, va[j], vb[j],
+                                      rnd[j], cp + 32 * j, sp + sh.sf_step * j, lane, finite);
             }
         }
     } else {
@@ -292,15 +301,19 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
                     vb[u] = __ldg(xp + 1);
                 }
             }
+            BlockDraws rnd[kUnroll];
+            if (kSR) {
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    rnd[u] = block_draws(p.sr_seed, (uint64_t)rr[u] * (uint64_t)sh.sf_cols + (uint64_t)bb[u]);
+            }
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const uint32_t t = t0 + warps * u;
                 if (t >= tasks) break;                               // uniform across the warp
                 uint32_t s = 0;
                 if (has[u]) {
-                    EncodeBlockOut o = encode_any<kRht, kSR>(
-                        va[u], vb[u], flips, g, tab, p.sr_seed,
-                        (uint64_t)rr[u] * (uint64_t)sh.sf_cols + (uint64_t)bb[u]);
+                    EncodeBlockOut o = encode_any<kRht, kSR>(va[u], vb[u], flips, g, tab, rnd[u]);
                     finite &= o.finite;
                     s = o.scale;
                     *reinterpret_cast<uint2 *>(p.codes + rr[u] * (p.cols / 2) + bb[u] * 8) = o.codes;

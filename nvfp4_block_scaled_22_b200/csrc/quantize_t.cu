@@ -219,10 +219,15 @@ __device__ __forceinline__ void encode_t_body(const EncodeParams &p) {
                            o1 = encode_block_amax(c, d, m, g, tab);
                        } else {
                            // output block n = output row * (R / 16) + block column
-                           const uint64_t n0 = (uint64_t)(c0 + 2 * lane) * (uint64_t)sf_cols +
-                                               (uint64_t)(r0 / 16 + k);
-                           o0 = encode_any<kRht, kSR>(a, b, f, g, tab, p.sr_seed, n0);
-                           o1 = encode_any<kRht, kSR>(c, d, f, g, tab, p.sr_seed, n0 + (uint64_t)sf_cols);
+                           BlockDraws r0d, r1d;
+                           if (kSR) {
+                               const uint64_t n0 = (uint64_t)(c0 + 2 * lane) * (uint64_t)sf_cols +
+                                                   (uint64_t)(r0 / 16 + k);
+                               r0d = block_draws(p.sr_seed, n0);
+                               r1d = block_draws(p.sr_seed, n0 + (uint64_t)sf_cols);
+                           }
+                           o0 = encode_any<kRht, kSR>(a, b, f, g, tab, r0d);
+                           o1 = encode_any<kRht, kSR>(c, d, f, g, tab, r1d);
                        }
                        finite &= o0.finite && o1.finite;
                        code0[k] = o0.codes;

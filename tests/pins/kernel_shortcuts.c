@@ -12,13 +12,21 @@
  *    multiply-add, and the corrected quotient RN(q + r * c) by a second one
  *    (the FMA-based correction step of Markstein, "IA-64 and Elementary
  *    Functions", 2000).
+ * 3. Stochastic rounding onto the E2M1 grid evaluated on the binary32 bit
+ *    pattern (lower bound by clearing mantissa bits, up-decision by an
+ *    integer compare of the draw with the cleared bits), against the
+ *    oracle's definition (neighbouring grid values, fraction compared with
+ *    u / 2^16 in double).
  */
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 
 static float f32(uint32_t u) { float x; memcpy(&x, &u, 4); return x; }
+
+uint8_t nvo_e2m1_sr(float y, uint32_t u16);
 static uint32_t bits(float x) { uint32_t u; memcpy(&u, &x, 4); return u; }
+static uint32_t bits_of(float x) { return bits(x); }
 
 /* Shortcut 1 over every non-negative finite BF16 pattern whose quotient is
  * normal (exponent field e of a in [4, 255)).  Returns mismatches. */
@@ -54,5 +62,33 @@ int64_t shortcut_div6_fma(uint32_t lo, uint32_t hi)
         if (bits(q1) != bits(a / 6.0f))
             ++bad;
     }
+    return bad;
+}
+
+static uint32_t sr_bits(float y, uint32_t u)
+{
+    uint32_t bits = bits_of(y);
+    uint32_t sign = (bits >> 28) & 8u, mag = bits & 0x7FFFFFFFu;
+    uint32_t e = mag >> 23, m = mag & 0x7FFFFFu;
+    int ge1 = e >= 127u;
+    uint32_t code_n = ge1 ? (((e - 126u) << 1) | (m >> 22)) : 1u;
+    int up_n = (u << (ge1 ? 6 : 7)) < (m & (ge1 ? 0x3FFFFFu : 0x7FFFFFu));
+    int up_s = (float)u < f32(mag) * 131072.0f;
+    uint32_t code = (e >= 126u) ? code_n + (uint32_t)up_n : (uint32_t)up_s;
+    return sign | (mag >= 0x40C00000u ? 7u : code);
+}
+
+/* Shortcut 3 over the binary32 patterns [lo, hi) (both signs) and the
+ * given draws.  Returns mismatches against the oracle's definition. */
+int64_t shortcut_sr(uint32_t lo, uint32_t hi, const uint32_t *draws, int n_draws, uint32_t stride)
+{
+    int64_t bad = 0;
+    for (uint64_t p = lo; p < hi; p += stride)
+        for (int i = 0; i < n_draws; ++i)
+            for (uint32_t s = 0; s < 2; ++s) {
+                float y = f32((uint32_t)p | (s << 31));
+                if (sr_bits(y, draws[i]) != nvo_e2m1_sr(y, draws[i]))
+                    ++bad;
+            }
     return bad;
 }

@@ -12,6 +12,8 @@ def _lib():
     L.shortcut_div6_table.restype = C.c_int64
     L.shortcut_div6_fma.restype = C.c_int64
     L.shortcut_div6_fma.argtypes = [C.c_uint32, C.c_uint32]
+    L.shortcut_sr.restype = C.c_int64
+    L.shortcut_sr.argtypes = [C.c_uint32, C.c_uint32, C.c_void_p, C.c_int, C.c_uint32]
     return L
 
 
@@ -29,3 +31,21 @@ def test_fp32_amax_over_six_fma_correction():
     assert L.shortcut_div6_fma(*binade(0)) == 0
     assert L.shortcut_div6_fma(0x01C00000, binade(-122)[1]) == 0   # 1.5 * 2^-124 .. 2^-121
     assert L.shortcut_div6_fma(*binade(127)) == 0
+
+
+def test_stochastic_rounding_on_the_bit_pattern():
+    """Every 31st binary32 magnitude below 8 with draws at the ends and in
+    the middle of the range, every 211th with 64 random draws, and every
+    pattern within 2^14 ulps of each grid value and segment boundary."""
+    import struct
+
+    import numpy as np
+    L = _lib()
+    draws = np.array([0, 1, 2, 63, 64, 0x7FFF, 0x8000, 0xFFFE, 0xFFFF], np.uint32)
+    assert L.shortcut_sr(0, 0x41000000, draws.ctypes.data, len(draws), 31) == 0
+    rnd = np.random.default_rng(5).integers(0, 1 << 16, 64).astype(np.uint32)
+    assert L.shortcut_sr(0, 0x41000000, rnd.ctypes.data, len(rnd), 211) == 0
+    for v in (0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0):
+        b = struct.unpack("<I", struct.pack("<f", v))[0]
+        assert L.shortcut_sr(b - (1 << 14), b + (1 << 14), draws.ctypes.data, len(draws), 1) == 0
+    assert L.shortcut_sr(0, 1 << 15, draws.ctypes.data, len(draws), 1) == 0   # zero and subnormals
