@@ -44,8 +44,8 @@ FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
 # the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
 # Reported only while the kernel's sources hash to the profiled version.
-GEMM_TRAFFIC_BYTES = 86.6e6 + 292.3e6
-GEMM_TRAFFIC_SRC_SHA = "a6d927ba934dfbba"
+GEMM_TRAFFIC_BYTES = 87.05e6 + 292.46e6
+GEMM_TRAFFIC_SRC_SHA = "6159f8c67b83198d"
 GEMM_SOURCES = ("gemm.cu", "gemm.h", "ptx.cuh")
 
 
