@@ -28,6 +28,11 @@
  *       so that the transposed weight holds the same quantized values;
  *       gradients are rounded stochastically (a value 0.7 of the way from
  *       one grid point to the next goes up with probability 0.7).
+ *  [PM] MXFP4, the format the pages compare NVFP4 with: "NVIDIA shrank
+ *       GLM-5.2 to 4 bits" section 3 (blocks of 32, power-of-two E8M0
+ *       scale), pre-training page section "E2M1 format and two-level
+ *       scaling" (32 values per UE8M0 scale, no tensor scale), KV page
+ *       section "FP4 formats compared" (about 4.25 bits per value).
  *  [PX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *       1, 2, 3" (SC 2011): the Philox4x32-10 counter-based generator.
  *  The FP32 evaluation order below is the convention the hot path is
@@ -666,4 +671,122 @@ int nvo_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, i
             }
         }
     return NVO_OK;
+}
+
+/* ------------------------------------------------------------------ MXFP4 */
+
+/* [PM] UE8M0 block scale: byte b encodes 2^(b - 127); 255 is NaN. */
+double nvo_ue8m0_decode(uint8_t b)
+{
+    return (b == 255) ? NAN : ldexp(1.0, (int)b - 127);
+}
+
+int64_t nvo_mx_scales_bytes(int64_t rows, int64_t cols, int layout)
+{
+    int64_t s = cols / 32;
+    if (layout == NVO_SF_LINEAR)
+        return rows * s;
+    return (rows + 127) / 128 * 128 * ((s + 3) / 4 * 4);
+}
+
+/* Scale positions: the 128x4 tiled layout (or row-major) over the
+ * cols / 32 scale columns, as for NVFP4 over cols / 16. */
+int64_t nvo_mx_sf_offset(int64_t r, int64_t c, int64_t cols, int layout)
+{
+    int64_t s = cols / 32;
+    if (layout == NVO_SF_LINEAR)
+        return r * s + c;
+    int64_t sp = (s + 3) / 4 * 4;
+    return ((r / 128) * (sp / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+/* [PM] Shared exponent of a 32-value block.  READING (the pages fix only
+ * "power of two"): the OCP microscaling rule X = floor(log2(amax)) - 2,
+ * 2 being the exponent of the largest E2M1 value (6 = 1.5 * 2^2), so the
+ * block amax lands in [4, 8) after scaling (values above 6 saturate);
+ * clamped to [-127, 127]; an all-zero block takes X = -127. */
+int nvo_mx_exponent(float amax)
+{
+    if (amax == 0.0f)
+        return -127;
+    int ex;
+    frexp((double)amax, &ex);          /* amax = f * 2^ex, f in [0.5, 1) */
+    int X = ex - 1 - 2;
+    if (X < -127)
+        X = -127;
+    if (X > 127)
+        X = 127;
+    return X;
+}
+
+/* [PM] MXFP4 quantization: per 32 consecutive values of a row, the scale
+ * byte X + 127 and codes e2m1_rne_satfinite(RN(x * 2^-X)) (the product by
+ * a power of two is exact unless it underflows).  No tensor scale.  Returns
+ * NVO_ERR_NONFINITE for Inf/NaN input (outputs unspecified). */
+int nvo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes,
+                    uint8_t *scales, int layout)
+{
+    if (cols % 32 != 0 || rows < 0 || cols < 0)
+        return NVO_ERR_SHAPE;
+    memset(scales, 0, (size_t)nvo_mx_scales_bytes(rows, cols, layout));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 32; ++b) {
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float v = fabsf(nvo_bf16_to_f32(x[r * ld + b * 32 + i]));
+                if (!isfinite(v))
+                    return NVO_ERR_NONFINITE;
+                if (v > amax)
+                    amax = v;
+            }
+            int X = nvo_mx_exponent(amax);
+            scales[nvo_mx_sf_offset(r, b, cols, layout)] = (uint8_t)(X + 127);
+            float inv = ldexpf(1.0f, -X);
+            uint8_t *cb = codes + r * (cols / 2) + b * 16;
+            for (int i = 0; i < 16; ++i) {
+                uint8_t c0 = nvo_e2m1_rne_satfinite(nvo_bf16_to_f32(x[r * ld + b * 32 + 2 * i]) * inv);
+                uint8_t c1 = nvo_e2m1_rne_satfinite(nvo_bf16_to_f32(x[r * ld + b * 32 + 2 * i + 1]) * inv);
+                cb[i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return NVO_OK;
+}
+
+/* x_hat = bf16(e2m1(code) * 2^X), exact before the BF16 rounding. */
+void nvo_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int layout, int64_t rows,
+                       int64_t cols, uint16_t *y, int64_t ld)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = codes[r * (cols / 2) + c / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+            double v = (double)nvo_e2m1_decode(code) *
+                       nvo_ue8m0_decode(scales[nvo_mx_sf_offset(r, c / 32, cols, layout)]);
+            y[r * ld + c] = nvo_f32_to_bf16((float)v);
+        }
+}
+
+/* Sampled FP64 reference of D = Ahat * What^T for MXFP4 operands (no
+ * tensor scales): ref[t] and abs[t] as in nvo_gemm_ref. */
+void nvo_gemm_ref_mx(const uint8_t *a_codes, const uint8_t *a_scales, int a_layout, int64_t m,
+                     const uint8_t *w_codes, const uint8_t *w_scales, int w_layout, int64_t n,
+                     int64_t k, const int64_t *i_idx, const int64_t *j_idx, int64_t count,
+                     double *ref, double *abs_out)
+{
+    (void)m;
+    (void)n;
+    for (int64_t t = 0; t < count; ++t) {
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t c = 0; c < k; ++c) {
+            uint8_t ab = a_codes[i_idx[t] * (k / 2) + c / 2], wb = w_codes[j_idx[t] * (k / 2) + c / 2];
+            double av = nvo_e2m1_decode((c & 1) ? (ab >> 4) : (ab & 15)) *
+                        nvo_ue8m0_decode(a_scales[nvo_mx_sf_offset(i_idx[t], c / 32, k, a_layout)]);
+            double wv = nvo_e2m1_decode((c & 1) ? (wb >> 4) : (wb & 15)) *
+                        nvo_ue8m0_decode(w_scales[nvo_mx_sf_offset(j_idx[t], c / 32, k, w_layout)]);
+            acc += av * wv;
+            aacc += fabs(av * wv);
+        }
+        ref[t] = acc;
+        abs_out[t] = aacc;
+    }
 }

@@ -19,6 +19,8 @@ __all__ = [
     "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
     "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
+    "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
+    "dequantize_mx", "gemm_ref_mx", "QuantizedMX",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -60,6 +62,14 @@ def lib() -> C.CDLL:
             "nvo_quantize_2d": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int, C.c_int,
                                           C.POINTER(C.c_float)]),
             "nvo_philox4x32_10": (None, [_p, _p, _p]),
+            "nvo_ue8m0_decode": (C.c_double, [C.c_uint8]),
+            "nvo_mx_scales_bytes": (_i64, [_i64, _i64, C.c_int]),
+            "nvo_mx_sf_offset": (_i64, [_i64, _i64, _i64, C.c_int]),
+            "nvo_mx_exponent": (C.c_int, [C.c_float]),
+            "nvo_quantize_mx": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int]),
+            "nvo_dequantize_mx": (None, [_p, _p, C.c_int, _i64, _i64, _p, _i64]),
+            "nvo_gemm_ref_mx": (None, [_p, _p, C.c_int, _i64, _p, _p, C.c_int, _i64, _i64, _p, _p,
+                                       _i64, _p, _p]),
             "nvo_e2m1_sr": (C.c_uint8, [C.c_float, C.c_uint32]),
             "nvo_sr_block_draws": (None, [C.c_uint64, _i64, _i64, _i64, _p]),
             "nvo_quantize_sr": (C.c_int, [_p, _i64, _i64, _i64, C.c_int, C.c_uint32, C.c_uint64, _p,
@@ -270,6 +280,63 @@ def quantize_sr(x, seed: int, layout: int = SF_SWIZZLED, sign_mask=None, g=None)
                                sign_mask or 0, seed, _ptr(codes), _ptr(scales), layout,
                                0 if g is None else 1, C.byref(gv))
     return st, Quantized(codes, scales, gv.value, rows, cols, layout)
+
+
+def ue8m0_decode(b: int) -> float:
+    return float(lib().nvo_ue8m0_decode(b))
+
+
+def mx_scales_bytes(rows: int, cols: int, layout: int) -> int:
+    return int(lib().nvo_mx_scales_bytes(rows, cols, layout))
+
+
+def mx_sf_offset(r: int, c: int, cols: int, layout: int) -> int:
+    return int(lib().nvo_mx_sf_offset(r, c, cols, layout))
+
+
+def mx_exponent(amax: float) -> int:
+    return int(lib().nvo_mx_exponent(float(np.float32(amax))))
+
+
+class QuantizedMX:
+    """Oracle MXFP4 tensor: codes [rows, cols/2] u8, UE8M0 scales (flat u8)."""
+
+    def __init__(self, codes, scales, rows, cols, layout):
+        self.codes, self.scales = codes, scales
+        self.rows, self.cols, self.layout = rows, cols, layout
+
+    def dequantize(self) -> np.ndarray:
+        return dequantize_mx(self.codes, self.scales, self.layout, self.rows, self.cols)
+
+
+def quantize_mx(x, layout: int = SF_SWIZZLED) -> tuple[int, QuantizedMX]:
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(mx_scales_bytes(rows, cols, layout), np.uint8)
+    st = lib().nvo_quantize_mx(_ptr(b), rows, cols, cols, _ptr(codes), _ptr(scales), layout)
+    return st, QuantizedMX(codes, scales, rows, cols, layout)
+
+
+def dequantize_mx(codes, scales, layout, rows, cols) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    y = np.zeros((rows, cols), np.uint16)
+    lib().nvo_dequantize_mx(_ptr(codes), _ptr(scales), layout, rows, cols, _ptr(y), cols)
+    return y
+
+
+def gemm_ref_mx(a: QuantizedMX, w: QuantizedMX, i_idx, j_idx):
+    assert a.cols == w.cols
+    i_idx = np.ascontiguousarray(i_idx, np.int64)
+    j_idx = np.ascontiguousarray(j_idx, np.int64)
+    n = len(i_idx)
+    ref = np.zeros(n, np.float64)
+    ab = np.zeros(n, np.float64)
+    lib().nvo_gemm_ref_mx(_ptr(a.codes), _ptr(a.scales), a.layout, a.rows, _ptr(w.codes),
+                          _ptr(w.scales), w.layout, w.rows, a.cols, _ptr(i_idx), _ptr(j_idx), n,
+                          _ptr(ref), _ptr(ab))
+    return ref, ab
 
 
 if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):
