@@ -237,6 +237,35 @@ NVFP4_API nvfp4_status nvfp4_quantize_sr(const void *x, int64_t ld, int32_t tran
                                          int32_t global_supplied, void *workspace,
                                          size_t workspace_bytes, void *stream);
 
+/* ---- MXFP4 ------------------------------------------------------------ */
+/* MXFP4, the format the pages compare NVFP4 with ("NVIDIA shrank GLM-5.2 to
+ * 4 bits", section 3: blocks of 32 with a power-of-two E8M0 scale; "NVFP4:
+ * how NVIDIA pre-trained a 12B model on 10T tokens", section "E2M1 format
+ * and two-level scaling": 32 values per UE8M0 scale; "FP4 KV-cache
+ * quantization", section "FP4 formats compared": about 4.25 bits/value).
+ * An nvfp4_tensor holds an MXFP4 tensor with: the same E2M1 codes and
+ * nibble order; one UE8M0 byte per 32 values (2^(byte - 127)) at the
+ * positions of the same two layouts over cols / 32 scale columns
+ * (nvfp4_mx_scales_bytes); `global` unused (may be NULL); cols % 32 == 0.
+ * Quantize: per block X = floor(log2(amax)) - 2 clamped to [-127, 127] (the
+ * OCP microscaling shared-exponent rule; -127 for a block of zeros or
+ * subnormals), byte X + 127, codes e2m1_rne_satfinite(x * 2^-X).
+ * Dequantize: bf16(e2m1(code) * 2^X).  Non-finite input is recorded as
+ * NVFP4_ERR_NONFINITE in the workspace status word (outputs unspecified). */
+NVFP4_API size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout);
+NVFP4_API nvfp4_status nvfp4_quantize_mx(const void *x, int64_t ld, const nvfp4_tensor *out,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+NVFP4_API nvfp4_status nvfp4_dequantize_mx(const nvfp4_tensor *in, void *y, int64_t ld,
+                                           void *stream);
+
+/* MXFP4 W4A4 linear: D = A_hat * W_hat^T with A, W MXFP4 tensors (block 32,
+ * UE8M0 scales, swizzled layout, no tensor scales: alpha = 1), on the same
+ * block-scaled tensor-core MMA as nvfp4_gemm with scale vector 2X.  Shapes,
+ * output and errors as nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D,
+                                     int64_t ldd, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
 /* Same quantization as nvfp4_quantize, for callers that cannot allocate
  * device memory when they quantize: code recorded into a CUDA graph (device
  * allocation cannot be captured), latency-critical paths that cannot afford

@@ -35,7 +35,8 @@ EXPORTED = (
     "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
-    "nvfp4_quantize_sr",
+    "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
+    "nvfp4_gemm_mx",
 )
 
 
@@ -86,6 +87,10 @@ def lib() -> C.CDLL:
             "nvfp4_quantize_2d": (C.c_int, [vp, i64, T, T, i32, vp, sz, vp]),
             "nvfp4_quantize_sr": (C.c_int, [vp, i64, i32, i32, C.c_uint32, C.c_uint64, T, i32, vp,
                                             sz, vp]),
+            "nvfp4_mx_scales_bytes": (sz, [i64, i64, i32]),
+            "nvfp4_quantize_mx": (C.c_int, [vp, i64, T, vp, sz, vp]),
+            "nvfp4_dequantize_mx": (C.c_int, [T, vp, i64, vp]),
+            "nvfp4_gemm_mx": (C.c_int, [T, T, vp, i64, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -152,6 +157,18 @@ class NVFP4Tensor:
 
     def nbytes(self) -> int:
         return self.codes.numel() + self.scales.numel()
+
+
+class MXFP4Tensor(NVFP4Tensor):
+    """Device MXFP4 tensor: packed codes and UE8M0 scales (one per 32
+    values); no tensor scale."""
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, layout: int = SF_SWIZZLED, device="cuda"):
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(lib().nvfp4_mx_scales_bytes(rows, cols, layout), dtype=torch.uint8,
+                             device=device)
+        return cls(codes, scales, None, rows, cols, layout)
 
 
 class Workspace:
@@ -274,6 +291,41 @@ def nvfp4_quantize_sr(x: torch.Tensor, seed: int, out: NVFP4Tensor | None = None
                                    0 if sign_mask is None else 1, sign_mask or 0, seed, C.byref(t),
                                    int(global_supplied), ws.ptr, ws.nbytes, _stream(stream)),
            "nvfp4_quantize_sr")
+    return out
+
+
+def nvfp4_quantize_mx(x: torch.Tensor, out: MXFP4Tensor | None = None, layout: int = SF_SWIZZLED,
+                      workspace: Workspace | None = None, stream=None) -> MXFP4Tensor:
+    """MXFP4 quantization (block 32, UE8M0 scales) of a 2-D BF16 tensor."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out is None:
+        out = MXFP4Tensor.empty(rows, cols, layout, x.device)
+    ws = workspace or default_workspace(x.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize_mx(x.data_ptr(), x.stride(0), C.byref(t), ws.ptr, ws.nbytes,
+                                   _stream(stream)), "nvfp4_quantize_mx")
+    return out
+
+
+def nvfp4_dequantize_mx(t: MXFP4Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((t.rows, t.cols), dtype=torch.bfloat16, device=t.codes.device)
+    ct = t.c_struct()
+    _check(lib().nvfp4_dequantize_mx(C.byref(ct), out.data_ptr(), out.stride(0), _stream(stream)),
+           "nvfp4_dequantize_mx")
+    return out
+
+
+def nvfp4_gemm_mx(a: MXFP4Tensor, w: MXFP4Tensor, out: torch.Tensor | None = None,
+                  workspace: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D = A_hat * W_hat^T for MXFP4 operands (BF16 out)."""
+    if out is None:
+        out = torch.empty((a.rows, w.rows), dtype=torch.bfloat16, device=a.codes.device)
+    ws = workspace or default_workspace(a.codes.device)
+    ta, tw = a.c_struct(), w.c_struct()
+    _check(lib().nvfp4_gemm_mx(C.byref(ta), C.byref(tw), out.data_ptr(), out.stride(0), ws.ptr,
+                               ws.nbytes, _stream(stream)), "nvfp4_gemm_mx")
     return out
 
 

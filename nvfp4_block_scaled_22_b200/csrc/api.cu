@@ -78,6 +78,18 @@ nvfp4_status check_tensor(const nvfp4_tensor *t) {
     return NVFP4_OK;
 }
 
+nvfp4_status check_mx_tensor(const nvfp4_tensor *t) {
+    if (t == nullptr || t->rows < 0 || t->cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (t->sf_layout != NVFP4_SF_SWIZZLED_128x4 && t->sf_layout != NVFP4_SF_LINEAR)
+        return NVFP4_ERR_INVALID_ARG;
+    if (t->cols % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (t->rows > 0 && t->cols > 0) {
+        if (t->codes == nullptr || t->scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(t->codes) || !aligned16(t->scales)) return NVFP4_ERR_ALIGNMENT;
+    }
+    return NVFP4_OK;
+}
+
 nvfp4_status check_workspace(void *ws, size_t bytes, size_t need) {
     if (ws == nullptr || bytes < need) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(ws)) return NVFP4_ERR_ALIGNMENT;
@@ -443,6 +455,82 @@ nvfp4_status nvfp4_quantize_2d(const void *w, int64_t ld, const nvfp4_tensor *ou
     return launched(launch_transpose_kernel((const void *)k_encode_t_2d, grid_t, args, s));
 }
 
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout) {
+    if (rows < 0 || cols < 0) return 0;
+    const int64_t s = cols / 32;
+    if (sf_layout == NVFP4_SF_LINEAR) return (size_t)(rows * s);
+    return (size_t)(ceil_div(rows, 128) * 128 * ceil_div(s, 4) * 4);
+}
+
+
+nvfp4_status nvfp4_quantize_mx(const void *x, int64_t ld, const nvfp4_tensor *out, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    nvfp4_status st = check_mx_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (out->rows > 0 && out->cols > 0) {
+        if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < out->cols) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(out->rows, 128) * 128
+                                                                         : out->rows;
+    const int64_t tasks = rows_out * ceil_div(ceil_div(out->cols / 32, 4) * 4, 32);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    EncodeParams p;
+    p.x = static_cast<const uint16_t *>(x);
+    p.ld = ld;
+    p.rows = out->rows;
+    p.cols = out->cols;
+    p.gather = nullptr;
+    p.src_rows = 0;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = nullptr;
+    p.global_supplied = 1;
+    p.partials = nullptr;
+    p.n_partials = 0;
+    p.status = reinterpret_cast<uint32_t *>(workspace);
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    if (grid < 1) grid = 1;
+    k_encode_mx<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_dequantize_mx(const nvfp4_tensor *in, void *y, int64_t ld, void *stream) {
+    nvfp4_status st = check_mx_tensor(in);
+    if (st != NVFP4_OK) return st;
+    if (in->rows > 0 && in->cols > 0) {
+        if (y == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(y) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < in->cols) return NVFP4_ERR_SHAPE;
+    }
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    if (in->rows == 0 || in->cols == 0) return NVFP4_OK;
+    DequantParams p;
+    p.codes = static_cast<const uint8_t *>(in->codes);
+    p.scales = static_cast<const uint8_t *>(in->scales);
+    p.layout = in->sf_layout;
+    p.global = nullptr;
+    p.rows = in->rows;
+    p.cols = in->cols;
+    p.y = static_cast<uint16_t *>(y);
+    p.ld = ld;
+    const int64_t tasks = in->rows * ceil_div(in->cols / 32, 32);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
+    int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
+    if (grid < 1) grid = 1;
+    k_dequantize_mx<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                                    const int32_t *d_gather, const nvfp4_tensor *out,
                                    int32_t global_supplied, void *workspace,
@@ -528,14 +616,15 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     return launched(cudaGetLastError());
 }
 
+
 static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
                                 const int32_t *d_group_rows, const nvfp4_tensor *A,
                                 const nvfp4_tensor *W, const float *gw, int64_t n, void *D,
                                 int64_t ldd, void *workspace, size_t workspace_bytes,
-                                void *stream) {
-    nvfp4_status st = check_tensor(A);
+                                void *stream, bool mx = false) {
+    nvfp4_status st = mx ? check_mx_tensor(A) : check_tensor(A);
     if (st != NVFP4_OK) return st;
-    st = check_tensor(W);
+    st = mx ? check_mx_tensor(W) : check_tensor(W);
     if (st != NVFP4_OK) return st;
     if (A->sf_layout != NVFP4_SF_SWIZZLED_128x4 || W->sf_layout != NVFP4_SF_SWIZZLED_128x4)
         return NVFP4_ERR_INVALID_ARG;
@@ -562,7 +651,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     if (st != NVFP4_OK) return st;
     st = get_encode();
     if (st != NVFP4_OK) return st;
-    const bool pair = groups == 0 && m >= kPairMinRows && sms >= 2 && g_use_pairs;
+    const bool pair = !mx && groups == 0 && m >= kPairMinRows && sms >= 2 && g_use_pairs;
     CUtensorMap tmA, tmB;
     st = encode_codes_map(&tmA, A->codes, A->rows, k, kBM);
     if (st != NVFP4_OK) return st;
@@ -595,7 +684,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     }
     const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, kBN);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, sms));
-    return launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream)));
+    return launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream), mx));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,
@@ -603,6 +692,13 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, i
     if (W == nullptr) return NVFP4_ERR_INVALID_ARG;
     return gemm_common(0, nullptr, nullptr, A, W, W->global, W->rows, D, ldd, workspace,
                        workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    if (W == nullptr) return NVFP4_ERR_INVALID_ARG;
+    return gemm_common(0, nullptr, nullptr, A, W, nullptr, W->rows, D, ldd, workspace,
+                       workspace_bytes, stream, true);
 }
 
 nvfp4_status nvfp4_grouped_gemm(int32_t groups, const int32_t *d_slot_offsets,

@@ -55,6 +55,8 @@ constexpr int kFirstEpiWarp = 2 + kSfWarps;
 // K-major, N = 256 (>> 3), UE4M3 scales (bit 23 = 0), M = 128 (>> 4).
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
+// The same for MXFP4 operands: UE8M0 scales (bit 23 = 1), scale vector 2X.
+constexpr uint32_t kIdescMx = kIdesc | (1u << 23);
 constexpr long long kDrainCycles = 2000000000ll;
 
 struct Shared {
@@ -123,9 +125,13 @@ __device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, int ntiles,
 
 }  // namespace
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const GemmParams p) {
+// kMx: MXFP4 operands (one UE8M0 scale per 32 values, 512-byte 128x4 tiles
+// covering 128 K values; no tensor scales, alpha = 1).  The MMA reads two
+// scale bytes per row and K=64 step; the scale writers put them in bytes
+// 0-1 of the same TMEM words the NVFP4 path fills with four.
+template <bool kMx>
+__device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                          const GemmParams &p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,7 +189,9 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int tiles = mtiles * ntiles;
     const int kblocks = p.k / 64;                    // 64-value MMA steps
     const int ktiles = (kblocks + 3) / 4;            // 256-value stages
-    const int64_t sf_rowblock_bytes = (int64_t)kblocks * 512;   // one 128-row band
+    // one 128-row band of scale tiles; a tile covers 64 (NVFP4) or 128 (MX) K
+    const int64_t sf_rowblock_bytes = (int64_t)(kMx ? (kblocks + 1) / 2 : kblocks) * 512;
+    constexpr int64_t kSfStageStride = kMx ? 1024 : 2048;      // scale bytes per band and stage
     const int my_tiles =
         (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total_k = my_tiles * ktiles;           // stages this CTA runs, in order
@@ -205,7 +213,7 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_or_abort(&sh->empty[stage], phase ^ 1, sh, p)) { ok = false; break; }
                     const int nkb = min(4, kblocks - 4 * kt);
-                    const uint32_t sf_bytes = (uint32_t)nkb * 512;
+                    const uint32_t sf_bytes = (uint32_t)(kMx ? (nkb + 1) / 2 : nkb) * 512;
                     uint8_t *sA = smem + stage * kStageBytes;
                     uint8_t *sB = sA + kStageA;
                     uint8_t *sSFA = sB + kStageB;
@@ -214,11 +222,12 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     mbar_arrive_expect_tx(&sh->sf_landed[stage], sf_bytes * (1 + halves));
                     armed[stage] = true;
                     armed_phase[stage] = phase;
-                    bulk_load(sSFA, p.sfa + sfa_base + (int64_t)kt * 2048, sf_bytes,
+                    bulk_load(sSFA, p.sfa + sfa_base + (int64_t)kt * kSfStageStride, sf_bytes,
                               &sh->sf_landed[stage]);
                     for (int h = 0; h < halves; ++h)
                         bulk_load(sSFB + h * 2048,
-                                  p.sfb + (int64_t)(brb + h) * sf_rowblock_bytes + (int64_t)kt * 2048,
+                                  p.sfb + (int64_t)(brb + h) * sf_rowblock_bytes +
+                                      (int64_t)kt * kSfStageStride,
                                   sf_bytes, &sh->sf_landed[stage]);
                     tma_load_2d(sA, &tmA, &sh->tma_ready[stage], kt * (kBK / 2), t.a_row0);
                     tma_load_2d(sB, &tmB, &sh->tma_ready[stage], kt * (kBK / 2), t.b_row0);
@@ -256,11 +265,19 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const uint8_t *sSFA = smem + stage * kStageBytes + kStageA + kStageB;
             const uint8_t *sSFB = sSFA + kStageSFA;
             const uint32_t col = lane_base + kAccCols + (uint32_t)stage * kSfCols;
+            // NVFP4: word q of tile kb is the four scales of row 32q+i for K
+            // block kb.  MX: tile kb/2 covers K blocks 2t, 2t+1 with two
+            // scales each (bytes 0-1 and 2-3 of the word).
+            auto pick = [](uint32_t w, int kb) -> uint32_t {
+                return kMx ? (w >> (16 * (kb & 1))) & 0xFFFFu : w;
+            };
             uint32_t v[16];
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(sSFA + 512 * kb + 16 * lane);
-                v[4 * kb] = w.x; v[4 * kb + 1] = w.y; v[4 * kb + 2] = w.z; v[4 * kb + 3] = w.w;
+                const int tile = kMx ? kb / 2 : kb;
+                const uint4 w = *reinterpret_cast<const uint4 *>(sSFA + 512 * tile + 16 * lane);
+                v[4 * kb] = pick(w.x, kb); v[4 * kb + 1] = pick(w.y, kb);
+                v[4 * kb + 2] = pick(w.z, kb); v[4 * kb + 3] = pick(w.w, kb);
             }
             tmem_st_32x32b_x16(col, v);
             uint32_t u[32];
@@ -268,9 +285,11 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(sSFB + 2048 * h + 512 * kb + 16 * lane);
+                    const int tile = kMx ? kb / 2 : kb;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(sSFB + 2048 * h + 512 * tile + 16 * lane);
                     const int o = 8 * kb + 4 * h;
-                    u[o] = w.x; u[o + 1] = w.y; u[o + 2] = w.z; u[o + 3] = w.w;
+                    u[o] = pick(w.x, kb); u[o + 1] = pick(w.y, kb);
+                    u[o + 2] = pick(w.z, kb); u[o + 3] = pick(w.w, kb);
                 }
             }
             tmem_st_32x32b_x32(col + 16, u);
@@ -312,15 +331,21 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     tc_fence_after();
                 }
                 const uint32_t first = kt != 0 ? 1u : 0u;
+                auto mma = [&](int kb, uint32_t acc) {
+                    if (kMx)
+                        mma_mxf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
+                                 kIdescMx, sfa + 4 * kb, sfa + 16 + 8 * kb, acc);
+                    else
+                        mma_nvf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
+                                 kIdesc, sfa + 4 * kb, sfa + 16 + 8 * kb, acc);
+                };
                 if (kt != ktiles - 1 || last_nkb == 4) {
-                    mma_nvf4(tmem, adesc0 + stage_off, bdesc0 + stage_off, kIdesc, sfa, sfa + 16, first);
-                    mma_nvf4(tmem, adesc0 + stage_off + 2, bdesc0 + stage_off + 2, kIdesc, sfa + 4, sfa + 24, 1u);
-                    mma_nvf4(tmem, adesc0 + stage_off + 4, bdesc0 + stage_off + 4, kIdesc, sfa + 8, sfa + 32, 1u);
-                    mma_nvf4(tmem, adesc0 + stage_off + 6, bdesc0 + stage_off + 6, kIdesc, sfa + 12, sfa + 40, 1u);
+                    mma(0, first);
+                    mma(1, 1u);
+                    mma(2, 1u);
+                    mma(3, 1u);
                 } else {
-                    for (int kb = 0; kb < last_nkb; ++kb)
-                        mma_nvf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb, kIdesc,
-                                 sfa + 4 * kb, sfa + 16 + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
+                    for (int kb = 0; kb < last_nkb; ++kb) mma(kb, (kt | kb) != 0 ? 1u : 0u);
                 }
                 tc_commit(&sh->empty[stage]);
                 if (kt == ktiles - 1) {
@@ -355,7 +380,8 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             // coordinates are derived again for the stores (fewer live
             // registers next to the 64 output words).
             const float alpha =
-                __frcp_rn(__fmul_rn(*p.ga, p.gw[tile_info(tile, mtiles, ntiles, p, s_off, s_rows).group]));
+                kMx ? 1.0f
+                    : __frcp_rn(__fmul_rn(*p.ga, p.gw[tile_info(tile, mtiles, ntiles, p, s_off, s_rows).group]));
             if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
             uint32_t o[64];
@@ -394,19 +420,34 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
 }
 
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+    gemm_body<false>(tmA, tmB, p);
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm_mxf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+    gemm_body<true>(tmA, tmB, p);
+}
+
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                        int grid, cudaStream_t stream) {
-    static bool attr_set[64] = {};
+                        int grid, cudaStream_t stream, bool mx) {
+    static bool attr_set[64][2] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmSmemBytes);
+    if (dev < 0 || dev >= 64 || !attr_set[dev][mx ? 1 : 0]) {
+        e = cudaFuncSetAttribute(mx ? k_gemm_mxf4 : k_gemm_nvf4,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        if (dev >= 0 && dev < 64) attr_set[dev][mx ? 1 : 0] = true;
     }
-    k_gemm_nvf4<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    if (mx)
+        k_gemm_mxf4<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    else
+        k_gemm_nvf4<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
     return cudaGetLastError();
 }
 

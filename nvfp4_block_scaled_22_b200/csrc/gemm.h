@@ -48,8 +48,9 @@ struct GemmParams {
     long long timeout_cycles;
 };
 
+// mx: MXFP4 operands (UE8M0 scales per 32 values, no tensor scales).
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                        int grid, cudaStream_t stream);
+                        int grid, cudaStream_t stream, bool mx = false);
 
 // Dense GEMM on CTA pairs (256x256 tiles); tmB must use 128-row boxes.
 cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,

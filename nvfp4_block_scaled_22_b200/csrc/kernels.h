@@ -96,6 +96,10 @@ inline int64_t transpose_tasks(int64_t x_rows, int64_t out_rows_padded) {
     return ((x_rows + 63) / 64) * ((out_rows_padded + 63) / 64);
 }
 
+// MXFP4 (block 32, UE8M0 scales, no tensor scale); 256 threads.
+__global__ void k_encode_mx(EncodeParams p);
+__global__ void k_dequantize_mx(DequantParams p);
+
 __global__ void k_dequantize(DequantParams p);
 __global__ void k_dequantize_narrow(DequantParams p);
 
