@@ -44,8 +44,8 @@ FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
 # the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
 # Reported only while the kernel's sources hash to the profiled version.
-GEMM_TRAFFIC_BYTES = 87.05e6 + 292.46e6
-GEMM_TRAFFIC_SRC_SHA = "6159f8c67b83198d"
+GEMM_TRAFFIC_BYTES = 88.24e6 + 292.66e6
+GEMM_TRAFFIC_SRC_SHA = "ece00d8fd2be476e"
 GEMM_SOURCES = ("gemm.cu", "gemm.h", "ptx.cuh")
 
 
@@ -619,6 +619,42 @@ def workload_line(name, args, device):
                                   "quantize_share": q_ms / ms,
                                   "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g}"}})
         return line
+    if name == "mxfp4":
+        # The format the pages compare NVFP4 with: block 32, power-of-two
+        # scales, no tensor scale -- quantize (one pass) and the W4A4 GEMM at
+        # the headline FFN shape, plus the 2^28-value sweep tensor.
+        m = 8192
+        w = inputs.ffn_weight(device=device)
+        qw = nb.nvfp4_quantize_mx(w, workspace=ws)
+        del w
+        a = inputs.ffn_activation(m, device=device)
+        qa = nb.MXFP4Tensor.empty(m, K, device=device)
+        d = torch.empty((m, N), dtype=torch.bfloat16, device=device)
+        qms = _timed(lambda: nb.nvfp4_quantize_mx(a, out=qa, workspace=ws), args.steps, args.warmup, flush)
+        gms = _timed(lambda: nb.nvfp4_gemm_mx(qa, qw, out=d, workspace=ws), args.steps, args.warmup, flush)
+        xs = inputs.sweep_tensor(1 << 28, device=device)
+        qs = nb.MXFP4Tensor.empty(xs.shape[0], xs.shape[1], device=device)
+        sms = _timed(lambda: nb.nvfp4_quantize_mx(xs, out=qs, workspace=ws), args.steps, args.warmup)
+        dms = _timed(lambda: nb.nvfp4_dequantize_mx(qs, out=xs), args.steps, args.warmup)
+        st = nb.nvfp4_check_status(ws)
+        flops = 2.0 * m * N * K
+        mx_bpv = 2.0 + 0.5 + 1.0 / 32
+        sgbs = (1 << 28) * mx_bpv / sms / 1e6
+        line.update({"metric": "MXFP4 W4A4 linear M=8192 TFLOP/s (quantize A + GEMM)",
+                     "value": flops / (qms + gms) / 1e9, "unit": "TFLOP/s", "higher_is_better": True,
+                     "ms_per_step": qms + gms,
+                     "config": {"workload": f"mxfp4 ffn linear M={m} N={N} K={K}; quantize sweep 2^28",
+                                "l2": "flushed (GEMM); sweep tensors exceed L2"},
+                     "gemm_ms": gms, "quantize_ms": qms, "gemm_tflops": flops / gms / 1e9,
+                     "quantize_2p28_ms": sms, "quantize_2p28_gbs": sgbs,
+                     "dequantize_2p28_gbs": (1 << 28) * (0.5 + 1.0 / 32 + 2.0) / dms / 1e6,
+                     "bytes_per_value_quantize": mx_bpv, "status": st,
+                     "roofline": {"kernel": "k_gemm_mxf4", "bound": "tensor", "achieved": flops / gms / 1e9,
+                                  "peak": fp4_peak, "unit": "TFLOP/s",
+                                  "frac": flops / gms / 1e9 / fp4_peak,
+                                  "quantize_frac_of_hbm": sgbs / hbm_gbs,
+                                  "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g}"}})
+        return line
     raise ValueError(name)
 
 
@@ -636,7 +672,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--workload", default="ffn8192",
-                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train"],
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")
