@@ -188,6 +188,15 @@ class MoeRouting:
             self.gather[o:o + (b - a)] = src_tokens[a:b].to(torch.int32)
         self.padded_rows = total
         self.real_rows = int(self.rows.sum())
+        # row of (token t, choice k) in the padded expert-major layout
+        slot_of_pair = torch.empty(tokens * topk, dtype=torch.int64)
+        flat_e_sorted = flat_e[perm]
+        pos = torch.arange(tokens * topk) - starts[flat_e_sorted]
+        slot_of_pair[perm] = self.slot_offsets.long()[flat_e_sorted] + pos
+        self.token_slots = slot_of_pair.view(tokens, topk).to(torch.int32)
+        # combine weights: the selected probabilities, renormalized to sum 1
+        w = self.topk_weights.double()
+        self.combine_weights = (w / w.sum(dim=1, keepdim=True)).float()
 
 
 def moe_activation(device="cpu", tokens=MOE_TOKENS, hidden=MOE_HIDDEN) -> torch.Tensor:

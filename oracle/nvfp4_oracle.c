@@ -33,6 +33,11 @@
  *       scale), pre-training page section "E2M1 format and two-level
  *       scaling" (32 values per UE8M0 scale, no tensor scale), KV page
  *       section "FP4 formats compared" (about 4.25 bits per value).
+ *  [PC] consumers of the quantized tensors: "NVIDIA shrank GLM-5.2 to 4
+ *       bits" section 2 (256 experts, 8 active per token: the expert
+ *       outputs are combined per token); "FP4 KV-cache quantization",
+ *       section on current implementations (the FP4 KV cache is
+ *       dequantized to FP8 before attention).
  *  [PX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *       1, 2, 3" (SC 2011): the Philox4x32-10 counter-based generator.
  *  The FP32 evaluation order below is the convention the hot path is
@@ -789,4 +794,48 @@ void nvo_gemm_ref_mx(const uint8_t *a_codes, const uint8_t *a_scales, int a_layo
         ref[t] = acc;
         abs_out[t] = aacc;
     }
+}
+
+/* ------------------------------------------------------------ consumers */
+
+/* [PC] MoE combine: y[t] = bf16(sum_k w[t][k] * out[slot[t][k]]) over the
+ * token's topk expert rows.  READINGS: the weights are the caller's
+ * (routing) combine weights; FP32 accumulation in k order, each step one
+ * fused multiply-add (acc = fma(w, x, acc), starting from 0); a slot of -1
+ * contributes nothing; one BF16 rounding at the end. */
+void nvo_moe_combine(const uint16_t *out, int64_t ld, const int32_t *slots, const float *w,
+                     int64_t tokens, int64_t topk, int64_t hidden, uint16_t *y, int64_t ldy)
+{
+    for (int64_t t = 0; t < tokens; ++t)
+        for (int64_t c = 0; c < hidden; ++c) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < topk; ++k) {
+                int32_t s = slots[t * topk + k];
+                if (s < 0)
+                    continue;
+                acc = fmaf(w[t * topk + k], nvo_bf16_to_f32(out[(int64_t)s * ld + c]), acc);
+            }
+            y[t * ldy + c] = nvo_f32_to_bf16(acc);
+        }
+}
+
+/* [PC] NVFP4 -> FP8 (E4M3) for an attention read.  READING (the page says
+ * only that the FP4 cache is dequantized to FP8): each value becomes
+ * e4m3_rne_satfinite(e2m1(code) * s_b / 8), with one per-tensor dequant
+ * factor RN(8 / g) returned in *fp8_scale, so x_hat ~= fp8 * fp8_scale.
+ * e2m1 * s_b / 8 is exact in FP32 (the 1/8 keeps 6 * 448 = 2688 inside the
+ * E4M3 range); the E4M3 rounding is the only one.  Sign kept. */
+void nvo_dequantize_fp8(const uint8_t *codes, const uint8_t *scales, int layout, float g,
+                        int64_t rows, int64_t cols, uint8_t *y, int64_t ld, float *fp8_scale)
+{
+    *fp8_scale = 8.0f / g;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = codes[r * (cols / 2) + c / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+            float sb = nvo_e4m3_decode(scales[nvo_sf_offset(r, c / 16, rows, cols, layout)]);
+            float v = nvo_e2m1_decode(code) * sb / 8.0f;
+            uint8_t e = nvo_e4m3_rne_satfinite(fabsf(v));
+            y[r * ld + c] = (uint8_t)(e | (signbit(v) ? 0x80 : 0));
+        }
 }

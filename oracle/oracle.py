@@ -20,7 +20,7 @@ __all__ = [
     "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
     "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
-    "dequantize_mx", "gemm_ref_mx", "QuantizedMX",
+    "dequantize_mx", "gemm_ref_mx", "QuantizedMX", "moe_combine", "dequantize_fp8",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -63,6 +63,9 @@ def lib() -> C.CDLL:
                                           C.POINTER(C.c_float)]),
             "nvo_philox4x32_10": (None, [_p, _p, _p]),
             "nvo_ue8m0_decode": (C.c_double, [C.c_uint8]),
+            "nvo_moe_combine": (None, [_p, _i64, _p, _p, _i64, _i64, _i64, _p, _i64]),
+            "nvo_dequantize_fp8": (None, [_p, _p, C.c_int, C.c_float, _i64, _i64, _p, _i64,
+                                          C.POINTER(C.c_float)]),
             "nvo_mx_scales_bytes": (_i64, [_i64, _i64, C.c_int]),
             "nvo_mx_sf_offset": (_i64, [_i64, _i64, _i64, C.c_int]),
             "nvo_mx_exponent": (C.c_int, [C.c_float]),
@@ -337,6 +340,27 @@ def gemm_ref_mx(a: QuantizedMX, w: QuantizedMX, i_idx, j_idx):
                           _ptr(w.scales), w.layout, w.rows, a.cols, _ptr(i_idx), _ptr(j_idx), n,
                           _ptr(ref), _ptr(ab))
     return ref, ab
+
+
+def moe_combine(out, slots, weights) -> np.ndarray:
+    """y[t] = bf16(sum_k w[t,k] * out[slots[t,k]]) (FMA chain in k order)."""
+    o = bf16_bits(out)
+    sl = np.ascontiguousarray(np.asarray(slots), np.int32)
+    w = np.ascontiguousarray(np.asarray(weights), np.float32)
+    tokens, topk = sl.shape
+    hidden = o.shape[1]
+    y = np.zeros((tokens, hidden), np.uint16)
+    lib().nvo_moe_combine(_ptr(o), hidden, _ptr(sl), _ptr(w), tokens, topk, hidden, _ptr(y), hidden)
+    return y
+
+
+def dequantize_fp8(q: Quantized) -> tuple[np.ndarray, float]:
+    """NVFP4 -> E4M3 bytes and the per-tensor dequant factor RN(8 / g)."""
+    y = np.zeros((q.rows, q.cols), np.uint8)
+    sc = C.c_float()
+    lib().nvo_dequantize_fp8(_ptr(np.ascontiguousarray(q.codes)), _ptr(np.ascontiguousarray(q.scales)),
+                             q.layout, float(q.g), q.rows, q.cols, _ptr(y), q.cols, C.byref(sc))
+    return y, float(sc.value)
 
 
 if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):
