@@ -655,6 +655,35 @@ def workload_line(name, args, device):
                                   "quantize_frac_of_hbm": sgbs / hbm_gbs,
                                   "peak_source": f"{peak_src} bf16 x {FP4_OVER_BF16:g}"}})
         return line
+    if name == "consumers":
+        # The steps after the path: MoE per-token combine of the expert
+        # outputs (4096 tokens x top-8 x 6144) and NVFP4 -> FP8 of one KV
+        # tensor (131072 x 1024).
+        r = inputs.MoeRouting()
+        g = torch.Generator(device=device).manual_seed(inputs.seed_for("moe", 9100))
+        out = torch.randn((r.padded_rows, inputs.MOE_HIDDEN), generator=g, device=device).to(torch.bfloat16)
+        slots, w = r.token_slots.to(device), r.combine_weights.to(device)
+        y = torch.empty((r.tokens, inputs.MOE_HIDDEN), dtype=torch.bfloat16, device=device)
+        cms = _timed(lambda: nb.nvfp4_moe_combine(out, slots, w, out=y), args.steps, args.warmup, flush)
+        cbytes = r.tokens * inputs.MOE_HIDDEN * 2 * (r.topk + 1)
+        x = inputs.kv_tensor(0, 0, device=device).view(inputs.KV_TOKENS, -1).contiguous()
+        q = nb.nvfp4_quantize(x, layout=nb.SF_LINEAR, workspace=ws)
+        f8 = torch.empty(x.shape, dtype=torch.uint8, device=device)
+        sc = torch.zeros(1, dtype=torch.float32, device=device)
+        fms = _timed(lambda: nb.nvfp4_dequantize_fp8(q, out=f8, scale=sc), args.steps, args.warmup, flush)
+        fbytes = x.numel() * (0.5625 + 1.0)
+        st = nb.nvfp4_check_status(ws)
+        cgbs = cbytes / cms / 1e6
+        line.update({"metric": "MoE top-8 combine GB/s (4096 tokens x 6144)", "value": cgbs, "unit": "GB/s",
+                     "higher_is_better": True, "ms_per_step": cms,
+                     "config": {"workload": "consumers: moe combine 4096 x top-8 x 6144; kv nvfp4->fp8 "
+                                            "131072 x 1024", "l2": "flushed"},
+                     "combine_ms": cms, "fp8_ms": fms, "fp8_gbs": fbytes / fms / 1e6, "status": st,
+                     "roofline": {"kernel": "k_moe_combine", "bound": "hbm", "achieved": cgbs,
+                                  "peak": hbm_gbs, "unit": "GB/s", "frac": cgbs / hbm_gbs,
+                                  "fp8_frac": fbytes / fms / 1e6 / hbm_gbs,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
+        return line
     raise ValueError(name)
 
 
@@ -672,7 +701,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--workload", default="ffn8192",
-                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4"],
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4", "consumers"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")

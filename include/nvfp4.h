@@ -237,6 +237,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_sr(const void *x, int64_t ld, int32_t tran
                                          int32_t global_supplied, void *workspace,
                                          size_t workspace_bytes, void *stream);
 
+/* ---- consumers -------------------------------------------------------- */
+/* MoE combine ("NVIDIA shrank GLM-5.2 to 4 bits", section 2: 8 of 256
+ * experts per token): y[t] = bf16(sum_k w[t][k] * out[slot[t][k]]), an FP32
+ * fused multiply-add chain in k order starting from 0; slot -1 contributes
+ * nothing, and so does any slot >= out_rows.  expert_out: out_rows BF16
+ * rows (the expert outputs, e.g. the padded expert-major layout of
+ * nvfp4_grouped_gemm), pitch ld; d_slots, d_weights:
+ * [tokens x topk] int32 / float (device); y: [tokens x hidden] BF16, pitch
+ * ldy.  hidden % 8 == 0, 1 <= topk <= 32, pointers and pitches 16-byte
+ * aligned. */
+NVFP4_API nvfp4_status nvfp4_moe_combine(const void *expert_out, int64_t ld, int64_t out_rows,
+                                         const int32_t *d_slots, const float *d_weights,
+                                         int64_t tokens, int32_t topk, int64_t hidden, void *y,
+                                         int64_t ldy, void *stream);
+
+/* NVFP4 -> FP8 (E4M3) for an attention read ("FP4 KV-cache quantization":
+ * current implementations dequantize the FP4 cache to FP8 before
+ * attention): y = e4m3_rne_satfinite(e2m1(code) * s_b / 8) per value (one
+ * byte, row-major, pitch ld bytes, ld % 16 == 0) and *d_fp8_scale =
+ * RN(8 / g), so x_hat ~= e4m3(y) * (*d_fp8_scale).  Values below half the
+ * smallest E4M3 subnormal become signed zeros. */
+NVFP4_API nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int64_t ld,
+                                            float *d_fp8_scale, void *stream);
+
 /* ---- MXFP4 ------------------------------------------------------------ */
 /* MXFP4, the format the pages compare NVFP4 with ("NVIDIA shrank GLM-5.2 to
  * 4 bits", section 3: blocks of 32 with a power-of-two E8M0 scale; "NVFP4:

@@ -36,7 +36,7 @@ EXPORTED = (
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
     "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
-    "nvfp4_gemm_mx",
+    "nvfp4_gemm_mx", "nvfp4_moe_combine", "nvfp4_dequantize_fp8",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> C.CDLL:
             "nvfp4_quantize_mx": (C.c_int, [vp, i64, T, vp, sz, vp]),
             "nvfp4_dequantize_mx": (C.c_int, [T, vp, i64, vp]),
             "nvfp4_gemm_mx": (C.c_int, [T, T, vp, i64, vp, sz, vp]),
+            "nvfp4_moe_combine": (C.c_int, [vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp]),
+            "nvfp4_dequantize_fp8": (C.c_int, [T, vp, i64, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -327,6 +329,35 @@ def nvfp4_gemm_mx(a: MXFP4Tensor, w: MXFP4Tensor, out: torch.Tensor | None = Non
     _check(lib().nvfp4_gemm_mx(C.byref(ta), C.byref(tw), out.data_ptr(), out.stride(0), ws.ptr,
                                ws.nbytes, _stream(stream)), "nvfp4_gemm_mx")
     return out
+
+
+def nvfp4_moe_combine(expert_out: torch.Tensor, slots: torch.Tensor, weights: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[t] = bf16(sum_k weights[t,k] * expert_out[slots[t,k]])."""
+    assert expert_out.dtype == torch.bfloat16 and expert_out.stride(1) == 1
+    assert slots.dtype == torch.int32 and weights.dtype == torch.float32
+    tokens, topk = slots.shape
+    hidden = expert_out.shape[1]
+    if out is None:
+        out = torch.empty((tokens, hidden), dtype=torch.bfloat16, device=expert_out.device)
+    _check(lib().nvfp4_moe_combine(expert_out.data_ptr(), expert_out.stride(0), expert_out.shape[0],
+                                   slots.contiguous().data_ptr(), weights.contiguous().data_ptr(),
+                                   tokens, topk, hidden, out.data_ptr(), out.stride(0),
+                                   _stream(stream)), "nvfp4_moe_combine")
+    return out
+
+
+def nvfp4_dequantize_fp8(t: NVFP4Tensor, out: torch.Tensor | None = None, scale: torch.Tensor | None = None,
+                         stream=None):
+    """NVFP4 -> E4M3 bytes (uint8) and the per-tensor factor RN(8/g)."""
+    if out is None:
+        out = torch.empty((t.rows, t.cols), dtype=torch.uint8, device=t.codes.device)
+    if scale is None:
+        scale = torch.zeros(1, dtype=torch.float32, device=t.codes.device)
+    ct = t.c_struct()
+    _check(lib().nvfp4_dequantize_fp8(C.byref(ct), out.data_ptr(), out.stride(0), scale.data_ptr(),
+                                      _stream(stream)), "nvfp4_dequantize_fp8")
+    return out, scale
 
 
 def nvfp4_global_scale(x: torch.Tensor, out: torch.Tensor | None = None,

@@ -531,6 +531,65 @@ nvfp4_status nvfp4_dequantize_mx(const nvfp4_tensor *in, void *y, int64_t ld, vo
     return launched(cudaGetLastError());
 }
 
+nvfp4_status nvfp4_moe_combine(const void *expert_out, int64_t ld, int64_t out_rows,
+                               const int32_t *d_slots, const float *d_weights, int64_t tokens,
+                               int32_t topk, int64_t hidden, void *y, int64_t ldy, void *stream) {
+    if (tokens < 0 || hidden < 0 || out_rows < 0 || topk < 1 || topk > kMaxTopk)
+        return NVFP4_ERR_INVALID_ARG;
+    if (hidden % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (tokens == 0 || hidden == 0) return NVFP4_OK;
+    if (expert_out == nullptr || d_slots == nullptr || d_weights == nullptr || y == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(expert_out) || !aligned16(y) || ld % 8 != 0 || ldy % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (ld < hidden || ldy < hidden) return NVFP4_ERR_SHAPE;
+    if (tokens > INT32_MAX) return NVFP4_ERR_SHAPE;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    CombineParams p;
+    p.out = static_cast<const uint16_t *>(expert_out);
+    p.ld = ld;
+    p.out_rows = out_rows;
+    p.slots = d_slots;
+    p.weights = d_weights;
+    p.topk = topk;
+    p.hidden = hidden;
+    p.y = static_cast<uint16_t *>(y);
+    p.ldy = ldy;
+    k_moe_combine<<<(unsigned)tokens, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int64_t ld, float *d_fp8_scale,
+                                  void *stream) {
+    nvfp4_status st = check_tensor(in);
+    if (st != NVFP4_OK) return st;
+    if (d_fp8_scale == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_fp8_scale) & 3u) != 0) return NVFP4_ERR_ALIGNMENT;
+    if (in->rows > 0 && in->cols > 0) {
+        if (y == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(y) || ld % 16 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < in->cols) return NVFP4_ERR_SHAPE;
+    }
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    Fp8Params p;
+    p.codes = static_cast<const uint8_t *>(in->codes);
+    p.scales = static_cast<const uint8_t *>(in->scales);
+    p.layout = in->sf_layout;
+    p.global = in->global;
+    p.rows = in->rows;
+    p.cols = in->cols;
+    p.y = static_cast<uint8_t *>(y);
+    p.ld = ld;
+    p.fp8_scale = d_fp8_scale;
+    const int64_t blocks = in->rows * (in->cols / 16);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(blocks, 256), 8LL * sms));
+    k_dequantize_fp8<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                                    const int32_t *d_gather, const nvfp4_tensor *out,
                                    int32_t global_supplied, void *workspace,

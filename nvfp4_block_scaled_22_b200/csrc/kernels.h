@@ -96,6 +96,34 @@ inline int64_t transpose_tasks(int64_t x_rows, int64_t out_rows_padded) {
     return ((x_rows + 63) / 64) * ((out_rows_padded + 63) / 64);
 }
 
+// Consumers.  MoE combine: one CTA of 256 threads per token.
+constexpr int kMaxTopk = 32;
+struct CombineParams {
+    const uint16_t *out;     // expert outputs, BF16, pitch ld
+    int64_t ld;
+    int64_t out_rows;        // rows of out: slots at or past it are skipped
+    const int32_t *slots;    // [tokens x topk] rows of out (-1 = none)
+    const float *weights;    // [tokens x topk]
+    int32_t topk;
+    int64_t hidden;
+    uint16_t *y;             // [tokens x hidden] BF16, pitch ldy
+    int64_t ldy;
+};
+__global__ void k_moe_combine(CombineParams p);
+
+// NVFP4 -> E4M3 bytes (pitch ld) and the per-tensor factor RN(8 / g).
+struct Fp8Params {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    int32_t layout;
+    const float *global;
+    int64_t rows, cols;
+    uint8_t *y;
+    int64_t ld;
+    float *fp8_scale;
+};
+__global__ void k_dequantize_fp8(Fp8Params p);
+
 // MXFP4 (block 32, UE8M0 scales, no tensor scale); 256 threads.
 __global__ void k_encode_mx(EncodeParams p);
 __global__ void k_dequantize_mx(DequantParams p);

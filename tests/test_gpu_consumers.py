@@ -1,0 +1,68 @@
+"""GPU parity of the consumer steps against the oracle: the MoE per-token
+combine (bit for bit: the same FMA chain in the same order) and the NVFP4
+-> FP8 conversion for attention reads (bit for bit)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_scaled_22_b200 import binding as nb
+from nvfp4_block_scaled_22_b200 import inputs
+from tests.gpu_util import to_host_quantized
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    nb.lib()
+    yield
+    assert nb.nvfp4_check_status() == 0
+
+
+def test_moe_combine_full_routing():
+    r = inputs.MoeRouting()
+    g = torch.Generator(device=DEV).manual_seed(inputs.seed_for("moe", 9100))
+    out = torch.randn((r.padded_rows, inputs.MOE_HIDDEN), generator=g, device=DEV).to(torch.bfloat16)
+    slots = r.token_slots.to(DEV)
+    w = r.combine_weights.to(DEV)
+    y = nb.nvfp4_moe_combine(out, slots, w)
+    torch.cuda.synchronize()
+    ref = oracle.moe_combine(out.cpu(), r.token_slots.numpy(), r.combine_weights.numpy())
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("tokens,topk,hidden", [(1, 1, 8), (37, 3, 2056), (300, 8, 6144)])
+def test_moe_combine_shapes_and_skipped_slots(tokens, topk, hidden):
+    rng = np.random.default_rng(tokens + topk)
+    rows = 64
+    out = torch.from_numpy(rng.standard_normal((rows, hidden)).astype(np.float32)).to(torch.bfloat16)
+    slots = rng.integers(-1, rows + 5, (tokens, topk)).astype(np.int32)   # -1 and out-of-range skipped
+    w = rng.random((tokens, topk)).astype(np.float32)
+    y = nb.nvfp4_moe_combine(out.to(DEV), torch.from_numpy(slots).to(DEV), torch.from_numpy(w).to(DEV))
+    s2 = np.where(slots >= rows, -1, slots)
+    ref = oracle.moe_combine(out, s2, w)
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
+def test_fp8_conversion_kv_tensor(layout):
+    x = inputs.kv_tensor(0, 1, device=DEV).view(inputs.KV_TOKENS, -1)[:8192]
+    q = nb.nvfp4_quantize(x.contiguous(), layout=layout)
+    y, sc = nb.nvfp4_dequantize_fp8(q)
+    torch.cuda.synchronize()
+    ref, rsc = oracle.dequantize_fp8(to_host_quantized(q))
+    assert np.float32(sc.item()) == np.float32(rsc)
+    assert np.array_equal(y.cpu().numpy(), ref)
+
+
+def test_fp8_conversion_ragged_and_tiny_scales():
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(130, 96, generator=g)
+    x[3] *= 1e-6                                      # tiny block scales: FP8 underflow
+    x[4] *= 1e4
+    q = nb.nvfp4_quantize(x.to(torch.bfloat16).to(DEV))
+    y, sc = nb.nvfp4_dequantize_fp8(q)
+    ref, rsc = oracle.dequantize_fp8(to_host_quantized(q))
+    assert np.float32(sc.item()) == np.float32(rsc) and np.array_equal(y.cpu().numpy(), ref)

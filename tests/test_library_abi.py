@@ -85,6 +85,8 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     t = binding.CTensor(16, 16, 0, 4, 48, 0)
     assert lib.nvfp4_quantize_mx(16, 48, t, 16, 1 << 16, 0) == 3                 # cols % 32
     assert lib.nvfp4_mx_scales_bytes(256, 1024, 1) == 256 * 32
+    assert lib.nvfp4_moe_combine(16, 16, 4, 16, 16, 4, 0, 16, 16, 16, 0) == 1    # topk 0
+    assert lib.nvfp4_moe_combine(16, 16, 4, 16, 16, 4, 2, 12, 16, 16, 0) == 3    # hidden % 8
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
