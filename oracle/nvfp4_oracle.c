@@ -38,6 +38,12 @@
  *       outputs are combined per token); "FP4 KV-cache quantization",
  *       section on current implementations (the FP4 KV cache is
  *       dequantized to FP8 before attention).
+ *  [PG] gated activation between the expert up and down projections (the
+ *       MoE expert block of the GLM page, section 2): SiLU-gated linear
+ *       unit h = silu(gate) * up.
+ *  [PE] Cody and Waite, "Software Manual for the Elementary Functions"
+ *       (1980): exp by reduction x = n ln2 + r with ln2 split in a high part
+ *       exact in few bits and a low correction, then a polynomial in r.
  *  [PX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *       1, 2, 3" (SC 2011): the Philox4x32-10 counter-based generator.
  *  The FP32 evaluation order below is the convention the hot path is
@@ -838,4 +844,91 @@ void nvo_dequantize_fp8(const uint8_t *codes, const uint8_t *scales, int layout,
             uint8_t e = nvo_e4m3_rne_satfinite(fabsf(v));
             y[r * ld + c] = (uint8_t)(e | (signbit(v) ? 0x80 : 0));
         }
+}
+
+/* ------------------------------------------------------- gated activation */
+
+/* [PE] exp(x) for the SiLU, with every step an IEEE binary32 operation in a
+ * fixed order (so any implementation of these steps gives the same bits):
+ * x clamped to [-87, 87]; n = rint(RN(x * RN(log2 e))); r = fma(-n, L_hi, x),
+ * r = fma(-n, L_lo, r) with L_hi = ln 2 rounded to a multiple of 2^-16 and
+ * L_lo = RN(ln 2 - L_hi); p = the degree-7 Taylor polynomial of e^r in
+ * Horner form with fma (coefficients RN(1/k!)); result RN(p * 2^n). */
+float nvo_exp_ref(float x)
+{
+    const float l2e = 1.44269504088896340736f;
+    const float l_hi = 0.693145751953125f;               /* 45426 / 65536 */
+    const float l_lo = (float)(0.69314718055994530942 - 0.693145751953125);
+    if (x > 87.0f)
+        x = 87.0f;
+    if (x < -87.0f)
+        x = -87.0f;
+    float n = rintf(x * l2e);
+    float r = fmaf(-n, l_hi, x);
+    r = fmaf(-n, l_lo, r);
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    return p * ldexpf(1.0f, (int)n);
+}
+
+/* [PG] h = silu(g) * u = RN(RN(g * RN(1 / RN(1 + exp(-g)))) * u). */
+float nvo_swiglu(float g, float u)
+{
+    float e = nvo_exp_ref(-g);
+    float s = 1.0f / (1.0f + e);
+    return (g * s) * u;
+}
+
+/* Quantize h = silu(gate) * up of a [rows x 2I] BF16 tensor (gate in
+ * columns 0..I-1, up in I..2I-1: READING, the pages give no layout) to
+ * NVFP4 [rows x I], the FP32 values h quantized with the plain two-level
+ * steps (amax over h; RN(amax_b / 6) by division). */
+int nvo_quantize_swiglu(const uint16_t *gu, int64_t rows, int64_t inter, int64_t ld, uint8_t *codes,
+                        uint8_t *scales, int layout, float *g_out)
+{
+    if (inter % 16 != 0 || rows < 0 || inter < 0)
+        return NVO_ERR_SHAPE;
+    float m = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < inter; ++c) {
+            float h = fabsf(nvo_swiglu(nvo_bf16_to_f32(gu[r * ld + c]), nvo_bf16_to_f32(gu[r * ld + inter + c])));
+            if (!isfinite(h))
+                return NVO_ERR_NONFINITE;
+            if (h > m)
+                m = h;
+        }
+    float g;
+    int st = nvo_global_scale(m, &g);
+    *g_out = g;
+    if (st != NVO_OK)
+        return st;
+    memset(scales, 0, (size_t)nvo_scales_bytes(rows, inter, layout));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < inter / 16; ++b) {
+            float y[16], amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                int64_t c = b * 16 + i;
+                y[i] = nvo_swiglu(nvo_bf16_to_f32(gu[r * ld + c]), nvo_bf16_to_f32(gu[r * ld + inter + c]));
+                if (fabsf(y[i]) > amax_b)
+                    amax_b = fabsf(y[i]);
+            }
+            float t = amax_b / 6.0f;
+            t = t * g;
+            uint8_t s = nvo_e4m3_rne_satfinite(t);
+            float e = (s == 0) ? 0.0f : g / nvo_e4m3_decode(s);
+            scales[nvo_sf_offset(r, b, rows, inter, layout)] = s;
+            uint8_t *cb = codes + r * (inter / 2) + b * 8;
+            for (int i = 0; i < 8; ++i) {
+                uint8_t c0 = nvo_e2m1_rne_satfinite(y[2 * i] * e);
+                uint8_t c1 = nvo_e2m1_rne_satfinite(y[2 * i + 1] * e);
+                cb[i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return NVO_OK;
 }

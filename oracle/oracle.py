@@ -21,6 +21,7 @@ __all__ = [
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
     "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
     "dequantize_mx", "gemm_ref_mx", "QuantizedMX", "moe_combine", "dequantize_fp8",
+    "exp_ref", "swiglu", "quantize_swiglu",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -64,6 +65,10 @@ def lib() -> C.CDLL:
             "nvo_philox4x32_10": (None, [_p, _p, _p]),
             "nvo_ue8m0_decode": (C.c_double, [C.c_uint8]),
             "nvo_moe_combine": (None, [_p, _i64, _p, _p, _i64, _i64, _i64, _p, _i64]),
+            "nvo_exp_ref": (C.c_float, [C.c_float]),
+            "nvo_swiglu": (C.c_float, [C.c_float, C.c_float]),
+            "nvo_quantize_swiglu": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int,
+                                              C.POINTER(C.c_float)]),
             "nvo_dequantize_fp8": (None, [_p, _p, C.c_int, C.c_float, _i64, _i64, _p, _i64,
                                           C.POINTER(C.c_float)]),
             "nvo_mx_scales_bytes": (_i64, [_i64, _i64, C.c_int]),
@@ -361,6 +366,27 @@ def dequantize_fp8(q: Quantized) -> tuple[np.ndarray, float]:
     lib().nvo_dequantize_fp8(_ptr(np.ascontiguousarray(q.codes)), _ptr(np.ascontiguousarray(q.scales)),
                              q.layout, float(q.g), q.rows, q.cols, _ptr(y), q.cols, C.byref(sc))
     return y, float(sc.value)
+
+
+def exp_ref(x: float) -> float:
+    return float(lib().nvo_exp_ref(float(np.float32(x))))
+
+
+def swiglu(g: float, u: float) -> float:
+    return float(lib().nvo_swiglu(float(np.float32(g)), float(np.float32(u))))
+
+
+def quantize_swiglu(gu, layout: int = SF_SWIZZLED) -> tuple[int, Quantized]:
+    """NVFP4 of h = silu(gate) * up for gu = [gate | up] (BF16, rows x 2I)."""
+    b = bf16_bits(gu)
+    rows, two_i = b.shape
+    inter = two_i // 2
+    codes = np.zeros((rows, inter // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, inter, layout), np.uint8)
+    g = C.c_float()
+    st = lib().nvo_quantize_swiglu(_ptr(b), rows, inter, two_i, _ptr(codes), _ptr(scales), layout,
+                                   C.byref(g))
+    return st, Quantized(codes, scales, g.value, rows, inter, layout)
 
 
 if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):

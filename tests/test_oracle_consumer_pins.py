@@ -76,3 +76,52 @@ def test_fp8_conversion_values():
                 e = max(np.floor(np.log2(abs(exact))), -6)
                 assert abs(got - exact) <= 2.0 ** (e - 3) / 2
             assert got == 0 or np.sign(got) == np.sign(exact)
+
+
+def test_exp_against_libm_and_its_constants():
+    """The fixed-order exp stays within 2 ulp of the correctly rounded value
+    on a dense sweep, and its ln 2 split is exact: L_hi + L_lo = ln 2 to the
+    precision of the sum."""
+    import math
+    xs = np.float32(np.linspace(-87, 87, 200001))
+    worst = 0.0
+    for x in xs[::7]:
+        got = np.float32(oracle.exp_ref(float(x)))
+        ref = math.exp(float(x))
+        ulp = np.spacing(np.float32(ref))
+        worst = max(worst, abs(float(got) - ref) / float(ulp))
+    assert worst <= 2.0
+    assert 0.693145751953125 * 65536 == 45426
+    assert abs(0.693145751953125 + float(np.float32(math.log(2) - 0.693145751953125)) - math.log(2)) < 1e-13
+
+
+def test_silu_closed_forms():
+    assert oracle.swiglu(0.0, 1.0) == 0.0
+    for g in (20.0, 50.0, 87.5):
+        assert oracle.swiglu(g, 1.0) == np.float32(g)           # sigmoid rounds to 1
+    for g in (-100.0, -90.0):
+        assert abs(oracle.swiglu(g, 1.0)) < 1e-35               # silu(-large) -> -0
+    rng = np.random.default_rng(3)
+    for g in rng.standard_normal(200) * 4:
+        g = float(np.float32(g))
+        ref = g / (1 + np.exp(-g))
+        assert abs(oracle.swiglu(g, 1.0) - ref) <= 4 * np.spacing(np.float32(abs(ref))) + 1e-45
+
+
+def test_quantize_swiglu_reduces_to_plain_quantize():
+    """gate >= 20 makes silu(gate) = gate exactly; with up a power of two the
+    product is exact, so quantize_swiglu([gate | up]) = quantize(gate * up)."""
+    rng = np.random.default_rng(4)
+    gate = 20.0 + np.abs(rng.standard_normal((40, 64))) * 50
+    up = 2.0 ** rng.integers(-3, 4, (40, 64))
+    gu = _bf16(np.concatenate([gate, up], axis=1))
+    gf = oracle.bf16_to_f32(oracle.bf16_bits(gu))
+    prod = _bf16(gf[:, :64].astype(np.float64) * gf[:, 64:])
+    assert np.array_equal(oracle.bf16_to_f32(oracle.bf16_bits(prod)), gf[:, :64] * gf[:, 64:])
+    st, qs = oracle.quantize_swiglu(gu)
+    st2, qp = oracle.quantize(prod)
+    assert st == st2 == oracle.OK and np.float32(qs.g) == np.float32(qp.g)
+    assert np.array_equal(qs.codes, qp.codes) and np.array_equal(qs.scales, qp.scales)
+    zero = _bf16(np.concatenate([gate, np.zeros_like(up)], axis=1))
+    st, qz = oracle.quantize_swiglu(zero)
+    assert st == oracle.OK and qz.g == 1.0 and not qz.scales.any()
