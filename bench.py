@@ -672,13 +672,19 @@ def workload_line(name, args, device):
         sc = torch.zeros(1, dtype=torch.float32, device=device)
         fms = _timed(lambda: nb.nvfp4_dequantize_fp8(q, out=f8, scale=sc), args.steps, args.warmup, flush)
         fbytes = x.numel() * (0.5625 + 1.0)
+        # gated activation + quantize of the MoE intermediate (real rows)
+        gu = torch.randn((r.real_rows, 2 * inputs.MOE_INTER), generator=g, device=device).to(torch.bfloat16)
+        qh = nb.NVFP4Tensor.empty(r.real_rows, inputs.MOE_INTER, device=device)
+        sms_ = _timed(lambda: nb.nvfp4_quantize_swiglu(gu, out=qh, workspace=ws), args.steps, args.warmup, flush)
+        sbytes = r.real_rows * inputs.MOE_INTER * (2 * 2 * 2 + 0.5625)     # two passes over gate|up
         st = nb.nvfp4_check_status(ws)
         cgbs = cbytes / cms / 1e6
         line.update({"metric": "MoE top-8 combine GB/s (4096 tokens x 6144)", "value": cgbs, "unit": "GB/s",
                      "higher_is_better": True, "ms_per_step": cms,
                      "config": {"workload": "consumers: moe combine 4096 x top-8 x 6144; kv nvfp4->fp8 "
                                             "131072 x 1024", "l2": "flushed"},
-                     "combine_ms": cms, "fp8_ms": fms, "fp8_gbs": fbytes / fms / 1e6, "status": st,
+                     "combine_ms": cms, "fp8_ms": fms, "fp8_gbs": fbytes / fms / 1e6,
+                     "swiglu_quantize_ms": sms_, "swiglu_quantize_gbs": sbytes / sms_ / 1e6, "status": st,
                      "roofline": {"kernel": "k_moe_combine", "bound": "hbm", "achieved": cgbs,
                                   "peak": hbm_gbs, "unit": "GB/s", "frac": cgbs / hbm_gbs,
                                   "fp8_frac": fbytes / fms / 1e6 / hbm_gbs,

@@ -252,6 +252,21 @@ NVFP4_API nvfp4_status nvfp4_moe_combine(const void *expert_out, int64_t ld, int
                                          int64_t tokens, int32_t topk, int64_t hidden, void *y,
                                          int64_t ldy, void *stream);
 
+/* Gated activation between the expert up and down projections, quantized
+ * for the down projection: out = NVFP4 of h = silu(gate) * up, where row r
+ * of gate_up holds gate in columns [0, out->cols) and up in [out->cols,
+ * 2 * out->cols) (BF16, pitch ld >= 2 * out->cols).  silu(g) = g / (1 +
+ * exp(-g)) with every step one binary32 RN operation in a fixed order: exp
+ * by Cody and Waite's reduction (x clamped to [-87, 87]; n = rint(x *
+ * RN(log2 e)); r = x - n ln2 with ln2 split into 0.693145751953125 and
+ * RN(ln2 - that); the degree-7 Taylor polynomial of e^r in Horner form with
+ * fused multiply-adds; times 2^n), then RN(1 / RN(1 + e)), RN(g * s),
+ * RN(. * up).  h (FP32) is quantized with the two-level steps of
+ * nvfp4_quantize (its own tensor amax).  Workspace and errors as
+ * nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_quantize_swiglu(const void *gate_up, int64_t ld, const nvfp4_tensor *out,
+                                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* NVFP4 -> FP8 (E4M3) for an attention read ("FP4 KV-cache quantization":
  * current implementations dequantize the FP4 cache to FP8 before
  * attention): y = e4m3_rne_satfinite(e2m1(code) * s_b / 8) per value (one

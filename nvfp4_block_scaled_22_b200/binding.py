@@ -36,7 +36,7 @@ EXPORTED = (
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
     "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
-    "nvfp4_gemm_mx", "nvfp4_moe_combine", "nvfp4_dequantize_fp8",
+    "nvfp4_gemm_mx", "nvfp4_moe_combine", "nvfp4_dequantize_fp8", "nvfp4_quantize_swiglu",
 )
 
 
@@ -93,6 +93,7 @@ def lib() -> C.CDLL:
             "nvfp4_gemm_mx": (C.c_int, [T, T, vp, i64, vp, sz, vp]),
             "nvfp4_moe_combine": (C.c_int, [vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp]),
             "nvfp4_dequantize_fp8": (C.c_int, [T, vp, i64, vp, vp]),
+            "nvfp4_quantize_swiglu": (C.c_int, [vp, i64, T, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -358,6 +359,21 @@ def nvfp4_dequantize_fp8(t: NVFP4Tensor, out: torch.Tensor | None = None, scale:
     _check(lib().nvfp4_dequantize_fp8(C.byref(ct), out.data_ptr(), out.stride(0), scale.data_ptr(),
                                       _stream(stream)), "nvfp4_dequantize_fp8")
     return out, scale
+
+
+def nvfp4_quantize_swiglu(gate_up: torch.Tensor, out: NVFP4Tensor | None = None,
+                          layout: int = SF_SWIZZLED, workspace: Workspace | None = None,
+                          stream=None) -> NVFP4Tensor:
+    """NVFP4 of silu(gate) * up for gate_up = [gate | up] (BF16, rows x 2I)."""
+    assert gate_up.dtype == torch.bfloat16 and gate_up.dim() == 2 and gate_up.stride(1) == 1
+    rows, two_i = gate_up.shape
+    if out is None:
+        out = NVFP4Tensor.empty(rows, two_i // 2, layout, gate_up.device)
+    ws = workspace or default_workspace(gate_up.device)
+    t = out.c_struct()
+    _check(lib().nvfp4_quantize_swiglu(gate_up.data_ptr(), gate_up.stride(0), C.byref(t), ws.ptr,
+                                       ws.nbytes, _stream(stream)), "nvfp4_quantize_swiglu")
+    return out
 
 
 def nvfp4_global_scale(x: torch.Tensor, out: torch.Tensor | None = None,

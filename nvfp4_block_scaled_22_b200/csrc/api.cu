@@ -590,6 +590,49 @@ nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int64_t ld, f
     return launched(cudaGetLastError());
 }
 
+nvfp4_status nvfp4_quantize_swiglu(const void *gate_up, int64_t ld, const nvfp4_tensor *out,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
+    nvfp4_status st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    const int64_t rows = out->rows, inter = out->cols;
+    if (rows > 0 && inter > 0) {
+        if (gate_up == nullptr) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(gate_up) || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+        if (ld < 2 * inter) return NVFP4_ERR_SHAPE;
+    }
+    st = check_workspace(workspace, workspace_bytes,
+                         nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, inter, 0, 0));
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SwigluParams p;
+    p.gu = static_cast<const uint16_t *>(gate_up);
+    p.ld = ld;
+    p.rows = rows;
+    p.inter = inter;
+    p.codes = static_cast<uint8_t *>(out->codes);
+    p.scales = static_cast<uint8_t *>(out->scales);
+    p.layout = out->sf_layout;
+    p.global = out->global;
+    p.partials = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    p.status = reinterpret_cast<uint32_t *>(workspace);
+    const int64_t tasks = rows * ceil_div(inter / 16, 32);
+    int grid = (int)std::min<int64_t>(std::min<int64_t>(ceil_div(tasks, 8), 4LL * sms), kMaxPartials);
+    if (grid < 1) grid = 1;
+    p.n_partials = grid;
+    k_amax_swiglu<<<grid, 256, 0, s>>>(p);
+    st = launched(cudaGetLastError());
+    if (st != NVFP4_OK) return st;
+    const int64_t rows_out = (out->sf_layout == NVFP4_SF_SWIZZLED_128x4) ? ceil_div(rows, 128) * 128 : rows;
+    const int64_t etasks = rows_out * ceil_div(ceil_div(inter / 16, 4) * 4, 32);
+    int egrid = (int)std::min<int64_t>(ceil_div(etasks, 8), 8LL * sms);
+    if (egrid < 1) egrid = 1;
+    k_encode_swiglu<<<egrid, 256, 0, s>>>(p);
+    return launched(cudaGetLastError());
+}
+
 nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                                    const int32_t *d_gather, const nvfp4_tensor *out,
                                    int32_t global_supplied, void *workspace,

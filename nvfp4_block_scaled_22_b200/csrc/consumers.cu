@@ -6,6 +6,9 @@
 // k_dequantize_fp8  : NVFP4 -> FP8 (E4M3) for an attention read ("FP4
 //                     KV-cache quantization": current implementations
 //                     dequantize the FP4 cache to FP8 before attention).
+// k_amax_swiglu,
+// k_encode_swiglu   : NVFP4 of the SiLU-gated activation h = silu(gate) * up
+//                     between the expert up and down projections.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -21,6 +24,57 @@ __device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// exp(x) by Cody and Waite's reduction and a degree-7 Taylor polynomial,
+// every step one binary32 RN operation in a fixed order (the same steps the
+// checker uses, so the bits agree): x clamped to [-87, 87] (NaN kept),
+// n = rint(RN(x * RN(log2 e))), r = x - n * ln2 with ln2 split in a 16-bit
+// high part and a low correction (two FMAs), Horner with FMA, times 2^n.
+__device__ __forceinline__ float exp_ref(float x) {
+    if (x != x) return x;
+    if (x > 87.0f) x = 87.0f;
+    if (x < -87.0f) x = -87.0f;
+    const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));           // RN(log2 e)
+    float r = __fmaf_rn(-n, 0.693145751953125f, x);                 // ln2 high part
+    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);                          // RN(ln2 - high)
+    float p = 1.0f / 5040.0f;
+    p = __fmaf_rn(p, r, 1.0f / 720.0f);
+    p = __fmaf_rn(p, r, 1.0f / 120.0f);
+    p = __fmaf_rn(p, r, 1.0f / 24.0f);
+    p = __fmaf_rn(p, r, 1.0f / 6.0f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    return __fmul_rn(p, __uint_as_float((uint32_t)((int)n + 127) << 23));   // 2^n, |n| <= 126
+}
+
+// h = RN(RN(g * RN(1 / RN(1 + exp(-g)))) * u).
+__device__ __forceinline__ float swiglu(float g, float u) {
+    const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_ref(-g)));
+    return __fmul_rn(__fmul_rn(g, s), u);
+}
+
+// h values of block b (16 columns) of row r: gate at column 16b + i, up at
+// inter + 16b + i.
+__device__ __forceinline__ void swiglu_block(const uint16_t *row, int64_t inter, int64_t b, float h[16]) {
+    const uint4 *gp = reinterpret_cast<const uint4 *>(row + b * 16);
+    const uint4 *up = reinterpret_cast<const uint4 *>(row + inter + b * 16);
+    const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1), u0 = __ldg(up), u1 = __ldg(up + 1);
+    const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[2 * i] = swiglu(__uint_as_float(gw[i] << 16), __uint_as_float(uw[i] << 16));
+        h[2 * i + 1] = swiglu(__uint_as_float(gw[i] & 0xFFFF0000u), __uint_as_float(uw[i] & 0xFFFF0000u));
+    }
+}
+
+__device__ __forceinline__ uint32_t abs_max16(const float h[16]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = absmax_nan(m, h[i]);
+    return __float_as_uint(m) & 0x7FFFFFFFu;
 }
 
 }  // namespace
@@ -85,6 +139,67 @@ __global__ void __launch_bounds__(256) k_dequantize_fp8(Fp8Params p) {
             out[2 * h + 1] = b[2] | (b[3] << 16);
         }
         *reinterpret_cast<uint4 *>(p.y + r * p.ld + c * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// ------------------------------------------------------ gated activation
+// Lane per 16-value block of h; tasks = (row, 32-block group), grid-stride.
+__global__ void __launch_bounds__(256) k_amax_swiglu(SwigluParams p) {
+    __shared__ uint32_t red[8];
+    const int lane = threadIdx.x & 31;
+    const int64_t blocks = p.inter / 16, groups = (blocks + 31) / 32;
+    uint32_t m = 0;
+    for (int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); t < p.rows * groups;
+         t += (int64_t)gridDim.x * 8) {
+        const int64_t r = t / groups, b = (t - r * groups) * 32 + lane;
+        if (b >= blocks) continue;
+        float h[16];
+        swiglu_block(p.gu + r * p.ld, p.inter, b, h);
+        m = max(m, abs_max16(h));
+    }
+    const uint32_t v = block_reduce_max(m, red);
+    if (threadIdx.x == 0) p.partials[blockIdx.x] = v;
+}
+
+__global__ void __launch_bounds__(256) k_encode_swiglu(SwigluParams p) {
+    __shared__ uint32_t red[8];
+    __shared__ EncodeTables tab;
+    float g;
+    if (!global_from_partials(p.partials, p.n_partials, p.status, &g, red)) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.global = g;
+    fill_tables(tab, g);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t blocks = p.inter / 16, blocks4 = (blocks + 3) / 4 * 4, col_tiles = blocks4 / 4;
+    const int64_t rows_out = (p.layout == 0) ? (p.rows + 127) / 128 * 128 : p.rows;
+    const int64_t groups = (blocks4 + 31) / 32;
+    for (int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); t < rows_out * groups;
+         t += (int64_t)gridDim.x * 8) {
+        const int64_t r = t / groups, b = (t - r * groups) * 32 + lane;
+        uint32_t s = 0;
+        if (r < p.rows && b < blocks) {
+            float h[16];
+            swiglu_block(p.gu + r * p.ld, p.inter, b, h);
+            const uint32_t bits = abs_max16(h);
+            s = e4m3_from_f32(__fmul_rn(div6_f32(__uint_as_float(bits)), g));
+            const float e = tab.inv_s[s & 0x7Fu];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) h[i] = __fmul_rn(h[i], e);
+            *reinterpret_cast<uint2 *>(p.codes + r * (p.inter / 2) + b * 8) =
+                make_uint2(e2m1x4_from_f32(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]),
+                           e2m1x4_from_f32(h[8], h[9], h[10], h[11], h[12], h[13], h[14], h[15]));
+        }
+        uint32_t word = s << (8 * (lane & 3));
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+        if ((lane & 3) == 0 && b < blocks4 && (p.layout == 0 || b < blocks)) {
+            uint8_t *sp = p.scales + sf_offset(r, b, blocks, col_tiles, p.layout);
+            if (p.layout == 0 || ((blocks & 3) == 0 && b + 4 <= blocks)) {
+                *reinterpret_cast<uint32_t *>(sp) = word;
+            } else {
+                for (int j = 0; j < 4 && b + j < blocks; ++j) sp[j] = (uint8_t)(word >> (8 * j));
+            }
+        }
     }
 }
 

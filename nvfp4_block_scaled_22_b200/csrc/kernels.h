@@ -124,6 +124,22 @@ struct Fp8Params {
 };
 __global__ void k_dequantize_fp8(Fp8Params p);
 
+// SiLU-gated activation + quantize: gu = [gate | up] BF16 rows x 2*inter.
+struct SwigluParams {
+    const uint16_t *gu;
+    int64_t ld;
+    int64_t rows, inter;
+    uint8_t *codes;
+    uint8_t *scales;
+    int32_t layout;
+    float *global;
+    uint32_t *partials;
+    int32_t n_partials;
+    uint32_t *status;
+};
+__global__ void k_amax_swiglu(SwigluParams p);
+__global__ void k_encode_swiglu(SwigluParams p);
+
 // MXFP4 (block 32, UE8M0 scales, no tensor scale); 256 threads.
 __global__ void k_encode_mx(EncodeParams p);
 __global__ void k_dequantize_mx(DequantParams p);

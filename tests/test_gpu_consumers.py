@@ -66,3 +66,17 @@ def test_fp8_conversion_ragged_and_tiny_scales():
     y, sc = nb.nvfp4_dequantize_fp8(q)
     ref, rsc = oracle.dequantize_fp8(to_host_quantized(q))
     assert np.float32(sc.item()) == np.float32(rsc) and np.array_equal(y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("rows,inter", [(1, 16), (37, 80), (300, 1040), (4096, 2048)])
+@pytest.mark.parametrize("layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
+def test_swiglu_quantize(rows, inter, layout):
+    g = torch.Generator().manual_seed(rows + inter)
+    gu = (torch.randn(rows, 2 * inter, generator=g) * 3).to(torch.bfloat16)
+    gu[0, :4] = torch.tensor([90.0, -90.0, 0.0, -0.0])          # clamp ends and zeros
+    q = nb.nvfp4_quantize_swiglu(gu.to(DEV), layout=layout)
+    assert nb.nvfp4_check_status() == 0
+    st, ref = oracle.quantize_swiglu(gu, layout)
+    assert st == oracle.OK
+    from tests.gpu_util import assert_quantized_equal
+    assert_quantized_equal(q, ref, f"swiglu {rows}x{inter}")
