@@ -73,7 +73,9 @@ __device__ __forceinline__ SignFlips sign_flips(uint32_t mask) {
     return f;
 }
 
-__device__ __forceinline__ void rht16(uint4 a, uint4 b, const SignFlips &f, float2 P[8]) {
+// Sign flips, conversion and butterfly stages 1, 2, 4 (pairs P[i] =
+// (z_i, z_{i+8})).
+__device__ __forceinline__ void rht16_stages124(uint4 a, uint4 b, const SignFlips &f, float2 P[8]) {
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -94,12 +96,42 @@ __device__ __forceinline__ void rht16(uint4 a, uint4 b, const SignFlips &f, floa
             }
         }
     }
-    const float2 q = make_float2(0.25f, 0.25f);
+}
+
+// The transform without the final quarter: P[i] = (z_i, z_{i+8}), y = z/4.
+__device__ __forceinline__ void rht16_unscaled(uint4 a, uint4 b, const SignFlips &f, float2 P[8]) {
+    rht16_stages124(a, b, f, P);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float u = P[i].x, v = P[i].y;
-        P[i] = mul_f32x2(make_float2(__fadd_rn(u, v), __fsub_rn(u, v)), q);
+        P[i] = make_float2(__fadd_rn(u, v), __fsub_rn(u, v));
     }
+}
+
+__device__ __forceinline__ void rht16(uint4 a, uint4 b, const SignFlips &f, float2 P[8]) {
+    rht16_unscaled(a, b, f, P);
+    const float2 q = make_float2(0.25f, 0.25f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) P[i] = mul_f32x2(P[i], q);
+}
+
+// max |y_i| of the transformed block without forming y, for the tensor
+// amax pass.  The last butterfly stage maps a pair (u, v) to (u + v, u - v);
+// one of the two exact values has magnitude |u| + |v|, and rounding is
+// symmetric, so max(|RN(u + v)|, |RN(u - v)|) = RN(|u| + |v|).  RN(x / 4) is
+// monotone, so the quarter is applied once to the maximum.  Inf and NaN
+// reach the result (NaN-propagating max), as in the full transform.
+__device__ __forceinline__ uint32_t rht16_abs_max_bits(uint4 a, uint4 b, const SignFlips &f) {
+    float2 P[8];
+    rht16_stages124(a, b, f, P);
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(fabsf(P[i].x), fabsf(P[i].y));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = absmax_nan(m[i], m[i + 4]);
+    m[0] = absmax_nan(m[0], m[2]);
+    m[1] = absmax_nan(m[1], m[3]);
+    return __float_as_uint(__fmul_rn(absmax_nan(m[0], m[1]), 0.25f)) & 0x7FFFFFFFu;
 }
 
 // max |y_i| as f32 bits; Inf and NaN patterns compare above every finite one.

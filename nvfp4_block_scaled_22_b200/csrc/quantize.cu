@@ -89,17 +89,10 @@ __global__ void __launch_bounds__(kThreads) k_amax_rht(const uint16_t *__restric
         for (; c + 32 < blocks; c += 64) {
             uint4 a0 = __ldg(p + 2 * c), b0 = __ldg(p + 2 * c + 1);
             uint4 a1 = __ldg(p + 2 * c + 64), b1 = __ldg(p + 2 * c + 65);
-            float2 y[8];
-            rht16(a0, b0, f, y);
-            m = max(m, abs_max_bits(y));
-            rht16(a1, b1, f, y);
-            m = max(m, abs_max_bits(y));
+            m = max(m, rht16_abs_max_bits(a0, b0, f));
+            m = max(m, rht16_abs_max_bits(a1, b1, f));
         }
-        if (c < blocks) {
-            float2 y[8];
-            rht16(__ldg(p + 2 * c), __ldg(p + 2 * c + 1), f, y);
-            m = max(m, abs_max_bits(y));
-        }
+        if (c < blocks) m = max(m, rht16_abs_max_bits(__ldg(p + 2 * c), __ldg(p + 2 * c + 1), f));
     }
     uint32_t v = block_reduce_max(m, red);
     if (threadIdx.x == 0) partials[blockIdx.x] = v;

@@ -160,11 +160,8 @@ __global__ void __launch_bounds__(kTThreads) k_amax_t_rht(const uint16_t *__rest
                        if (r0 + 16 * k >= R) break;                    // uniform across the warp
                        uint4 a, b, c, d;
                        column_blocks(tile, k, lane, a, b, c, d);
-                       float2 y[8];
-                       rht16(a, b, f, y);                              // zero columns stay zero
-                       m = max(m, abs_max_bits(y));
-                       rht16(c, d, f, y);
-                       m = max(m, abs_max_bits(y));
+                       m = max(m, rht16_abs_max_bits(a, b, f));        // zero columns stay zero
+                       m = max(m, rht16_abs_max_bits(c, d, f));
                    }
                });
     const uint32_t v = block_reduce_max(m, red);
