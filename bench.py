@@ -59,6 +59,23 @@ def gemm_traffic():
     return GEMM_TRAFFIC_BYTES if h.hexdigest()[:16] == GEMM_TRAFFIC_SRC_SHA else None
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of `values` over all ranks (identity with one
+    rank): every multi-GPU time in the JSON line is the slowest rank's."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(world, units_per_step, steps, total_ms):
+    """Whole-job rate of `world` independent replicas (weak scaling): the
+    units every rank processed over the slowest rank's time."""
+    return world * units_per_step * steps / (total_ms / 1e3)
+
+
 def env_rank():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
             int(os.environ.get("WORLD_SIZE", "1")))
@@ -752,13 +769,10 @@ def main():
     total_ms = sum(step_ms)
     gemm_avg = sum(gemm_ms) / len(gemm_ms)
     quant_avg = sum(quant_ms) / len(quant_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms, gemm_avg, quant_avg], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, gemm_avg, quant_avg = t.tolist()
+    total_ms, gemm_avg, quant_avg = max_over_ranks([total_ms, gemm_avg, quant_avg], dist, device)
     flops = 2.0 * M * N * K
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value = replica_throughput(world, flops, args.steps, total_ms) / 1e12
     gemm_tflops = flops / (gemm_avg / 1e3) / 1e12
 
     sweep_ms, sweep_ms1, sst = (float("nan"),) * 2 + (0,)
@@ -767,10 +781,7 @@ def main():
     e2e_ms, h2d, d2h = float("nan"), 0, 0
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup)
-    if dist is not None:
-        t = torch.tensor([sweep_ms, sweep_ms1, e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        sweep_ms, sweep_ms1, e2e_ms = t.tolist()
+    sweep_ms, sweep_ms1, e2e_ms = max_over_ranks([sweep_ms, sweep_ms1, e2e_ms], dist, device)
 
     if rank == 0:
         gbs_2pass = SWEEP_N * QUANT_BYTES_PER_VALUE_2PASS / (sweep_ms / 1e3) / 1e9
