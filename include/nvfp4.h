@@ -100,10 +100,14 @@ NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
 /* Bytes of the block-scale array for the given layout (see above). */
 NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout);
 
-/* Bytes of workspace the operation needs (at least 16; the first 4 bytes
- * are the status word).  The arguments are the operation's sizes
- * (rows/cols, or m/n/k) and the group count for grouped calls; the current
- * implementation needs a fixed amount per operation. */
+/* Bytes of workspace the operation can use (the first 4 bytes are the
+ * status word).  The arguments are the operation's sizes (rows/cols, or
+ * m/n/k) and the group count for grouped calls.  Quantize calls need the
+ * returned amount.  A dense GEMM needs only 256 bytes; with M <= 128 the
+ * returned amount also holds the FP32 partial sums of the split-K path (K
+ * split over up to 8 SMs per output tile when there are fewer output tiles
+ * than SMs), which a smaller workspace turns off without changing what is
+ * computed beyond the FP32 summation order. */
 NVFP4_API size_t nvfp4_workspace_bytes(int32_t op, int64_t a, int64_t b, int64_t c, int32_t groups);
 
 /* ---- quantize --------------------------------------------------------- */
@@ -340,7 +344,9 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t
 /* ---- GEMM ------------------------------------------------------------- */
 
 /* W4A4 linear layer on the FP4 tensor cores (block-scaled MMA, FP32
- * accumulation):  D[i,j] = bf16_rne(alpha * sum_k a_ik * w_jk), where a and w
+ * accumulation; for small M with a large enough workspace the K range is
+ * split over several SMs and the FP32 partial sums are added in split order
+ * by a second kernel):  D[i,j] = bf16_rne(alpha * sum_k a_ik * w_jk), where a and w
  * are the E2M1 codes times their E4M3 block scales and
  * alpha = RN(1 / RN(gA * gW)) is formed on the device from *A->global and
  * *W->global.  ("NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens",

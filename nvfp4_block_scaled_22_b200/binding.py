@@ -179,7 +179,9 @@ class Workspace:
 
     def __init__(self, device="cuda", nbytes: int | None = None):
         if nbytes is None:
-            nbytes = max(nvfp4_workspace_bytes(op) for op in range(5))
+            # room for the split-K slices of small-M GEMMs (a smaller
+            # workspace only turns the split off)
+            nbytes = max(max(nvfp4_workspace_bytes(op) for op in range(5)), 32 << 20)
         self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
     @property

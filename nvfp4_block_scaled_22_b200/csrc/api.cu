@@ -274,11 +274,17 @@ size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout) {
     return (size_t)(ceil_div(rows, 128) * 128 * ceil_div(s, 4) * 4);
 }
 
-size_t nvfp4_workspace_bytes(int32_t op, int64_t, int64_t, int64_t, int32_t) {
+size_t nvfp4_workspace_bytes(int32_t op, int64_t m, int64_t n, int64_t k, int32_t groups) {
     switch (op) {
         case NVFP4_OP_QUANTIZE:
         case NVFP4_OP_QUANTIZE_GATHER:
             return kStatusBytes + 4 * kMaxPartials;
+        case NVFP4_OP_GEMM:
+            // dense GEMMs with few output tiles may split K into up to 8 FP32
+            // slices; a smaller workspace only turns the split off
+            if (groups == 0 && m > 0 && n > 0 && k > 0 && m <= kBM)
+                return kStatusBytes + (size_t)std::min<int64_t>(8, ceil_div(k / 64, 4)) * m * n * 4;
+            return kStatusBytes;
         default:
             return kStatusBytes;
     }
@@ -745,8 +751,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(D) & 1u) != 0) return NVFP4_ERR_ALIGNMENT;
     if (ldd < n) return NVFP4_ERR_SHAPE;
-    st = check_workspace(workspace, workspace_bytes,
-                         nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, groups));
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);   // more enables split-K
     if (st != NVFP4_OK) return st;
     int sms = 0;
     st = current_device(&sms);
@@ -779,14 +784,43 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.n_fastest = (A->rows * (k / 2) > kL2SweepBytes && A->rows > W->rows) ? 1 : 0;
     p.status = reinterpret_cast<uint32_t *>(workspace);
     p.timeout_cycles = g_timeout_cycles;
+    p.splits = 1;
+    p.partial = nullptr;
+    // Split-K for dense GEMMs with fewer output tiles than SMs (small M):
+    // pick the split count that minimises the stage count of the busiest SM
+    // (ties: fewer splits), if the FP32 slices fit in the workspace.
+    const int64_t tiles_mn = ceil_div(m, kBM) * ceil_div(n, kBN);
+    const int ktiles = (int)ceil_div(k / 64, 4);
+    if (!mx && !pair && groups == 0 && tiles_mn < sms && n % 16 == 0 && p.d_vec16) {
+        int best = 1;
+        int64_t best_cost = ktiles;                              // one unit per SM
+        for (int sp = 2; sp <= std::min(8, ktiles); ++sp) {
+            const int64_t cost = ceil_div(tiles_mn * sp, sms) * ceil_div(ktiles, sp);
+            const size_t need = kStatusBytes + (size_t)sp * (size_t)m * (size_t)n * 4;
+            if (cost < best_cost && need <= workspace_bytes) {
+                best = sp;
+                best_cost = cost;
+            }
+        }
+        if (best > 1) {
+            p.splits = best;
+            p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+        }
+    }
     if (pair) {
         const int64_t pair_tiles = ceil_div(m, 256) * ceil_div(n, 256);
         const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tiles, sms / 2));
         return launched(launch_gemm_pair(tmA, tmB, p, clusters, static_cast<cudaStream_t>(stream)));
     }
-    const int64_t tiles = ceil_div(m, kBM) * ceil_div(n, kBN);
+    const int64_t tiles = tiles_mn * p.splits;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, sms));
-    return launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream), mx));
+    st = launched(launch_gemm(tmA, tmB, p, grid, static_cast<cudaStream_t>(stream), mx));
+    if (st != NVFP4_OK || p.splits == 1) return st;
+    const int64_t quads = m * (n / 4);
+    const int fgrid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(quads, 256), 4LL * sms));
+    k_splitk_finalize<<<fgrid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        p.partial, p.splits, (int)m, (int)n, p.ga, p.gw, p.d, p.ldd);
+    return launched(cudaGetLastError());
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,

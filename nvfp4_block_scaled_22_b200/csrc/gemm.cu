@@ -129,7 +129,9 @@ __device__ __forceinline__ TileInfo tile_info(int tile, int mtiles, int ntiles,
 // covering 128 K values; no tensor scales, alpha = 1).  The MMA reads two
 // scale bytes per row and K=64 step; the scale writers put them in bytes
 // 0-1 of the same TMEM words the NVFP4 path fills with four.
-template <bool kMx>
+// kSplit: split-K instance (p.splits > 1, dense only); the other instances
+// take the whole K range per tile and compile without that bookkeeping.
+template <bool kMx, bool kSplit>
 __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                           const GemmParams &p) {
     extern __shared__ uint8_t smem_raw[];
@@ -186,15 +188,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
 
     const int mtiles = (p.groups == 0) ? (p.m + kBM - 1) / kBM : s_off[p.groups] / kBM;
     const int ntiles = (p.n + kBN - 1) / kBN;
-    const int tiles = mtiles * ntiles;
+    // Split-K (dense, small M): tile index = split * (mtiles * ntiles) + output
+    // tile; split s covers stages [s * ktiles / splits, (s + 1) * ktiles / splits).
+    const int tiles_mn = mtiles * ntiles;
+    const int splits = kSplit ? p.splits : 1;
+    const int tiles = tiles_mn * splits;
     const int kblocks = p.k / 64;                    // 64-value MMA steps
     const int ktiles = (kblocks + 3) / 4;            // 256-value stages
     // one 128-row band of scale tiles; a tile covers 64 (NVFP4) or 128 (MX) K
     const int64_t sf_rowblock_bytes = (int64_t)(kMx ? (kblocks + 1) / 2 : kblocks) * 512;
     constexpr int64_t kSfStageStride = kMx ? 1024 : 2048;      // scale bytes per band and stage
-    const int my_tiles =
-        (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const int total_k = my_tiles * ktiles;           // stages this CTA runs, in order
+    auto krange = [&](int tile, int &kt0, int &kt1) {
+        if (!kSplit) {
+            kt0 = 0;
+            kt1 = ktiles;
+            return;
+        }
+        const int sp = tile / tiles_mn;
+        kt0 = (sp * ktiles) / splits;
+        kt1 = ((sp + 1) * ktiles) / splits;
+    };
+    int total_k = 0;                                  // stages this CTA runs, in order
+    if (kSplit) {
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            int a, b;
+            krange(tile, a, b);
+            total_k += b - a;
+        }
+    } else {
+        total_k = ((int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0) * ktiles;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -206,11 +229,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             for (int s = 0; s < kStages; ++s) armed[s] = false;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-                const TileInfo t = tile_info(tile, mtiles, ntiles, p, s_off, s_rows);
+                const TileInfo t = tile_info(kSplit ? tile % tiles_mn : tile, mtiles, ntiles, p, s_off, s_rows);
                 const int64_t sfa_base = (int64_t)(t.a_row0 / kBM) * sf_rowblock_bytes;
                 const int brb = t.b_row0 / kBM;
                 const int halves = (brb + 1 < p.b_row_blocks) ? 2 : 1;
-                for (int kt = 0; kt < ktiles; ++kt) {
+                int kt0, kt1;
+                krange(tile, kt0, kt1);
+                for (int kt = kt0; kt < kt1; ++kt) {
                     if (!wait_or_abort(&sh->empty[stage], phase ^ 1, sh, p)) { ok = false; break; }
                     const int nkb = min(4, kblocks - 4 * kt);
                     const uint32_t sf_bytes = (uint32_t)(kMx ? (nkb + 1) / 2 : nkb) * 512;
@@ -316,7 +341,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             // is incremental (no divisions), and the MMA waits once per pair.
             const int last_nkb = kblocks - 4 * (ktiles - 1);
             uint32_t acc_phase = 0;
-            int stage = 0, kt = 0;
+            int stage = 0;
+            int mma_tile = blockIdx.x, kt0, kt1;           // current tile and its stage range
+            krange(mma_tile, kt0, kt1);
+            int kt = kt0;
             uint32_t stage_off = 0;                       // stage * kStageBytes / 16
             uint32_t sfa = tmem + kAccCols;               // stage's TMEM scale columns
             for (int g = 0; g < total_k; ++g) {
@@ -326,11 +354,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                         break;
                     tc_fence_after();
                 }
-                if (kt == 0) {   // first stage of a tile: the accumulator must be free
+                if (kt == kt0) {   // first stage of a tile: the accumulator must be free
                     if (!wait_or_abort(&sh->acc_empty, acc_phase ^ 1, sh, p)) break;
                     tc_fence_after();
                 }
-                const uint32_t first = kt != 0 ? 1u : 0u;
+                const uint32_t first = kt != kt0 ? 1u : 0u;
                 auto mma = [&](int kb, uint32_t acc) {
                     if (kMx)
                         mma_mxf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
@@ -345,13 +373,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     mma(2, 1u);
                     mma(3, 1u);
                 } else {
-                    for (int kb = 0; kb < last_nkb; ++kb) mma(kb, (kt | kb) != 0 ? 1u : 0u);
+                    for (int kb = 0; kb < last_nkb; ++kb) mma(kb, (kt != kt0 || kb != 0) ? 1u : 0u);
                 }
                 tc_commit(&sh->empty[stage]);
-                if (kt == ktiles - 1) {
+                if (kt == kt1 - 1) {
                     tc_commit(&sh->acc_full);
                     acc_phase ^= 1;
-                    kt = 0;
+                    mma_tile += gridDim.x;
+                    krange(mma_tile, kt0, kt1);
+                    kt = kt0;
                 } else {
                     ++kt;
                 }
@@ -376,6 +406,34 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         const int chalf = (warp - kFirstEpiWarp) / 4;          // column half of the tile
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            if (kSplit) {
+                // split-K: this split's FP32 sums, unscaled, into its slice;
+                // each lane holds one row (16 columns per TMEM load)
+                if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
+                tc_fence_after();
+                const TileInfo t = tile_info(tile % tiles_mn, mtiles, ntiles, p, s_off, s_rows);
+                const int row = t.a_row0 + quarter * 32 + lane;
+                const int col0 = t.nt * kBN + chalf * 128;
+                float *dst = p.partial + ((int64_t)(tile / tiles_mn) * p.m + row) * p.n + col0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                           (uint32_t)(chalf * 128 + 16 * c), r);
+                    tmem_ld_wait();
+                    if (row < p.m && col0 + 16 * c < p.n) {        // n % 16 == 0 in this mode
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            reinterpret_cast<uint4 *>(dst + 16 * c)[q] =
+                                make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->acc_empty);
+                acc_phase ^= 1;
+                continue;
+            }
             // Only alpha is held across the accumulator loads; the tile's
             // coordinates are derived again for the stores (fewer live
             // registers next to the 64 output words).
@@ -420,34 +478,63 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     }
 }
 
+// D = bf16(RN(RN(sum of the split slices in split order) * alpha)), alpha =
+// RN(1 / RN(gA * gW)); four columns per thread (n % 16 == 0).
+__global__ void __launch_bounds__(256) k_splitk_finalize(const float *partial, int splits, int m,
+                                                         int n, const float *ga, const float *gw,
+                                                         uint16_t *d, int64_t ldd) {
+    const float alpha = __frcp_rn(__fmul_rn(*ga, *gw));
+    const int64_t quads = (int64_t)m * (n / 4);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < quads;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / (n / 4), col = (i - row * (n / 4)) * 4;
+        float4 acc = __ldg(reinterpret_cast<const float4 *>(partial + row * n + col));
+        for (int s = 1; s < splits; ++s) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(partial + ((int64_t)s * m + row) * n + col));
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
+        }
+        uint32_t *dp = reinterpret_cast<uint32_t *>(d + row * ldd + col);
+        dp[0] = bf16x2_from_f32(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
+        dp[1] = bf16x2_from_f32(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+    }
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmParams p) {
-    gemm_body<false>(tmA, tmB, p);
+    gemm_body<false, false>(tmA, tmB, p);
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm_nvf4_splitk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+    gemm_body<false, true>(tmA, tmB, p);
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm_mxf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmParams p) {
-    gemm_body<true>(tmA, tmB, p);
+    gemm_body<true, false>(tmA, tmB, p);
 }
 
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t stream, bool mx) {
-    static bool attr_set[64][2] = {};
+    static bool attr_set[64][3] = {};
+    const int which = mx ? 1 : (p.splits > 1 ? 2 : 0);
+    void (*kernel)(const CUtensorMap, const CUtensorMap, const GemmParams) =
+        mx ? k_gemm_mxf4 : (p.splits > 1 ? k_gemm_nvf4_splitk : k_gemm_nvf4);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev][mx ? 1 : 0]) {
-        e = cudaFuncSetAttribute(mx ? k_gemm_mxf4 : k_gemm_nvf4,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+    if (dev < 0 || dev >= 64 || !attr_set[dev][which]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev][mx ? 1 : 0] = true;
+        if (dev >= 0 && dev < 64) attr_set[dev][which] = true;
     }
-    if (mx)
-        k_gemm_mxf4<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
-    else
-        k_gemm_nvf4<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
+    kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
     return cudaGetLastError();
 }
 

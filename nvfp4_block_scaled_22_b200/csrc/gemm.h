@@ -44,6 +44,8 @@ struct GemmParams {
     int32_t a_row_blocks;     // ceil(A rows / 128), bounds the grouped slots
     int32_t b_row_blocks;     // ceil(W rows / 128), bounds the SFB reads
     int32_t n_fastest;        // tile order: 0 = M fastest, 1 = N fastest
+    int32_t splits;           // K splits (1 = none); > 1: FP32 slices to `partial`
+    float *partial;           // splits x m x n FP32 partial sums (split-K only)
     uint32_t *status;
     long long timeout_cycles;
 };
@@ -60,6 +62,11 @@ cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, con
 // stay in L2.  M fastest sweeps A; when A's codes exceed this many bytes
 // and W is the smaller operand, N fastest sweeps W instead.
 constexpr int64_t kL2SweepBytes = 48ll << 20;
+
+// Split-K finalize: D = bf16(RN(sum_s partial[s] * alpha)), sums in split
+// order; 256 threads.
+__global__ void k_splitk_finalize(const float *partial, int splits, int m, int n, const float *ga,
+                                  const float *gw, uint16_t *d, int64_t ldd);
 
 // Dense GEMMs with at least this many rows run on CTA pairs.
 constexpr int64_t kPairMinRows = 256;
