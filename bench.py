@@ -44,8 +44,8 @@ FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
 # the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
 # Reported only while the kernel's sources hash to the profiled version.
-GEMM_TRAFFIC_BYTES = 88.24e6 + 292.66e6
-GEMM_TRAFFIC_SRC_SHA = "ece00d8fd2be476e"
+GEMM_TRAFFIC_BYTES = 87.85e6 + 292.76e6
+GEMM_TRAFFIC_SRC_SHA = "6c187c6de44d0cf0"
 GEMM_SOURCES = ("gemm.cu", "gemm.h", "ptx.cuh")
 
 
