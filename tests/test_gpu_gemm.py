@@ -187,3 +187,28 @@ def test_grouped_bad_offsets_rejected_on_device():
     offs = torch.tensor([0, 128, 512], dtype=torch.int32, device=DEV)   # beyond A's rows
     nb.nvfp4_grouped_gemm(offs, rows, qa, qw, gws, n, out=out)
     assert nb.nvfp4_check_status() == 3
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 2048, 5120), (100, 4096, 1024), (128, 256, 2048), (1, 512, 256)])
+def test_split_k_against_oracle_and_unsplit(m, n, k):
+    """Small-M GEMMs split K across SMs when the workspace holds the FP32
+    slices: within tolerance of the oracle, deterministic across calls, and
+    within tolerance of the unsplit kernel (a 256-byte workspace turns the
+    split off)."""
+    a = _rand(m, k, m + n + k)
+    w = _rand(n, k, 3 * m + n, 0.05)
+    qa, ra = _quant_both(a, "split A")
+    qw, rw = _quant_both(w, "split W")
+    big = nb.Workspace(DEV, 64 << 20)
+    small = nb.Workspace(DEV, 256)
+    d1 = nb.nvfp4_gemm(qa, qw, workspace=big)
+    d2 = nb.nvfp4_gemm(qa, qw, workspace=big)
+    d0 = nb.nvfp4_gemm(qa, qw, workspace=small)
+    torch.cuda.synchronize()
+    assert nb.nvfp4_check_status(big) == 0 and nb.nvfp4_check_status(small) == 0
+    assert torch.equal(d1, d2)                                   # split order fixed
+    ii, jj = np.meshgrid(np.arange(m), np.arange(n), indexing="ij")
+    ref, ab = oracle.gemm_ref(ra, rw, ii.ravel(), jj.ravel())
+    tol = gemm_tolerance(ref, ab)
+    for d in (d1, d0):
+        assert np.all(np.abs(bf16_to_f64(d).ravel() - ref) <= tol)
