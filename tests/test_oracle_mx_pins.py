@@ -114,3 +114,63 @@ def test_gemm_reference_against_exact_integers():
             tot += ia * iw * 2 ** (sa + sw + 300)       # shift to keep integers
         assert ref[t] == tot / 4 / 2.0 ** 300
         assert ab[t] >= abs(ref[t])
+
+
+def test_shared_exponent_closed_form_and_clamps():
+    """X = floor(log2 amax) - 2 for every finite amax, computed here from the
+    float's own bit pattern (not frexp), then clamped to [-127, 127]; an
+    all-zero block takes -127."""
+    rng = np.random.default_rng(9)
+    bits = rng.integers(1, 0x7F800000, 4000, dtype=np.int64).astype(np.uint32)
+    extra = np.array([1, 2, 0x007FFFFF, 0x00800000, 0x40800000, 0x40C00000, 0x407FFFFF,
+                      0x7F7FFFFF, 0x3F800000], np.uint32)      # subnormals, 4, 6, <4, max, 1
+    for b in np.concatenate([bits, extra]):
+        v = float(np.uint32(b).view(np.float32))
+        e = int(b) >> 23
+        if e == 0:                                    # subnormal: 2^-149 * mantissa
+            fl = int(b).bit_length() - 1 - 149
+        else:
+            fl = e - 127
+        want = max(-127, min(127, fl - 2))
+        assert oracle.mx_exponent(v) == want, hex(int(b))
+    assert oracle.mx_exponent(0.0) == -127
+    assert oracle.mx_exponent(6.0) == 0 and oracle.mx_exponent(4.0) == 0
+    assert oracle.mx_exponent(3.999) == -1 and oracle.mx_exponent(8.0) == 1
+
+
+def test_scale_layouts_cover_every_byte_once():
+    """Linear: row-major over cols/32 scale columns.  Swizzled: the same
+    128x4 tiling as the NVFP4 layout, taken over cols/32 scale columns, so
+    each position equals the NVFP4 offset of a tensor with half the columns;
+    rows pad to 128 and scale columns to 4, every padded position is hit
+    exactly once."""
+    for rows, cols in [(1, 32), (130, 96), (256, 1024), (300, 32 * 9)]:
+        s = cols // 32
+        assert oracle.mx_scales_bytes(rows, cols, oracle.SF_LINEAR) == rows * s
+        for r in range(rows):
+            for c in range(s):
+                assert oracle.mx_sf_offset(r, c, cols, oracle.SF_LINEAR) == r * s + c
+        rp, sp = (rows + 127) // 128 * 128, (s + 3) // 4 * 4
+        assert oracle.mx_scales_bytes(rows, cols, oracle.SF_SWIZZLED) == rp * sp
+        offs = [oracle.mx_sf_offset(r, c, cols, oracle.SF_SWIZZLED) for r in range(rp) for c in range(sp)]
+        assert sorted(offs) == list(range(rp * sp))
+        for r in range(0, rp, 7):
+            for c in range(sp):
+                assert (oracle.mx_sf_offset(r, c, cols, oracle.SF_SWIZZLED)
+                        == oracle.sf_offset(r, c, rows, cols // 2, oracle.SF_SWIZZLED))
+
+
+def test_dequantize_is_code_times_power_of_two():
+    """Every stored value decodes to sign * grid[code] * 2^(byte - 127),
+    rounded to BF16 (exact here: the products are short binary fractions),
+    in both scale layouts."""
+    x = _rand(130, 96, 10)
+    for layout in (oracle.SF_LINEAR, oracle.SF_SWIZZLED):
+        _, q = oracle.quantize_mx(x, layout)
+        y = oracle.bf16_to_f32(q.dequantize()).astype(np.float64)
+        nib = _nibbles(q)
+        for r in range(0, 130, 3):
+            for c in range(96):
+                byte = int(q.scales[oracle.mx_sf_offset(r, c // 32, 96, layout)])
+                v = GRID[nib[r, c] & 7] * (-1.0 if nib[r, c] & 8 else 1.0) * 2.0 ** (byte - 127)
+                assert y[r, c] == v
