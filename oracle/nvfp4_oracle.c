@@ -59,6 +59,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define NVO_OK 0
@@ -930,5 +931,83 @@ int nvo_quantize_swiglu(const uint16_t *gu, int64_t rows, int64_t inter, int64_t
                 cb[i] = (uint8_t)(c0 | (c1 << 4));
             }
         }
+    return NVO_OK;
+}
+
+/* ------------------------------------------------------- attention read */
+
+/* [PC] One decode step of attention over an NVFP4 KV cache (the KV page:
+ * every generated token re-reads the cache, and the FP4 values are
+ * restored to higher precision before the attention arithmetic).
+ * READINGS: K and V are NVFP4 tensors [tokens x heads_kv * head_dim] (one
+ * row per cached token, head h in columns h*head_dim .. +head_dim-1,
+ * blocks of 16 along head_dim) with tensor scales gk, gv; query head h
+ * (BF16 row h of q, pitch ldq) attends with KV head h / (heads_q /
+ * heads_kv) (grouped-query attention); the restored values are the exact
+ * reals e2m1 * s_b / g (no intermediate FP8 rounding); the scores are
+ * scale * q . k and the weights their softmax over all tokens.  Computed in
+ * FP64 with the maximum score subtracted before exp, for the query heads
+ * h_begin <= h < h_end (rows h - h_begin of the outputs):
+ *   o[h][d]      = sum_t p_t v[t][d] / sum_t p_t
+ *   abs_o[h][d]  = sum_t p_t |v[t][d]| / sum_t p_t   (for the tolerance)
+ *   score_abs[h] = max_t |scale| * sum_d |q_d k[t][d]| (for the tolerance)
+ * tokens == 0 gives o = abs_o = 0.  Returns NVO_ERR_SHAPE for a head count
+ * that does not divide, head_dim % 16 != 0 or a bad size or head range. */
+int nvo_attention_decode(const uint16_t *q, int64_t ldq, int64_t heads_q, const uint8_t *kc,
+                         const uint8_t *ks, float gk, const uint8_t *vc, const uint8_t *vs,
+                         float gv, int layout, int64_t tokens, int64_t heads_kv, int64_t head_dim,
+                         double scale, int64_t h_begin, int64_t h_end, double *o, double *abs_o,
+                         double *score_abs)
+{
+    if (heads_kv <= 0 || heads_q <= 0 || heads_q % heads_kv != 0 || head_dim <= 0 ||
+        head_dim % 16 != 0 || tokens < 0 || h_begin < 0 || h_end > heads_q || h_begin > h_end)
+        return NVO_ERR_SHAPE;
+    const int64_t group = heads_q / heads_kv, cols = heads_kv * head_dim;
+    double *p = (double *)malloc((size_t)(tokens + 1) * sizeof(double));
+    double *num = (double *)malloc((size_t)head_dim * 2 * sizeof(double));
+    if (p == NULL || num == NULL) {
+        free(p);
+        free(num);
+        return NVO_ERR_SHAPE;
+    }
+    double *anum = num + head_dim;
+    for (int64_t h = h_begin; h < h_end; ++h) {
+        const int64_t c0 = (h / group) * head_dim, row = h - h_begin;
+        double mx = -INFINITY, amax = 0.0;
+        for (int64_t t = 0; t < tokens; ++t) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t d = 0; d < head_dim; ++d) {
+                double qd = (double)nvo_bf16_to_f32(q[h * ldq + d]);
+                double kd = elem_f64(kc, ks, layout, (double)gk, tokens, cols, t, c0 + d);
+                acc += qd * kd;
+                aacc += fabs(qd * kd);
+            }
+            p[t] = scale * acc;
+            if (p[t] > mx)
+                mx = p[t];
+            if (fabs(scale) * aacc > amax)
+                amax = fabs(scale) * aacc;
+        }
+        score_abs[row] = amax;
+        double den = 0.0;
+        for (int64_t t = 0; t < tokens; ++t) {
+            p[t] = exp(p[t] - mx);
+            den += p[t];
+        }
+        for (int64_t d = 0; d < head_dim; ++d)
+            num[d] = anum[d] = 0.0;
+        for (int64_t t = 0; t < tokens; ++t)
+            for (int64_t d = 0; d < head_dim; ++d) {
+                double vd = elem_f64(vc, vs, layout, (double)gv, tokens, cols, t, c0 + d);
+                num[d] += p[t] * vd;
+                anum[d] += p[t] * fabs(vd);
+            }
+        for (int64_t d = 0; d < head_dim; ++d) {
+            o[row * head_dim + d] = tokens > 0 ? num[d] / den : 0.0;
+            abs_o[row * head_dim + d] = tokens > 0 ? anum[d] / den : 0.0;
+        }
+    }
+    free(p);
+    free(num);
     return NVO_OK;
 }

@@ -21,7 +21,7 @@ __all__ = [
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
     "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
     "dequantize_mx", "gemm_ref_mx", "QuantizedMX", "moe_combine", "dequantize_fp8",
-    "exp_ref", "swiglu", "quantize_swiglu",
+    "exp_ref", "swiglu", "quantize_swiglu", "attention_decode",
 ]
 
 SF_SWIZZLED, SF_LINEAR = 0, 1
@@ -66,6 +66,9 @@ def lib() -> C.CDLL:
             "nvo_ue8m0_decode": (C.c_double, [C.c_uint8]),
             "nvo_moe_combine": (None, [_p, _i64, _p, _p, _i64, _i64, _i64, _p, _i64]),
             "nvo_exp_ref": (C.c_float, [C.c_float]),
+            "nvo_attention_decode": (C.c_int, [_p, _i64, _i64, _p, _p, C.c_float, _p, _p, C.c_float,
+                                               C.c_int, _i64, _i64, _i64, C.c_double, _i64, _i64,
+                                               _p, _p, _p]),
             "nvo_swiglu": (C.c_float, [C.c_float, C.c_float]),
             "nvo_quantize_swiglu": (C.c_int, [_p, _i64, _i64, _i64, _p, _p, C.c_int,
                                               C.POINTER(C.c_float)]),
@@ -391,3 +394,26 @@ def quantize_swiglu(gu, layout: int = SF_SWIZZLED) -> tuple[int, Quantized]:
 
 if os.environ.get("NVFP4_ORACLE_EAGER_BUILD"):
     lib()
+
+
+def attention_decode(q, k: Quantized, v: Quantized, heads_kv: int, scale: float,
+                     heads=None):
+    """One decode step of grouped-query attention over NVFP4 K and V
+    [tokens x heads_kv * head_dim] in FP64 on the exact restored values.
+    q: BF16 [heads_q x head_dim].  `heads` = (begin, end) limits the query
+    heads computed (default all).  Returns (status, o, abs_o, score_abs):
+    o and abs_o [end - begin x head_dim] float64, score_abs [end - begin]."""
+    qb = bf16_bits(q)
+    heads_q, head_dim = qb.shape
+    assert k.layout == v.layout and k.rows == v.rows and k.cols == v.cols
+    h0, h1 = (0, heads_q) if heads is None else heads
+    n = max(h1 - h0, 0)
+    o = np.zeros((n, head_dim), np.float64)
+    ao = np.zeros((n, head_dim), np.float64)
+    sa = np.zeros(max(n, 1), np.float64)
+    kc, ks = np.ascontiguousarray(k.codes), np.ascontiguousarray(k.scales)
+    vc, vs = np.ascontiguousarray(v.codes), np.ascontiguousarray(v.scales)
+    st = lib().nvo_attention_decode(_ptr(qb), head_dim, heads_q, _ptr(kc), _ptr(ks), float(np.float32(k.g)),
+                                    _ptr(vc), _ptr(vs), float(np.float32(v.g)), k.layout, k.rows,
+                                    heads_kv, head_dim, float(scale), h0, h1, _ptr(o), _ptr(ao), _ptr(sa))
+    return st, o, ao, sa[:n]
