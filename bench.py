@@ -41,6 +41,8 @@ L2_FLUSH_BYTES = 256 << 20
 QUANT_BYTES_PER_VALUE_2PASS = 4.5625
 ENCODE_BYTES_PER_VALUE = 2.5625
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
+ATTN_FP32_LANES = 148 * 128  # FP32 FMA lanes of a B200 (148 SMs x 128)
+SM_MAX_MHZ = 1965           # clocks.max.sm of the B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
 # the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
 # Reported only while the kernel's sources hash to the profiled version.
@@ -707,6 +709,52 @@ def workload_line(name, args, device):
                                   "fp8_frac": fbytes / fms / 1e6 / hbm_gbs,
                                   "peak_source": f"{peak_src} hbm_gbs"}})
         return line
+    if name == "attention":
+        # One decode step read straight from the NVFP4 KV cache: 32 layers,
+        # each K and V [131072 tokens x 8 KV heads x 128] (the KV workload),
+        # 64 query heads (8 per KV head).  The cache (4.8 GB) is far larger
+        # than L2, so no flush is needed between steps.
+        T, H = inputs.KV_TOKENS, inputs.KV_HEADS
+        layers = []
+        for layer in range(inputs.KV_LAYERS):
+            kq = []
+            for kv in (0, 1):
+                x = inputs.kv_tensor(layer, kv, device=device).view(T, -1)
+                kq.append(nb.nvfp4_quantize(x, layout=nb.SF_LINEAR, workspace=ws))
+                del x
+            layers.append((inputs.kv_query(layer, device=device), kq[0], kq[1]))
+        heads_q = inputs.KV_QUERY_HEADS
+        aws = nb.Workspace(device, nb.nvfp4_workspace_bytes(nb.OP_ATTENTION, T, heads_q, H))
+        outs = [torch.empty((heads_q, 128), dtype=torch.bfloat16, device=device) for _ in layers]
+
+        def step():
+            for (qq, kk, vv), o in zip(layers, outs):
+                nb.nvfp4_attention_decode(qq, kk, vv, H, out=o, workspace=aws)
+
+        ms = _timed(step, args.steps, args.warmup)
+        one = _timed(lambda: nb.nvfp4_attention_decode(layers[0][0], layers[0][1], layers[0][2], H,
+                                                       out=outs[0], workspace=aws),
+                     args.steps, args.warmup, flush)
+        st = nb.nvfp4_check_status(ws)
+        cache_bytes = inputs.KV_LAYERS * 2 * T * H * 128 * 0.5625
+        gbs = cache_bytes / ms / 1e6
+        flops_layer = 4.0 * heads_q * T * 128            # scores and weighted sum, 2 flops per MAC
+        alu_peak = ATTN_FP32_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
+        achieved = flops_layer / one / 1e9
+        line.update({"metric": "NVFP4 KV-cache decode attention GB/s of cache read (32 layers x K,V, "
+                               "128K tokens, 64 query / 8 KV heads)",
+                     "value": gbs, "unit": "GB/s", "higher_is_better": True, "ms_per_step": ms,
+                     "config": {"workload": "attention decode 32 x {K,V} x [131072 x 8 x 128], 64 query heads",
+                                "l2": "inputs (4.8 GB cache) larger than L2; one-layer timing flushed"},
+                     "tokens_per_s": 1e3 / ms, "ms_per_layer": one, "status": st,
+                     "hbm_frac": gbs / hbm_gbs,
+                     "roofline": {"kernel": "k_attn_partial + k_attn_combine (one layer)", "bound": "alu",
+                                  "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                                  "frac": achieved / alu_peak,
+                                  "algorithmic_flops_per_launch": flops_layer,
+                                  "peak_source": "148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz",
+                                  "hbm_frac_per_layer": T * H * 128 * 2 * 0.5625 / one / 1e6 / hbm_gbs}})
+        return line
     raise ValueError(name)
 
 
@@ -724,7 +772,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--workload", default="ffn8192",
-                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4", "consumers"],
+                    choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4", "consumers",
+                             "attention"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")

@@ -89,7 +89,8 @@ typedef enum {
     NVFP4_OP_DEQUANTIZE = 1,
     NVFP4_OP_GEMM = 2,
     NVFP4_OP_GROUPED_GEMM = 3,
-    NVFP4_OP_QUANTIZE_GATHER = 4
+    NVFP4_OP_QUANTIZE_GATHER = 4,
+    NVFP4_OP_ATTENTION = 5          /* a = tokens, b = query heads, c = KV heads */
 } nvfp4_op;
 
 /* ---- sizes ------------------------------------------------------------ */
@@ -279,6 +280,35 @@ NVFP4_API nvfp4_status nvfp4_quantize_swiglu(const void *gate_up, int64_t ld, co
  * smallest E4M3 subnormal become signed zeros. */
 NVFP4_API nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int64_t ld,
                                             float *d_fp8_scale, void *stream);
+
+/* Decode attention read straight from an NVFP4 KV cache ("FP4 KV-cache
+ * quantization": each decode step re-reads the whole cache; the FP4 values
+ * are restored before the attention arithmetic).  One query token,
+ * grouped-query attention: query head h (BF16 row h of q, 128 values,
+ * pitch ldq elements) attends with KV head h / (heads_q / heads_kv) over
+ * all K->rows cached tokens:
+ *   s_t = scale * q_h . k_t,  p = softmax(s),  o_h = sum_t p_t v_t
+ * with k, v the exact restored values e2m1(code) * s_b / g (no FP8 or BF16
+ * copy of the cache is made; the values are restored in registers).
+ * K, V  : NVFP4 [tokens x heads_kv * 128], LINEAR scale layout (the KV
+ *         cache layout of nvfp4_quantize), equal shapes; head j of a token
+ *         in columns 128j .. 128j + 127.
+ * heads_q: a multiple of heads_kv with heads_q / heads_kv <= 8.
+ * o     : BF16 [heads_q x 128], pitch ldo elements (round to nearest even of
+ *         the FP32 result).  tokens == 0 gives o = 0.
+ * q 4-byte aligned with even ldq; o 2-byte aligned.  Workspace:
+ *   nvfp4_workspace_bytes(NVFP4_OP_ATTENTION, tokens, heads_q, heads_kv, 0)
+ *   (per chunk of tokens and query head: the running maximum, the weight sum
+ *   and the 128 unnormalised outputs in FP32).
+ * Arithmetic: FP32 (scores in log2 units with scale * log2(e) / g_K folded
+ *   into the query, exp2, an online softmax over token chunks merged in
+ *   chunk order), deterministic for given sizes.  Non-finite q or scale
+ *   bytes give unspecified (NaN) outputs; no status is recorded. */
+NVFP4_API nvfp4_status nvfp4_attention_decode(const void *q, int64_t ldq, int32_t heads_q,
+                                              const nvfp4_tensor *K, const nvfp4_tensor *V,
+                                              int32_t heads_kv, float scale, void *o, int64_t ldo,
+                                              void *workspace, size_t workspace_bytes,
+                                              void *stream);
 
 /* ---- MXFP4 ------------------------------------------------------------ */
 /* MXFP4, the format the pages compare NVFP4 with ("NVIDIA shrank GLM-5.2 to

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libnvfp4.so")
 SF_SWIZZLED = 0
 SF_LINEAR = 1
 
-OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_GROUPED_GEMM, OP_QUANTIZE_GATHER = range(5)
+OP_QUANTIZE, OP_DEQUANTIZE, OP_GEMM, OP_GROUPED_GEMM, OP_QUANTIZE_GATHER, OP_ATTENTION = range(6)
 
 STATUS_NAMES = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_ALIGNMENT", 3: "NVFP4_ERR_SHAPE",
@@ -37,6 +37,7 @@ EXPORTED = (
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
     "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
     "nvfp4_gemm_mx", "nvfp4_moe_combine", "nvfp4_dequantize_fp8", "nvfp4_quantize_swiglu",
+    "nvfp4_attention_decode",
 )
 
 
@@ -94,6 +95,8 @@ def lib() -> C.CDLL:
             "nvfp4_moe_combine": (C.c_int, [vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp]),
             "nvfp4_dequantize_fp8": (C.c_int, [T, vp, i64, vp, vp]),
             "nvfp4_quantize_swiglu": (C.c_int, [vp, i64, T, vp, sz, vp]),
+            "nvfp4_attention_decode": (C.c_int, [vp, i64, i32, T, T, i32, C.c_float, vp, i64, vp, sz,
+                                                 vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -361,6 +364,30 @@ def nvfp4_dequantize_fp8(t: NVFP4Tensor, out: torch.Tensor | None = None, scale:
     _check(lib().nvfp4_dequantize_fp8(C.byref(ct), out.data_ptr(), out.stride(0), scale.data_ptr(),
                                       _stream(stream)), "nvfp4_dequantize_fp8")
     return out, scale
+
+
+def nvfp4_attention_decode(q: torch.Tensor, k: NVFP4Tensor, v: NVFP4Tensor, heads_kv: int,
+                           scale: float | None = None, out: torch.Tensor | None = None,
+                           workspace: Workspace | None = None, stream=None) -> torch.Tensor:
+    """One decode step of grouped-query attention read straight from an
+    NVFP4 KV cache: q BF16 [heads_q x 128]; k, v NVFP4 [tokens x heads_kv *
+    128] in the linear scale layout.  Returns BF16 [heads_q x 128].  The
+    softmax scale defaults to 1 / sqrt(128)."""
+    assert q.dtype == torch.bfloat16 and q.dim() == 2 and q.stride(1) == 1
+    heads_q = q.shape[0]
+    if scale is None:
+        scale = 128 ** -0.5
+    if out is None:
+        out = torch.empty((heads_q, 128), dtype=torch.bfloat16, device=q.device)
+    need = nvfp4_workspace_bytes(OP_ATTENTION, k.rows, heads_q, heads_kv)
+    ws = workspace or default_workspace(q.device)
+    if ws.nbytes < need:
+        ws = Workspace(q.device, need)
+    tk, tv = k.c_struct(), v.c_struct()
+    _check(lib().nvfp4_attention_decode(q.data_ptr(), q.stride(0), heads_q, C.byref(tk), C.byref(tv),
+                                        heads_kv, float(scale), out.data_ptr(), out.stride(0), ws.ptr,
+                                        ws.nbytes, _stream(stream)), "nvfp4_attention_decode")
+    return out
 
 
 def nvfp4_quantize_swiglu(gate_up: torch.Tensor, out: NVFP4Tensor | None = None,

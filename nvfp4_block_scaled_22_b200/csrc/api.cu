@@ -262,6 +262,20 @@ nvfp4_status check_transposed(const void *x, int64_t ld, const nvfp4_tensor *out
 
 extern "C" {
 
+// Token chunks of the attention read: about one CTA per SM of a B200 (148
+// SMs) over all KV heads, at least one 256-token sub-tile per chunk.  Fixed
+// by the sizes alone, so the workspace size and the summation order do not
+// depend on the device.
+static int64_t attn_chunk_tokens(int64_t tokens, int64_t heads_kv) {
+    const int64_t subs = ceil_div(tokens, kAttnSub);
+    const int64_t want = std::max<int64_t>(1, std::min<int64_t>(subs, 148 / heads_kv));
+    return ceil_div(subs, want) * kAttnSub;
+}
+
+static int64_t attn_chunks(int64_t tokens, int64_t heads_kv) {
+    return tokens > 0 ? ceil_div(tokens, attn_chunk_tokens(tokens, heads_kv)) : 0;
+}
+
 size_t nvfp4_codes_bytes(int64_t rows, int64_t cols) {
     if (rows < 0 || cols < 0) return 0;
     return (size_t)(rows * (cols / 2));
@@ -284,6 +298,11 @@ size_t nvfp4_workspace_bytes(int32_t op, int64_t m, int64_t n, int64_t k, int32_
             // slices; a smaller workspace only turns the split off
             if (groups == 0 && m > 0 && n > 0 && k > 0 && m <= kBM)
                 return kStatusBytes + (size_t)std::min<int64_t>(8, ceil_div(k / 64, 4)) * m * n * 4;
+            return kStatusBytes;
+        case NVFP4_OP_ATTENTION:
+            // m = tokens, n = query heads, k = KV heads
+            if (m > 0 && n > 0 && k > 0)
+                return kStatusBytes + (size_t)attn_chunks(m, k) * n * (kAttnDim + 2) * 4;
             return kStatusBytes;
         default:
             return kStatusBytes;
@@ -593,6 +612,63 @@ nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int64_t ld, f
     const int64_t blocks = in->rows * (in->cols / 16);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(blocks, 256), 8LL * sms));
     k_dequantize_fp8<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_attention_decode(const void *q, int64_t ldq, int32_t heads_q,
+                                    const nvfp4_tensor *K, const nvfp4_tensor *V, int32_t heads_kv,
+                                    float scale, void *o, int64_t ldo, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    nvfp4_status st = check_tensor(K);
+    if (st != NVFP4_OK) return st;
+    st = check_tensor(V);
+    if (st != NVFP4_OK) return st;
+    if (heads_q < 1 || heads_kv < 1 || !(scale == scale) || scale > 3.4e38f || scale < -3.4e38f)
+        return NVFP4_ERR_INVALID_ARG;
+    if (heads_q % heads_kv != 0 || heads_q / heads_kv > kAttnMaxGroup) return NVFP4_ERR_SHAPE;
+    if (K->sf_layout != NVFP4_SF_LINEAR || V->sf_layout != NVFP4_SF_LINEAR) return NVFP4_ERR_SHAPE;
+    if (K->rows != V->rows || K->cols != V->cols || K->cols != (int64_t)heads_kv * kAttnDim)
+        return NVFP4_ERR_SHAPE;
+    if (q == nullptr || o == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0 || ldq % 2 != 0 ||
+        (reinterpret_cast<uintptr_t>(o) & 1u) != 0)
+        return NVFP4_ERR_ALIGNMENT;
+    if (ldq < kAttnDim || ldo < kAttnDim) return NVFP4_ERR_SHAPE;
+    const int64_t tokens = K->rows;
+    const int64_t chunks = attn_chunks(tokens, heads_kv);
+    st = check_workspace(workspace, workspace_bytes,
+                         kStatusBytes + (size_t)chunks * heads_q * (kAttnDim + 2) * 4);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    AttnParams p;
+    p.q = static_cast<const uint16_t *>(q);
+    p.ldq = ldq;
+    p.kc = static_cast<const uint8_t *>(K->codes);
+    p.ks = static_cast<const uint8_t *>(K->scales);
+    p.vc = static_cast<const uint8_t *>(V->codes);
+    p.vs = static_cast<const uint8_t *>(V->scales);
+    p.gk = K->global;
+    p.gv = V->global;
+    p.tokens = tokens;
+    p.cols = K->cols;
+    p.heads_kv = heads_kv;
+    p.group = heads_q / heads_kv;
+    p.scale = scale;
+    p.chunk = tokens > 0 ? attn_chunk_tokens(tokens, heads_kv) : kAttnSub;
+    p.n_chunks = (int32_t)chunks;
+    p.part_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    p.part_ml = p.part_o + chunks * heads_q * kAttnDim;
+    p.o = static_cast<uint16_t *>(o);
+    p.ldo = ldo;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (chunks > 0) {
+        k_attn_partial<<<dim3((unsigned)chunks, (unsigned)heads_kv), kAttnThreads, 0, s>>>(p);
+        st = launched(cudaGetLastError());
+        if (st != NVFP4_OK) return st;
+    }
+    k_attn_combine<<<(unsigned)heads_q, kAttnDim, 0, s>>>(p);
     return launched(cudaGetLastError());
 }
 

@@ -147,4 +147,33 @@ __global__ void k_dequantize_mx(DequantParams p);
 __global__ void k_dequantize(DequantParams p);
 __global__ void k_dequantize_narrow(DequantParams p);
 
+// Decode attention over an NVFP4 KV cache: one query token, grouped query
+// heads, head_dim 128, K and V [tokens x heads_kv * 128] in the linear
+// scale layout.  Pass 1 (grid chunks x heads_kv, kAttnThreads threads):
+// per chunk of tokens and KV head, the running score maximum m, the weight
+// sum l and the unnormalised output O of each of the group's query heads.
+// Pass 2 (grid heads_q, 128 threads): merge the chunks, o = O / l / g_V.
+constexpr int kAttnDim = 128;        // head_dim
+constexpr int kAttnMaxGroup = 8;     // query heads per KV head
+constexpr int kAttnThreads = 256;
+constexpr int kAttnSub = 256;        // tokens per sub-tile (one per thread)
+struct AttnParams {
+    const uint16_t *q;               // BF16 [heads_q x 128], pitch ldq
+    int64_t ldq;
+    const uint8_t *kc, *ks;          // K codes [tokens x cols/2], scales [tokens x cols/16]
+    const uint8_t *vc, *vs;
+    const float *gk, *gv;            // tensor scales
+    int64_t tokens, cols;            // cols = heads_kv * 128
+    int32_t heads_kv, group;         // heads_q = group * heads_kv
+    float scale;                     // softmax scale
+    int64_t chunk;                   // tokens per pass-1 CTA, a multiple of kAttnSub
+    int32_t n_chunks;
+    float *part_o;                   // [n_chunks][heads_q][128]
+    float *part_ml;                  // [n_chunks][heads_q][2]: m (log2 units), l
+    uint16_t *o;                     // BF16 [heads_q x 128], pitch ldo
+    int64_t ldo;
+};
+__global__ void k_attn_partial(AttnParams p);
+__global__ void k_attn_combine(AttnParams p);
+
 }  // namespace nvfp4

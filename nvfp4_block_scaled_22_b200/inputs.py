@@ -239,6 +239,15 @@ def kv_tensor(layer: int, kv: int, device="cpu", tokens: int = KV_TOKENS) -> tor
     return x.view(tokens, KV_HEADS, KV_HEAD_DIM).to(torch.bfloat16)
 
 
+KV_QUERY_HEADS = 64        # grouped-query attention: 8 query heads per KV head
+
+
+def kv_query(layer: int, device="cpu", heads_q: int = KV_QUERY_HEADS) -> torch.Tensor:
+    """Query of one decode step for layer ``layer``: BF16 [heads_q x head_dim], N(0,1)."""
+    g = _gen("kv", 1000 + layer, device)
+    return _randn((heads_q, KV_HEAD_DIM), g, device).to(torch.bfloat16)
+
+
 # --------------------------------------------------------------------------
 # wgrad: inputs of the weight-gradient GEMM dW = dY^T X of the FFN linear
 # --------------------------------------------------------------------------

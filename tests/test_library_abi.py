@@ -90,3 +90,28 @@ def test_host_side_argument_errors_need_no_gpu(lib):
     a = binding.CTensor(16, 16, 16, 128, 96, 0)      # K % 64 != 0
     w = binding.CTensor(16, 16, 16, 256, 96, 0)
     assert lib.nvfp4_gemm(a, w, 16, 256, 16, 1 << 16, 0) == 3
+
+
+def test_attention_argument_errors_and_workspace_size(lib):
+    """Host checks of the attention read return before any CUDA call; the
+    workspace holds per chunk and query head the 128 outputs, m and l."""
+    k = binding.CTensor(16, 16, 16, 1000, 1024, 1)      # 8 KV heads x 128, linear
+    ws = 1 << 20
+    assert lib.nvfp4_attention_decode(16, 128, 64, k, k, 8, 0.1, 16, 128, 16, ws, 0) != 3
+    assert lib.nvfp4_attention_decode(16, 128, 60, k, k, 8, 0.1, 16, 128, 16, ws, 0) == 3  # heads
+    assert lib.nvfp4_attention_decode(16, 128, 72, k, k, 8, 0.1, 16, 128, 16, ws, 0) == 3  # group 9
+    assert lib.nvfp4_attention_decode(16, 128, 64, k, k, 4, 0.1, 16, 128, 16, ws, 0) == 3  # cols
+    sw = binding.CTensor(16, 16, 16, 1000, 1024, 0)      # swizzled scales
+    assert lib.nvfp4_attention_decode(16, 128, 64, sw, sw, 8, 0.1, 16, 128, 16, ws, 0) == 3
+    v = binding.CTensor(16, 16, 16, 999, 1024, 1)
+    assert lib.nvfp4_attention_decode(16, 128, 64, k, v, 8, 0.1, 16, 128, 16, ws, 0) == 3  # rows
+    assert lib.nvfp4_attention_decode(18, 128, 64, k, k, 8, 0.1, 16, 128, 16, ws, 0) == 2  # q align
+    assert lib.nvfp4_attention_decode(16, 129, 64, k, k, 8, 0.1, 16, 128, 16, ws, 0) == 2  # odd ldq
+    assert lib.nvfp4_attention_decode(16, 128, 64, k, k, 8, float("nan"), 16, 128, 16, ws, 0) == 1
+    assert lib.nvfp4_attention_decode(16, 128, 64, k, k, 8, 0.1, 16, 128, 16, 300, 0) == 6  # ws
+    # 131072 tokens, 8 KV heads: 18 chunks of 7424 tokens; 64 query heads
+    need = binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, 131072, 64, 8)
+    assert need == 256 + 18 * 64 * 130 * 4
+    assert binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, 0, 64, 8) == 256
+    # one KV head: up to 148 chunks, never more chunks than 256-token sub-tiles
+    assert binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, 1000, 2, 1) == 256 + 4 * 2 * 130 * 4
