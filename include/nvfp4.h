@@ -300,10 +300,12 @@ NVFP4_API nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int
  *   nvfp4_workspace_bytes(NVFP4_OP_ATTENTION, tokens, heads_q, heads_kv, 0)
  *   (per chunk of tokens and query head: the running maximum, the weight sum
  *   and the 128 unnormalised outputs in FP32).
- * Arithmetic: FP32 (scores in log2 units with scale * log2(e) / g_K folded
- *   into the query, exp2, an online softmax over token chunks merged in
- *   chunk order), deterministic for given sizes.  Non-finite q or scale
- *   bytes give unspecified (NaN) outputs; no status is recorded. */
+ * Arithmetic: scores q . (e2m1 * s_b) on the tensor cores (BF16 operands,
+ *   both exact; FP32 accumulation) times RN(RN(scale * log2(e)) / g_K), so
+ *   in log2 units; exp2 and an online softmax over token chunks merged in
+ *   chunk order; the weighted V sum in FP32.  Deterministic for given sizes.
+ *   Non-finite q or scale bytes give unspecified (NaN) outputs; no status
+ *   is recorded. */
 NVFP4_API nvfp4_status nvfp4_attention_decode(const void *q, int64_t ldq, int32_t heads_q,
                                               const nvfp4_tensor *K, const nvfp4_tensor *V,
                                               int32_t heads_kv, float scale, void *o, int64_t ldo,

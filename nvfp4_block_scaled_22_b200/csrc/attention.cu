@@ -13,13 +13,19 @@
 // what was summed before (the online softmax of flash-decoding).
 //
 // k_attn_partial, per sub-tile of 256 tokens of the CTA's chunk:
-//   A  thread = token: its 128 K values restored, the 8 head scores by
-//      packed FP32 FMAs against the query in shared memory (every lane reads
-//      the same query word: broadcast); CTA maximum per head -> new running
-//      maximum and rescale factor; weights -> shared memory.
+//   A  scores on the tensor cores (mma.sync m16n8k16, BF16 operands, FP32
+//      accumulation): each warp takes two 16-token tiles; the K values
+//      restored to BF16 (e2m1 * s_b has at most 6 significant bits, so the
+//      restore is exact) are the A operand and the query (BF16, exact) the
+//      B operand, 8 query heads as the 8 columns.  The 128 dims are dealt
+//      to the eight 16-wide k-steps so that each lane's A values come from
+//      one 16-byte piece of the token's code row (lane column pair c holds
+//      dims 32c .. 32c + 31); the query columns follow the same order.
+//      Scores times c, the CTA maximum per head -> new running maximum and
+//      rescale factor; weights -> shared memory.
 //   B  thread = (8 dims, token phase 0..15): the V values of its dims for
 //      every 16th token of the sub-tile times the weights of all 8 heads,
-//      into 64 FP32 accumulators (rescaled first).
+//      into 64 FP32 accumulators (rescaled first, packed FP32 FMAs).
 // After the chunk the token phases are summed in a fixed order (a shuffle,
 // then three halvings through shared memory) and the chunk's O, m and l
 // are written.  k_attn_combine merges the chunks in chunk order:
@@ -56,67 +62,79 @@ __device__ __forceinline__ float2 restore_pair(uint32_t byte, float2 s2) {
     return mul_f32x2(f32x2_from_f16x2(f16x2_from_e2m1x2(byte & 0xFFu)), s2);
 }
 
+// The same two values as BF16 (exact: at most 6 significant bits, within
+// 2^-10 .. 2688), low nibble in the low half.
+__device__ __forceinline__ uint32_t restore_bf16x2(uint32_t byte, float s) {
+    const float2 v = f32x2_from_f16x2(f16x2_from_e2m1x2(byte & 0xFFu));
+    return bf16x2_from_f32(__fmul_rn(v.x, s), __fmul_rn(v.y, s));
+}
+
+// D += A B for one 16x8x16 tile: A 16x16 row-major, B 16x8 column-major,
+// BF16 operands, FP32 accumulators (thread fragments of the PTX mma.sync
+// m16n8k16 shape: a row group g = lane / 4 and a column pair c = lane % 4).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) {
-    // qs[i][hp] = (q[2hp][2i], q[2hp][2i+1], q[2hp+1][2i], q[2hp+1][2i+1]) * c
-    __shared__ float4 qs[kAttnDim / 2][kAttnMaxGroup / 2];
     // ps[t][hp] = (p[2hp], p[2hp], p[2hp+1], p[2hp+1]) of token t of the sub-tile
     __shared__ float4 ps[kAttnSub][kAttnMaxGroup / 2];
     __shared__ float wred[kAttnThreads / 32][kAttnMaxGroup];
     __shared__ float m_sh[kAttnMaxGroup], alpha_sh[kAttnMaxGroup];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, c = lane & 3;    // pass A: MMA fragment row group, column pair
     const int hk = blockIdx.y, G = p.group;
     const int heads_q = p.group * p.heads_kv;
     const int64_t t0 = (int64_t)blockIdx.x * p.chunk;
     const int64_t t1 = min(p.tokens, t0 + p.chunk);
     const int64_t row_codes = p.cols / 2, row_scales = p.cols / 16;
+    const float ck = __fdiv_rn(__fmul_rn(p.scale, kLog2e), *p.gk);
 
-    {
-        const float c = __fdiv_rn(__fmul_rn(p.scale, kLog2e), *p.gk);
-        float *qf = reinterpret_cast<float *>(&qs[0][0]);
-        for (int e = tid; e < (kAttnDim / 2) * kAttnMaxGroup; e += kAttnThreads) {
-            const int i = e >> 3, h = e & 7;     // float pair e: dims 2i, 2i + 1 of head h
-            float lo = 0.0f, hi = 0.0f;
-            if (h < G) {
-                const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(
-                    p.q + (int64_t)(hk * G + h) * p.ldq + 2 * i));
-                lo = __fmul_rn(__uint_as_float(w << 16), c);
-                hi = __fmul_rn(__uint_as_float(w & 0xFFFF0000u), c);
-            }
-            qf[i * 16 + 2 * h] = lo;
-            qf[i * 16 + 2 * h + 1] = hi;
-        }
-        if (tid < kAttnMaxGroup) m_sh[tid] = neg_inf();
+    // B operand of the score MMAs: query head g, dims 32c .. 32c + 31 as
+    // BF16 pairs; step j uses dims 32c + 4j .. + 3 (qb[2j], qb[2j + 1]).
+    uint32_t qb[16];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) qb[n] = 0u;
+    if (g < G) {
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q + (int64_t)(hk * G + g) * p.ldq + 32 * c);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) qb[n] = __ldg(qrow + n);
     }
+    if (tid < kAttnMaxGroup) m_sh[tid] = neg_inf();
     __syncthreads();
 
-    float lsum[kAttnMaxGroup];
+    float lsum[2] = {0.0f, 0.0f};             // heads 2c, 2c + 1 over this lane's tokens
     float2 oacc[kAttnMaxGroup][4];
 #pragma unroll
-    for (int h = 0; h < kAttnMaxGroup; ++h) {
-        lsum[h] = 0.0f;
+    for (int h = 0; h < kAttnMaxGroup; ++h)
 #pragma unroll
         for (int i = 0; i < 4; ++i) oacc[h][i] = make_float2(0.0f, 0.0f);
-    }
     const int dg = tid & 15, tp = tid >> 4;   // pass B: dims 8dg .. 8dg + 7, token phase
 
-    // K words of the first sub-tile; each later sub-tile's are loaded while
-    // the previous one is in pass B, and a sub-tile's V words while its
-    // scores are computed, so HBM latency overlaps the arithmetic.
+    // Pass A rows of this lane: tokens 32 warp + 16 u + g + 8 r of the
+    // sub-tile (u = MMA tile 0/1, r = fragment row half), code bytes
+    // 16c .. 16c + 15 of the KV head's 64 (dims 32c .. 32c + 31) and the
+    // scales of blocks 2c, 2c + 1.  Loaded one sub-tile ahead.
     uint4 kw[4];
-    uint2 ksw;
+    uint32_t ksw[4];
     auto load_k = [&](int64_t base) {
-        const int64_t t = base + tid;
-        ksw = make_uint2(0u, 0u);
 #pragma unroll
-        for (int n = 0; n < 4; ++n) kw[n] = make_uint4(0u, 0u, 0u, 0u);
-        if (t < t1) {
-            const uint4 *kp = reinterpret_cast<const uint4 *>(p.kc + t * row_codes + hk * 64);
-#pragma unroll
-            for (int n = 0; n < 4; ++n) kw[n] = __ldg(kp + n);
-            ksw = __ldg(reinterpret_cast<const uint2 *>(p.ks + t * row_scales + hk * 8));
+        for (int e = 0; e < 4; ++e) {
+            const int64_t t = base + 32 * warp + 16 * (e >> 1) + g + 8 * (e & 1);
+            kw[e] = make_uint4(0u, 0u, 0u, 0u);
+            ksw[e] = 0u;
+            if (t < t1) {
+                kw[e] = __ldg(reinterpret_cast<const uint4 *>(p.kc + t * row_codes + hk * 64 + 16 * c));
+                ksw[e] = __ldg(reinterpret_cast<const uint16_t *>(p.ks + t * row_scales + hk * 8 + 2 * c));
+            }
         }
     };
     load_k(t0);
@@ -136,38 +154,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
             }
         }
 
-        // ---- A: scores of token base + tid for the 8 heads
-        const bool valid = tid < n_sub;
-        float2 acc[kAttnMaxGroup];
+        // ---- A: scores S[token][head] = sum_d (e2m1 * s_b)[token][d] q[head][d]
+        // on the tensor cores (BF16 operands, both exact; FP32 accumulate):
+        // two 16-token tiles per warp, eight k-steps of 16 dims each.
+        float sc[2][4];
 #pragma unroll
-        for (int h = 0; h < kAttnMaxGroup; ++h) acc[h] = make_float2(0.0f, 0.0f);
+        for (int u = 0; u < 2; ++u) {
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const uint4 w0 = kw[2 * u], w1 = kw[2 * u + 1];          // rows g, g + 8
+            const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {                 // block b: dims 16b .. 16b + 15
-            const float sf = f32_from_e4m3(((b < 4 ? ksw.x : ksw.y) >> (8 * (b & 3))) & 0xFFu);
-            const float2 sf2 = make_float2(sf, sf);
-            const uint32_t w0 = (b & 1) ? kw[b >> 1].z : kw[b >> 1].x;
-            const uint32_t w1 = (b & 1) ? kw[b >> 1].w : kw[b >> 1].y;
+            for (int j = 0; j < 8; ++j) {                            // dims 32c + 4j .. + 3
+                const float s0 = f32_from_e4m3((ksw[2 * u] >> (8 * (j >> 2))) & 0xFFu);
+                const float s1 = f32_from_e4m3((ksw[2 * u + 1] >> (8 * (j >> 2))) & 0xFFu);
+                const uint32_t b0 = r0[j >> 1] >> (16 * (j & 1)), b1 = r1[j >> 1] >> (16 * (j & 1));
+                uint32_t a[4];
+                a[0] = restore_bf16x2(b0, s0);          // row g,     dims +0, +1
+                a[1] = restore_bf16x2(b1, s1);          // row g + 8, dims +0, +1
+                a[2] = restore_bf16x2(b0 >> 8, s0);     // row g,     dims +2, +3
+                a[3] = restore_bf16x2(b1 >> 8, s1);     // row g + 8, dims +2, +3
+                mma_bf16_16816(d, a, qb[2 * j], qb[2 * j + 1]);
+            }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {             // byte j: dims 16b + 2j, 16b + 2j + 1
-                const float2 k2 = restore_pair((j < 4 ? w0 : w1) >> (8 * (j & 3)), sf2);
-                const int i = 8 * b + j;
-#pragma unroll
-                for (int hp = 0; hp < kAttnMaxGroup / 2; ++hp) {
-                    const float4 qq = qs[i][hp];
-                    acc[2 * hp] = fma_f32x2(k2, make_float2(qq.x, qq.y), acc[2 * hp]);
-                    acc[2 * hp + 1] = fma_f32x2(k2, make_float2(qq.z, qq.w), acc[2 * hp + 1]);
-                }
+            for (int e = 0; e < 4; ++e) {    // d: (g, 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1)
+                const int tl = 32 * warp + 16 * u + g + 8 * (e >> 1);
+                sc[u][e] = tl < n_sub ? __fmul_rn(d[e], ck) : neg_inf();
             }
         }
         if (base + kAttnSub < t1) load_k(base + kAttnSub);
-        float s2[kAttnMaxGroup];
 #pragma unroll
-        for (int h = 0; h < kAttnMaxGroup; ++h) {
-            s2[h] = valid ? __fadd_rn(acc[h].x, acc[h].y) : neg_inf();
-            float v = s2[h];
+        for (int e = 0; e < 2; ++e) {        // heads 2c + e
+            float v = fmaxf(fmaxf(sc[0][e], sc[0][e + 2]), fmaxf(sc[1][e], sc[1][e + 2]));
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-            if (lane == 0) wred[warp][h] = v;
+            for (int off = 4; off <= 16; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+            if (g == 0) wred[warp][2 * c + e] = v;
         }
         __syncthreads();
         if (tid < kAttnMaxGroup) {
@@ -180,15 +200,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
             m_sh[tid] = mn;
         }
         __syncthreads();
-        float pv[kAttnMaxGroup];
+        {
+            const float m0 = m_sh[2 * c], m1 = m_sh[2 * c + 1];
+            float l0 = 0.0f, l1 = 0.0f;
 #pragma unroll
-        for (int h = 0; h < kAttnMaxGroup; ++h) {
-            pv[h] = valid ? exp2f(s2[h] - m_sh[h]) : 0.0f;
-            lsum[h] = __fmaf_rn(lsum[h], alpha_sh[h], pv[h]);
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int tl = 32 * warp + 16 * u + g + 8 * r;
+                    const bool ok = tl < n_sub;
+                    const float p0 = ok ? exp2f(sc[u][2 * r] - m0) : 0.0f;
+                    const float p1 = ok ? exp2f(sc[u][2 * r + 1] - m1) : 0.0f;
+                    l0 += p0;
+                    l1 += p1;
+                    ps[tl][c] = make_float4(p0, p0, p1, p1);
+                }
+            lsum[0] = __fmaf_rn(lsum[0], alpha_sh[2 * c], l0);
+            lsum[1] = __fmaf_rn(lsum[1], alpha_sh[2 * c + 1], l1);
         }
-#pragma unroll
-        for (int hp = 0; hp < kAttnMaxGroup / 2; ++hp)
-            ps[tid][hp] = make_float4(pv[2 * hp], pv[2 * hp], pv[2 * hp + 1], pv[2 * hp + 1]);
         __syncthreads();
 
         // ---- B: weighted V of tokens tp, tp + 16, ... of the sub-tile
@@ -219,13 +248,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
         __syncthreads();   // ps and alpha_sh are rewritten by the next sub-tile
     }
 
-    // ---- chunk totals: weight sums per head
+    // ---- chunk totals: weight sums per head (lanes of one column pair c)
 #pragma unroll
-    for (int h = 0; h < kAttnMaxGroup; ++h) {
-        float v = lsum[h];
+    for (int e = 0; e < 2; ++e) {
+        float v = lsum[e];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-        if (lane == 0) wred[warp][h] = v;
+        for (int off = 4; off <= 16; off <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+        if (g == 0) wred[warp][2 * c + e] = v;
     }
     // O: the two token phases of a warp, then warps 4..7 onto 0..3, 2..3
     // onto 0..1, 1 onto 0, through the (now free) weight buffer.

@@ -2,9 +2,12 @@
 the oracle's FP64 attention on the exact restored values.
 
 Tolerance, derived from the kernel's FP32 arithmetic (u = 2^-24):
-  * scores (log2 units): the query times RN(RN(scale * log2 e) / g_K)
-    (3u per term), then two FMA chains of 64 terms and one add: at most
-    68u * log2(e) * score_abs, score_abs = max_t |scale| sum_d |q_d k_td|;
+  * scores (log2 units): exact products of BF16 operands summed in FP32
+    over eight 16-term tensor-core steps, then one multiply by
+    RN(RN(scale * log2 e) / g_K): allowed 68u * log2(e) * score_abs,
+    score_abs = max_t |scale| sum_d |q_d k_td| (more than the eight steps
+    lose even if each step's internal sum is off by 2 ulp of each of its 16
+    products);
   * weights: exp2 of (score - running max), the subtraction (at most
     2u * log2(e) * score_abs) and exp2 itself (2 ulp), and the rescales of
     the chunk merge (2 ulp): relative error eps <= 72u * score_abs + 8u
