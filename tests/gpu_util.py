@@ -41,3 +41,13 @@ def gemm_tolerance(ref: np.ndarray, abs_sum: np.ndarray) -> np.ndarray:
 
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
+
+
+def attention_chunking(tokens: int, heads_kv: int):
+    """Tokens per chunk and chunk count of the attention read (about one CTA
+    per SM of 148 over the KV heads, whole 256-token sub-tiles); the
+    tolerance of the attention parity tests depends on it."""
+    subs = -(-tokens // 256)
+    want = max(1, min(subs, 148 // heads_kv))
+    chunk = -(-subs // want) * 256
+    return chunk, (-(-tokens // chunk) if tokens > 0 else 0)

@@ -30,7 +30,7 @@ import torch
 import oracle
 from nvfp4_block_scaled_22_b200 import binding as nb
 from nvfp4_block_scaled_22_b200 import inputs
-from tests.gpu_util import assert_quantized_equal, bf16_to_f64, bf16_ulp
+from tests.gpu_util import assert_quantized_equal, attention_chunking, bf16_to_f64, bf16_ulp
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -44,17 +44,8 @@ def _lib():
     assert nb.nvfp4_check_status() == 0
 
 
-def _chunking(tokens, heads_kv):
-    """Tokens per chunk and chunk count of the attention read (about one CTA
-    per SM of 148 over the KV heads, whole 256-token sub-tiles)."""
-    subs = -(-tokens // 256)
-    want = max(1, min(subs, 148 // heads_kv))
-    chunk = -(-subs // want) * 256
-    return chunk, -(-tokens // chunk)
-
-
 def _fp32_bound(abs_o, score_abs, tokens, heads_kv):
-    chunk, n_chunks = _chunking(max(tokens, 1), heads_kv)
+    chunk, n_chunks = attention_chunking(max(tokens, 1), heads_kv)
     eps = 72 * U * score_abs[:, None] + 8 * U
     n = chunk / 16 + 2 * chunk / 256 + 8 + n_chunks + 8
     return 2 * (2 * eps + 2 * n * U + 2 * U) * abs_o

@@ -115,3 +115,15 @@ def test_attention_argument_errors_and_workspace_size(lib):
     assert binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, 0, 64, 8) == 256
     # one KV head: up to 148 chunks, never more chunks than 256-token sub-tiles
     assert binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, 1000, 2, 1) == 256 + 4 * 2 * 130 * 4
+
+
+def test_attention_chunking_matches_the_library(lib):
+    """The chunk count the attention parity tolerance assumes is the one
+    the library's workspace size implies."""
+    from tests.gpu_util import attention_chunking
+    for tokens in (1, 255, 256, 257, 1000, 4099, 20000, 131072, 1 << 20):
+        for heads_kv in (1, 2, 3, 8, 37, 200):
+            heads_q = heads_kv * 2
+            ws = binding.nvfp4_workspace_bytes(binding.OP_ATTENTION, tokens, heads_q, heads_kv)
+            n_lib = (ws - 256) // (heads_q * 130 * 4)
+            assert n_lib == attention_chunking(tokens, heads_kv)[1], (tokens, heads_kv)
