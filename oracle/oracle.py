@@ -16,7 +16,8 @@ __all__ = [
     "SF_SWIZZLED", "SF_LINEAR", "OK", "ERR_SHAPE", "ERR_NONFINITE", "ERR_RANGE",
     "lib", "bf16_bits", "bf16_to_f32", "f32_to_bf16", "e2m1_decode", "e2m1_rne",
     "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
-    "global_scale", "quantize", "quantize_with_global", "dequantize", "gemm_ref",
+    "global_scale", "quantize", "quantize_with_global", "quantize_parallel", "dequantize",
+    "gemm_ref",
     "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
     "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
@@ -185,6 +186,64 @@ def quantize(x, layout: int = SF_SWIZZLED) -> tuple[int, Quantized]:
     st = lib().nvo_quantize(_ptr(b), rows, cols, cols, _ptr(codes), _ptr(scales), layout,
                             C.byref(g))
     return st, Quantized(codes, scales, g.value, rows, cols, layout)
+
+
+def _row_ranges(rows: int, threads: int) -> list[tuple[int, int]]:
+    """Disjoint row ranges starting at multiples of 128: a range of the 128x4
+    scale layout then owns one contiguous run of scale bytes, as does a range
+    of the row-major layout."""
+    per = -(-rows // max(1, threads))
+    step = max(128, -(-per // 128) * 128)
+    return [(r, min(rows, r + step)) for r in range(0, rows, step)]
+
+
+def quantize_parallel(x, layout: int = SF_SWIZZLED, threads: int | None = None
+                      ) -> tuple[int, Quantized]:
+    """`quantize` with its row loops spread over host threads (the C calls
+    release the GIL).  The steps are the same calls in the same order of
+    definition: the tensor amax is the maximum of the ranges' exact maxima
+    (a maximum does not depend on grouping), g follows from it once, and
+    every range is encoded by `quantize_with_global` with that g, each
+    writing only its own rows' codes and scale bytes.  Bit-identical to
+    `quantize` by construction; a CPU test checks it."""
+    from concurrent.futures import ThreadPoolExecutor
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    if threads is None:
+        threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros(scales_bytes(rows, cols, layout), np.uint8)
+    if cols % 16 != 0:
+        return ERR_SHAPE, Quantized(codes, scales, 0.0, rows, cols, layout)
+    ranges = _row_ranges(rows, threads)
+    L = lib()
+
+    def amax_of(rr):
+        out = C.c_float()
+        st = L.nvo_tensor_amax(b.ctypes.data + 2 * rr[0] * cols, rr[1] - rr[0], cols, cols,
+                               C.byref(out))
+        return st, out.value
+
+    with ThreadPoolExecutor(max(1, len(ranges))) as ex:
+        parts = list(ex.map(amax_of, ranges))
+        amax = 0.0
+        for st, a in parts:
+            if st != OK:
+                return st, Quantized(codes, scales, 0.0, rows, cols, layout)
+            amax = max(amax, a)
+        st, g = global_scale(amax)
+        if st != OK:
+            return st, Quantized(codes, scales, g, rows, cols, layout)
+
+        def encode(rr):
+            r0, r1 = rr
+            sf0 = scales_bytes(r0, cols, layout)
+            L.nvo_quantize_with_global(b.ctypes.data + 2 * r0 * cols, r1 - r0, cols, cols,
+                                       float(np.float32(g)), codes.ctypes.data + r0 * (cols // 2),
+                                       scales.ctypes.data + sf0, layout)
+
+        list(ex.map(encode, ranges))
+    return OK, Quantized(codes, scales, g, rows, cols, layout)
 
 
 def dequantize(codes, scales, layout, g, rows, cols) -> np.ndarray:
