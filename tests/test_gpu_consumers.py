@@ -1,6 +1,7 @@
 """GPU parity of the consumer steps against the oracle: the MoE per-token
 combine (bit for bit: the same FMA chain in the same order) and the NVFP4
--> FP8 conversion for attention reads (bit for bit)."""
+-> FP8 conversion for attention reads (bit for bit, after the quantize of
+the same input is itself checked against the oracle)."""
 import numpy as np
 import pytest
 import torch
@@ -8,7 +9,7 @@ import torch
 import oracle
 from nvfp4_block_scaled_22_b200 import binding as nb
 from nvfp4_block_scaled_22_b200 import inputs
-from tests.gpu_util import to_host_quantized
+from tests.gpu_util import assert_quantized_equal
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -46,15 +47,26 @@ def test_moe_combine_shapes_and_skipped_slots(tokens, topk, hidden):
     assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref)
 
 
-@pytest.mark.parametrize("layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
-def test_fp8_conversion_kv_tensor(layout):
-    x = inputs.kv_tensor(0, 1, device=DEV).view(inputs.KV_TOKENS, -1)[:8192]
-    q = nb.nvfp4_quantize(x.contiguous(), layout=layout)
+def _fp8_case(x_dev, layout, what):
+    """GPU quantize then GPU NVFP4 -> FP8, against the oracle's own quantize
+    of the same BF16 input followed by the oracle's conversion: both steps
+    are checked, and no oracle input comes from the GPU."""
+    q = nb.nvfp4_quantize(x_dev, layout=layout)
     y, sc = nb.nvfp4_dequantize_fp8(q)
     torch.cuda.synchronize()
-    ref, rsc = oracle.dequantize_fp8(to_host_quantized(q))
+    assert nb.nvfp4_check_status() == 0
+    st, r = oracle.quantize(x_dev.cpu(), layout)
+    assert st == oracle.OK
+    assert_quantized_equal(q, r, what)
+    ref, rsc = oracle.dequantize_fp8(r)
     assert np.float32(sc.item()) == np.float32(rsc)
     assert np.array_equal(y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
+def test_fp8_conversion_kv_tensor(layout):
+    x = inputs.kv_tensor(0, 1, device=DEV).view(inputs.KV_TOKENS, -1)[:8192].contiguous()
+    _fp8_case(x, layout, "kv rows for fp8")
 
 
 def test_fp8_conversion_ragged_and_tiny_scales():
@@ -62,10 +74,7 @@ def test_fp8_conversion_ragged_and_tiny_scales():
     x = torch.randn(130, 96, generator=g)
     x[3] *= 1e-6                                      # tiny block scales: FP8 underflow
     x[4] *= 1e4
-    q = nb.nvfp4_quantize(x.to(torch.bfloat16).to(DEV))
-    y, sc = nb.nvfp4_dequantize_fp8(q)
-    ref, rsc = oracle.dequantize_fp8(to_host_quantized(q))
-    assert np.float32(sc.item()) == np.float32(rsc) and np.array_equal(y.cpu().numpy(), ref)
+    _fp8_case(x.to(torch.bfloat16).to(DEV), nb.SF_SWIZZLED, "ragged fp8")
 
 
 @pytest.mark.parametrize("rows,inter", [(1, 16), (37, 80), (300, 1040), (4096, 2048)])
@@ -78,5 +87,4 @@ def test_swiglu_quantize(rows, inter, layout):
     assert nb.nvfp4_check_status() == 0
     st, ref = oracle.quantize_swiglu(gu, layout)
     assert st == oracle.OK
-    from tests.gpu_util import assert_quantized_equal
     assert_quantized_equal(q, ref, f"swiglu {rows}x{inter}")

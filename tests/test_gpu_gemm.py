@@ -92,18 +92,32 @@ def test_output_pitch_and_untouched_padding():
     assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab))
 
 
+def tile_samples(m, n, rng, tm=128, tn=256):
+    """Outputs that touch every tm x tn output tile: per tile one random
+    interior output, its last row at a random column, its last column at a
+    random row, and its last (row, column) corner.  Any fault tied to a
+    tile index, a CTA's wave or a ragged edge lands on at least one."""
+    mt, nt = -(-m // tm), -(-n // tn)
+    ti, tj = np.meshgrid(np.arange(mt), np.arange(nt), indexing="ij")
+    ti, tj = ti.ravel(), tj.ravel()
+    r0, c0 = ti * tm, tj * tn
+    rl = np.minimum(r0 + tm, m) - 1                   # last row / column of the tile
+    cl = np.minimum(c0 + tn, n) - 1
+    ri = r0 + (rng.random(ti.size) * (rl - r0 + 1)).astype(np.int64)
+    ci = c0 + (rng.random(tj.size) * (cl - c0 + 1)).astype(np.int64)
+    return np.concatenate([ri, rl, ri, rl]), np.concatenate([ci, ci, cl, cl])
+
+
 def _sampled(d, ra, rw, m, n, count, seed, gw=None, rows_map=None):
     rng = np.random.default_rng(seed)
     i = rng.integers(0, m, count)
     j = rng.integers(0, n, count)
-    # corners and tile edges
-    edge_i = np.array([0, m - 1, min(127, m - 1), min(128, m - 1)])
-    edge_j = np.array([0, n - 1, min(255, n - 1), min(256, n - 1)])
-    i = np.concatenate([i, np.repeat(edge_i, 4)])
-    j = np.concatenate([j, np.tile(edge_j, 4)])
+    ti, tj = tile_samples(m, n, rng)
+    i = np.concatenate([i, ti])
+    j = np.concatenate([j, tj])
     wj = j if rows_map is None else rows_map(i, j)
     ref, ab = oracle.gemm_ref(ra, rw, i, wj, gw=None if gw is None else gw(i))
-    got = bf16_to_f64(d)[i, j]
+    got = bf16_to_f64(d[torch.from_numpy(i).to(d.device), torch.from_numpy(j).to(d.device)])
     tol = gemm_tolerance(ref, ab)
     bad = np.nonzero(np.abs(got - ref) > tol)[0]
     assert bad.size == 0, f"{bad.size} sampled outputs outside tolerance, e.g. {i[bad[:4]]},{j[bad[:4]]}"

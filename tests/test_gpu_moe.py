@@ -1,8 +1,12 @@
 """MoE expert block at full size (256 experts, top-8 of 4096 tokens, hidden
-6144, intermediate 2048) against the oracle on sampled experts and outputs.
+6144, intermediate 2048) against the oracle, on every expert.
 
-Oracle inputs come only from the seeded generators: the down projection is
-checked on a generated intermediate (not on the GPU's up-projection output).
+Per expert: its tensor scale and the sampled weight rows are checked bit for
+bit against the oracle (four experts' weights in full), and outputs are
+sampled so that every expert's first and last real row and every 256-column
+output tile are touched.  Oracle inputs come only from the seeded generators:
+the down projection is checked on a generated intermediate (not on the GPU's
+up-projection output).
 """
 import numpy as np
 import pytest
@@ -16,7 +20,7 @@ from tests.gpu_util import assert_quantized_equal, bf16_to_f64, gemm_tolerance
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 E, H, I = inputs.MOE_EXPERTS, inputs.MOE_HIDDEN, inputs.MOE_INTER
-SAMPLE_EXPERTS = (0, 17, 128, 255)
+FULL_EXPERTS = (0, 17, 128, 255)
 
 
 @pytest.fixture(scope="module")
@@ -30,28 +34,68 @@ def _stacked(which, n, k):
     sfb = nb.nvfp4_scales_bytes(n, k)
     for e in range(E):
         w = inputs.moe_expert_weight(which, e, device=DEV)
-        sub = nb.NVFP4Tensor(q.codes[e * n:(e + 1) * n], q.scales[e * sfb:(e + 1) * sfb],
-                             g[e:e + 1], n, k, nb.SF_SWIZZLED)
-        nb.nvfp4_quantize(w, out=sub)
+        nb.nvfp4_quantize(w, out=_slice(q, g, e, n, k, sfb))
     assert nb.nvfp4_check_status() == 0
     return q, g, sfb
 
 
-def _expert_ref(which, e, n, k, q, g, sfb):
-    """Oracle quantization of expert e's weight, checked against the GPU slice."""
+def _slice(q, g, e, n, k, sfb):
+    return nb.NVFP4Tensor(q.codes[e * n:(e + 1) * n], q.scales[e * sfb:(e + 1) * sfb],
+                          g[e:e + 1], n, k, nb.SF_SWIZZLED)
+
+
+def _sf_table(n, k):
+    """Byte offset of block (row, block column) in one expert's 128x4 scale
+    slice, from the oracle's layout function."""
+    t = np.empty((n, k // 16), np.int64)
+    for r in range(n):
+        for c in range(k // 16):
+            t[r, c] = oracle.sf_offset(r, c, n, k, oracle.SF_SWIZZLED)
+    return t
+
+
+def _tile_cols(n, rng):
+    """One random column in every 256-column output tile, plus the last."""
+    c = np.arange(0, n, 256) + rng.integers(0, 256, -(-n // 256))
+    return np.unique(np.concatenate([np.minimum(c, n - 1), [n - 1]]))
+
+
+def _edge_rows(routing, e, rng):
+    """First, last and one random real row of expert e's slot (global rows)."""
+    o, r = int(routing.slot_offsets[e]), int(routing.rows[e])
+    if r == 0:
+        return np.zeros(0, np.int64)
+    return np.unique(np.array([o, o + r - 1, o + int(rng.integers(0, r))], np.int64))
+
+
+def _at(d, i, j):
+    """D[i, j] as float64, gathered on the device."""
+    it = torch.from_numpy(np.ascontiguousarray(i, np.int64)).to(DEV)
+    jt = torch.from_numpy(np.ascontiguousarray(j, np.int64)).to(DEV)
+    return bf16_to_f64(d[it, jt])
+
+
+def _expert_check(which, e, n, k, q, g, sfb, cols, sf_table):
+    """Oracle tensor scale of expert e's weight (over all of it) and the
+    oracle quantization of weight rows `cols` under it, both checked bit for
+    bit against the GPU's stacked tensor.  Returns those rows as an oracle
+    tensor (row-major scales) for the GEMM reference."""
     w = inputs.moe_expert_weight(which, e, device=DEV).cpu()
-    st, ref = oracle.quantize(w)
+    if e in FULL_EXPERTS:
+        st, full = oracle.quantize_parallel(w)
+        assert st == oracle.OK
+        assert_quantized_equal(_slice(q, g, e, n, k, sfb), full, f"W_{which}[{e}]")
+    st, amax = oracle.tensor_amax(w)
     assert st == oracle.OK
-    sub = nb.NVFP4Tensor(q.codes[e * n:(e + 1) * n], q.scales[e * sfb:(e + 1) * sfb],
-                         g[e:e + 1], n, k, nb.SF_SWIZZLED)
-    assert_quantized_equal(sub, ref, f"W_{which}[{e}]")
-    return ref
-
-
-def _sample_rows(routing, e, count, rng):
-    o = int(routing.slot_offsets[e])
-    r = int(routing.rows[e])
-    return o + rng.integers(0, r, count)
+    st, gw = oracle.global_scale(amax)
+    assert st == oracle.OK
+    assert np.float32(g[e].item()) == np.float32(gw), f"W_{which}[{e}] tensor scale"
+    sub = oracle.quantize_with_global(w[torch.from_numpy(cols)], gw, oracle.SF_LINEAR)
+    rows = torch.from_numpy(e * n + cols).to(DEV)
+    assert np.array_equal(q.codes[rows].cpu().numpy(), sub.codes), f"W_{which}[{e}] codes"
+    sf = q.scales[e * sfb:(e + 1) * sfb].cpu().numpy()
+    assert np.array_equal(sf[sf_table[cols]].ravel(), sub.scales), f"W_{which}[{e}] scales"
+    return sub
 
 
 def test_routing_structure(routing):
@@ -81,18 +125,21 @@ def test_up_projection_full_size(routing):
     g = oracle.global_scale(amax)[1]
     assert float(gx[0]) == g
     rng = np.random.default_rng(1)
-    qx_codes = qx.codes.cpu().numpy()
-    for e in SAMPLE_EXPERTS:
-        ref_w = _expert_ref("up", e, I, H, wu, gu, sfb)
-        rows = _sample_rows(routing, e, 6, rng)
-        src = routing.gather[rows].long()
+    sf_table = _sf_table(I, H)
+    for e in range(E):
+        cols = _tile_cols(I, rng)
+        ref_w = _expert_check("up", e, I, H, wu, gu, sfb, cols, sf_table)
+        rows = _edge_rows(routing, e, rng)
+        if rows.size == 0:
+            continue
+        src = routing.gather[torch.from_numpy(rows)].long()
         qa = oracle.quantize_with_global(xc[src], g)
-        assert np.array_equal(qa.codes, qx_codes[rows]), f"gathered codes, expert {e}"
-        cols = rng.integers(0, I, 40)
+        assert np.array_equal(qa.codes, qx.codes[torch.from_numpy(rows).to(DEV)].cpu().numpy()), \
+            f"gathered codes, expert {e}"
         ii = np.repeat(np.arange(len(rows)), len(cols))
-        jj = np.tile(cols, len(rows))
+        jj = np.tile(np.arange(len(cols)), len(rows))
         ref, ab = oracle.gemm_ref(qa, ref_w, ii, jj)
-        got = bf16_to_f64(h)[rows[ii], jj]
+        got = _at(h, rows[ii], cols[jj])
         assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab)), f"expert {e}"
 
 
@@ -111,15 +158,19 @@ def test_down_projection_full_size(routing):
     assert nb.nvfp4_check_status() == 0
 
     hc = hmid.cpu()
-    st, rq = oracle.quantize(hc)                 # padding rows are zero: same amax
+    st, rq = oracle.quantize_parallel(hc)        # padding rows are zero: same amax
+    assert st == oracle.OK
     assert_quantized_equal(qh, rq, "intermediate")
     rng = np.random.default_rng(2)
-    for e in SAMPLE_EXPERTS:
-        ref_w = _expert_ref("down", e, H, I, wd, gd, sfb)
-        rows = _sample_rows(routing, e, 5, rng)
-        cols = rng.integers(0, H, 40)
+    sf_table = _sf_table(H, I)
+    for e in range(E):
+        cols = _tile_cols(H, rng)
+        ref_w = _expert_check("down", e, H, I, wd, gd, sfb, cols, sf_table)
+        rows = _edge_rows(routing, e, rng)
+        if rows.size == 0:
+            continue
         ii = np.repeat(rows, len(cols))
-        jj = np.tile(cols, len(rows))
+        jj = np.tile(np.arange(len(cols)), len(rows))
         ref, ab = oracle.gemm_ref(rq, ref_w, ii, jj)
-        got = bf16_to_f64(y)[ii, jj]
+        got = _at(y, ii, cols[jj])
         assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab)), f"expert {e}"

@@ -74,7 +74,7 @@ def test_sweep_largest_full_compare():
     x = inputs.sweep_tensor(n, device=DEV)
     q = nb.nvfp4_quantize(x)
     assert nb.nvfp4_check_status() == 0
-    st, ref = oracle.quantize(x.cpu())
+    st, ref = oracle.quantize_parallel(x.cpu())
     assert st == oracle.OK
     assert_quantized_equal(q, ref, "sweep 2^28")
 
@@ -92,10 +92,34 @@ def test_kv_tensor_linear_layout():
     x = inputs.kv_tensor(0, 1, device=DEV).view(-1, inputs.KV_HEADS * inputs.KV_HEAD_DIM)
     q = nb.nvfp4_quantize(x, layout=nb.SF_LINEAR)
     assert nb.nvfp4_check_status() == 0
-    st, ref = oracle.quantize(x.cpu(), oracle.SF_LINEAR)
+    st, ref = oracle.quantize_parallel(x.cpu(), oracle.SF_LINEAR)
     assert_quantized_equal(q, ref, "kv layer0 V")
     # 0.5625 bytes per value, no padding
     assert q.nbytes() == x.numel() * 9 // 16
+    # dequantize round trip of the full tensor, bit for bit
+    y = nb.nvfp4_dequantize(q)
+    assert np.array_equal(y.cpu().view(torch.int16).numpy().view(np.uint16), ref.dequantize())
+
+
+def test_kv_cache_every_tensor():
+    """All 64 tensors of the KV workload (32 layers x K, V), one at a time,
+    each bit for bit against the oracle, in the workspace and output buffers
+    a cache would reuse."""
+    T, C = inputs.KV_TOKENS, inputs.KV_HEADS * inputs.KV_HEAD_DIM
+    q = nb.NVFP4Tensor.empty(T, C, nb.SF_LINEAR, DEV)
+    ws = nb.Workspace(DEV)
+    total = 0
+    for layer in range(inputs.KV_LAYERS):
+        for kv in (0, 1):
+            x = inputs.kv_tensor(layer, kv, device=DEV).view(T, C)
+            nb.nvfp4_quantize(x, out=q, workspace=ws)
+            assert nb.nvfp4_check_status(ws) == 0
+            st, ref = oracle.quantize_parallel(x.cpu(), oracle.SF_LINEAR)
+            assert st == oracle.OK
+            assert_quantized_equal(q, ref, f"kv layer {layer} {'KV'[kv]}")
+            total += q.nbytes()
+    # the KV page's worked example: 36 KiB per token over the 64 tensors
+    assert total == T * 36 * 1024
 
 
 def test_zero_tensor_and_empty():
