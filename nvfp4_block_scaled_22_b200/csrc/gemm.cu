@@ -259,8 +259,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
             }
-            if (!ok) {
-                // Let every copy already issued land before the CTA can exit.
+            // Let every copy already issued land before the CTA can exit: after
+            // an abort (here or in another role) the consumers may never wait
+            // on the last stages armed; in a normal run those phases have
+            // completed and each check returns at once.
+            {
                 for (int s = 0; s < kStages; ++s) {
                     if (!armed[s]) continue;
                     const long long t0 = clock64();
@@ -328,6 +331,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             }
             if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
+        tmem_st_wait();   // no store in flight when TMEM is released (abort path)
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {

@@ -184,7 +184,11 @@ k_gemm_nvf4_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (++stage == kPStages) { stage = 0; phase ^= 1; }
                 }
             }
-            if (!ok) {
+            // Let every copy already issued land before the CTA can exit: after
+            // an abort (here or in another role) the consumers may never wait
+            // on the last stages armed; in a normal run those phases have
+            // completed and each check returns at once.
+            {
                 for (int s = 0; s < kPStages; ++s) {
                     if (!armed[s]) continue;
                     const long long t0 = clock64();
@@ -238,6 +242,7 @@ k_gemm_nvf4_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             }
             if (++stage == kPStages) { stage = 0; phase ^= 1; }
         }
+        tmem_st_wait();   // no store in flight when TMEM is released (abort path)
     } else if (warp == 1) {
         // -------------------------------------------- MMA (leader CTA only)
         if (lane == 0 && leader) {
