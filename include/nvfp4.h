@@ -350,12 +350,15 @@ NVFP4_API nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *
  * It takes no workspace: its scratch (status word plus up to 1024 per-block
  * partial maxima, 4352 bytes) is a fixed device array inside the library
  * that every GPU loading the library keeps until the process exits.  The
- * scratch does not grow with the tensor, so every size nvfp4_quantize
- * accepts is accepted here; a launch needing more partial slots than the
- * array holds would be refused with NVFP4_ERR_WORKSPACE.
- * - The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ * scratch does not grow with the tensor (the amax pass runs at most four
+ * blocks per SM, each striding over rows), so every size nvfp4_quantize
+ * accepts is accepted here; a device with more than 256 SMs would need more
+ * than the 1024 partial slots and is refused with NVFP4_ERR_WORKSPACE.
+ * - The first call in a CUDA context looks up the array's device address
+ *   (with that device current) and caches it against the context; make that
+ *   first call before any stream capture.  After cudaDeviceReset the new
+ *   context looks the address up again on its first call (again before any
+ *   capture).
  * - All calls share the array and the status word is cleared by every call:
  *   calls whose kernels can overlap on the GPU (unordered streams) race and
  *   must not be issued.

@@ -17,6 +17,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -34,21 +35,60 @@ constexpr size_t kNoAllocScratchBytes = kNoAllocStatusBytes + 4 * kNoAllocPartia
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevs = 64;
-void *g_scratch_ptr[kMaxDevs] = {};
+struct ScratchAddr {
+    unsigned long long ctx = 0;   // unique ID of the context the address belongs to
+    void *ptr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevs];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device.  The array's
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Unique ID of the calling thread's current CUDA context, 0 if there is none
+// yet or the driver cannot say.  A context destroyed and created again (for
+// instance by cudaDeviceReset) gets a new ID, and its copy of the scratch
+// array may live at a new address.
+unsigned long long current_context_id() {
+    std::call_once(g_ctx_once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_current == nullptr || g_ctx_get_id == nullptr || g_ctx_current(&c) != CUDA_SUCCESS ||
+        c == nullptr || g_ctx_get_id(c, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current context.  The array's
 // name in host code is only a host-side stand-in, so the address is looked
-// up once per device (with that device current) and cached.
+// up with cudaGetSymbolAddress (with the device current) the first time a
+// context calls, and cached against that context's ID; a new context
+// (after a device reset) looks it up again.
 cudaError_t scratch_address(int dev, void **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    ScratchAddr &a = g_scratch_addr[dev];
+    const unsigned long long id = current_context_id();
+    if (id == 0 || a.ptr == nullptr || a.ctx != id) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+        a.ptr = p;
+        a.ctx = current_context_id();   // the lookup has made the context current
     }
-    *out = g_scratch_ptr[dev];
+    *out = a.ptr;
     return cudaSuccess;
 }
 
@@ -93,12 +133,15 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t ld, const 
         return NVFP4_ERR_CUDA;
     if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED_DEVICE;
 
-    // The amax pass writes one partial maximum per CTA; the launch below is
-    // capped at the scratch's capacity, and a launch needing more partial
-    // slots than the scratch holds is refused.
-    const int amax_ctas = (int)std::max<int64_t>(
-        1, std::min<int64_t>(std::min<int64_t>(ceil_div64(out->rows, 8), 4LL * sms), kNoAllocPartials));
+    // The amax pass writes one partial maximum per CTA and runs at most four
+    // CTAs per SM (they stride over any number of rows, so the tensor's size
+    // never needs more).  A device with more than 256 SMs would need more
+    // partial slots than the array holds: refused, not truncated.
+    const int amax_ctas =
+        (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(out->rows, 8), 4LL * sms));
     if (amax_ctas > kNoAllocPartials) return NVFP4_ERR_WORKSPACE;
+    const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
+    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
 
     void *scratch = nullptr;
     if (scratch_address(dev, &scratch) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -128,14 +171,19 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t ld, const 
     p.partials = partials;
     p.n_partials = n_partials;
     p.status = status;
-    const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
-    if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
     const bool narrow = tasks_are_groups(out->cols);
     void (*kernel)(EncodeParams) = narrow ? k_encode_narrow : k_encode;
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>(ceil_div64(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms));
     kernel<<<grid, 256, 0, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) {
+        // The amax pass may already have flagged the shared status word:
+        // clear it anyway (best effort), or the next clean call would report
+        // this call's error.
+        k_status_to_global<<<1, 32, 0, s>>>(status, out->global);
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
     k_status_to_global<<<1, 32, 0, s>>>(status, out->global);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     return NVFP4_OK;
