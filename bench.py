@@ -477,7 +477,7 @@ def workload_line(name, args, device):
         return line
 
     if name == "kv":
-        L, T = inputs.KV_LAYERS, inputs.KV_TOKENS
+        L, T = args.layers, inputs.KV_TOKENS
         C = inputs.KV_HEADS * inputs.KV_HEAD_DIM
         xs = [inputs.kv_tensor(l, kv, device=device).view(T, C) for l in range(L) for kv in (0, 1)]
         qs = [nb.NVFP4Tensor.empty(T, C, nb.SF_LINEAR, device) for _ in xs]
@@ -500,7 +500,7 @@ def workload_line(name, args, device):
         per_token = sum(q.nbytes() for q in qs) // T
         line.update({"metric": "NVFP4 KV-cache quantize GB/s (32 layers x K,V, 128K tokens)",
                      "value": qgbs, "unit": "GB/s", "higher_is_better": True, "ms_per_step": qms,
-                     "config": {"workload": "kv cache 32 x {K,V} x [131072 x 8 x 128]"},
+                     "config": {"workload": f"kv cache {L} x {{K,V}} x [131072 x 8 x 128]"},
                      "bytes_per_token": per_token, "bytes_per_value": per_token / (2 * L * C),
                      "dequantize_ms": dms, "dequantize_gbs": dgbs, "status": st,
                      "roofline": {"kernel": "k_amax + k_encode", "bound": "hbm", "achieved": qgbs,
@@ -716,7 +716,7 @@ def workload_line(name, args, device):
         # than L2, so no flush is needed between steps.
         T, H = inputs.KV_TOKENS, inputs.KV_HEADS
         layers = []
-        for layer in range(inputs.KV_LAYERS):
+        for layer in range(args.layers):
             kq = []
             for kv in (0, 1):
                 x = inputs.kv_tensor(layer, kv, device=device).view(T, -1)
@@ -736,7 +736,7 @@ def workload_line(name, args, device):
                                                        out=outs[0], workspace=aws),
                      args.steps, args.warmup, flush)
         st = nb.nvfp4_check_status(ws)
-        cache_bytes = inputs.KV_LAYERS * 2 * T * H * 128 * 0.5625
+        cache_bytes = len(layers) * 2 * T * H * 128 * 0.5625
         gbs = cache_bytes / ms / 1e6
         # Scores run on the tensor cores; the weighted V sum (2 flops per
         # MAC, heads_q x T x 128 MACs) on the FP32 pipes bounds the design.
@@ -746,7 +746,8 @@ def workload_line(name, args, device):
         line.update({"metric": "NVFP4 KV-cache decode attention GB/s of cache read (32 layers x K,V, "
                                "128K tokens, 64 query / 8 KV heads)",
                      "value": gbs, "unit": "GB/s", "higher_is_better": True, "ms_per_step": ms,
-                     "config": {"workload": "attention decode 32 x {K,V} x [131072 x 8 x 128], 64 query heads",
+                     "config": {"workload": f"attention decode {len(layers)} x {{K,V}} x [131072 x 8 x 128], "
+                                            "64 query heads",
                                 "l2": "inputs (4.8 GB cache) larger than L2; one-layer timing flushed"},
                      "tokens_per_s": 1e3 / ms, "ms_per_layer": one, "status": st,
                      "hbm_frac": gbs / hbm_gbs,
@@ -778,6 +779,9 @@ def main():
                     choices=["ffn8192", "ffn16", "ffn512", "sweep", "moe", "kv", "wgrad", "train", "mxfp4", "consumers",
                              "attention"],
                     help="ffn8192 is the headline; the others measure the remaining scope rows")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="kv / attention workloads: layers of the KV cache (the workload has 32; "
+                         "fewer give a case small enough for a multi-pass ncu capture)")
     ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
                     help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")
     args = ap.parse_args()
