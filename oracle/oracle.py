@@ -17,7 +17,7 @@ __all__ = [
     "lib", "bf16_bits", "bf16_to_f32", "f32_to_bf16", "e2m1_decode", "e2m1_rne",
     "e4m3_decode", "e4m3_rne", "scales_bytes", "sf_offset", "tensor_amax",
     "global_scale", "quantize", "quantize_with_global", "quantize_parallel", "dequantize",
-    "gemm_ref",
+    "gemm_ref", "gemm_ref_parallel", "tensor_amax_parallel", "host_threads",
     "dot_exact_i64", "Quantized", "rht16", "rht16_inverse", "quantize_rht", "quantize_2d",
     "philox4x32_10", "e2m1_sr", "sr_block_draws", "quantize_sr",
     "ue8m0_decode", "mx_scales_bytes", "mx_sf_offset", "mx_exponent", "quantize_mx",
@@ -197,6 +197,36 @@ def _row_ranges(rows: int, threads: int) -> list[tuple[int, int]]:
     return [(r, min(rows, r + step)) for r in range(0, rows, step)]
 
 
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def tensor_amax_parallel(x, threads: int | None = None) -> tuple[int, float]:
+    """`tensor_amax` over disjoint row ranges on host threads; the maximum of
+    the ranges' exact maxima is the tensor's (a maximum does not depend on
+    grouping)."""
+    from concurrent.futures import ThreadPoolExecutor
+    b = bf16_bits(x)
+    rows, cols = b.shape
+    ranges = _row_ranges(rows, threads or host_threads())
+    L = lib()
+
+    def amax_of(rr):
+        out = C.c_float()
+        st = L.nvo_tensor_amax(b.ctypes.data + 2 * rr[0] * cols, rr[1] - rr[0], cols, cols,
+                               C.byref(out))
+        return st, out.value
+
+    amax = 0.0
+    with ThreadPoolExecutor(max(1, len(ranges))) as ex:
+        for st, a in ex.map(amax_of, ranges):
+            if st != OK:
+                return st, 0.0
+            amax = max(amax, a)
+    return OK, amax
+
+
 def quantize_parallel(x, layout: int = SF_SWIZZLED, threads: int | None = None
                       ) -> tuple[int, Quantized]:
     """`quantize` with its row loops spread over host threads (the C calls
@@ -273,6 +303,22 @@ def gemm_ref(a: Quantized, w: Quantized, i_idx, j_idx, gw=None):
                        _ptr(w.codes), _ptr(w.scales), w.layout, _ptr(gw), w.rows, a.cols,
                        _ptr(i_idx), _ptr(j_idx), n, _ptr(ref), _ptr(ab))
     return ref, ab
+
+
+def gemm_ref_parallel(a: Quantized, w: Quantized, i_idx, j_idx, threads: int | None = None):
+    """`gemm_ref` with the sampled outputs split over host threads (each
+    output is computed by the same C routine, independently)."""
+    from concurrent.futures import ThreadPoolExecutor
+    i_idx = np.ascontiguousarray(i_idx, np.int64)
+    j_idx = np.ascontiguousarray(j_idx, np.int64)
+    n = len(i_idx)
+    t = max(1, min(threads or host_threads(), n))
+    bounds = [(n * q) // t for q in range(t + 1)]
+    with ThreadPoolExecutor(t) as ex:
+        parts = list(ex.map(lambda q: gemm_ref(a, w, i_idx[bounds[q]:bounds[q + 1]],
+                                               j_idx[bounds[q]:bounds[q + 1]]), range(t)))
+    return (np.concatenate([p[0] for p in parts]) if parts else np.zeros(0),
+            np.concatenate([p[1] for p in parts]) if parts else np.zeros(0))
 
 
 def dot_exact_i64(a: Quantized, w: Quantized, i: int, j: int) -> int:

@@ -40,3 +40,16 @@ def test_parallel_special_tensors():
     tiny = torch.full((256, 32), 1e-37, dtype=torch.bfloat16)
     assert oracle.quantize_parallel(tiny, threads=2)[0] == oracle.ERR_RANGE
     assert oracle.quantize_parallel(torch.zeros(0, 16, dtype=torch.bfloat16))[0] == oracle.OK
+
+
+def test_parallel_amax_and_gemm_reference():
+    g = torch.Generator().manual_seed(99)
+    x = (torch.randn(700, 96, generator=g) * 3).to(torch.bfloat16)
+    assert oracle.tensor_amax_parallel(x, threads=5) == oracle.tensor_amax(x)
+    st, qa = oracle.quantize(x[:37])
+    st2, qw = oracle.quantize(x[100:300])
+    rng = np.random.default_rng(0)
+    i, j = rng.integers(0, 37, 501), rng.integers(0, 200, 501)
+    r1, a1 = oracle.gemm_ref(qa, qw, i, j)
+    r2, a2 = oracle.gemm_ref_parallel(qa, qw, i, j, threads=7)
+    assert np.array_equal(r1, r2) and np.array_equal(a1, a2)
