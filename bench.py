@@ -44,8 +44,9 @@ FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 ATTN_FP32_LANES = 148 * 128  # FP32 FMA lanes of a B200 (148 SMs x 128)
 SM_MAX_MHZ = 1965           # clocks.max.sm of the B200
 # DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
-# the ncu capture in profiles/k_gemm_nvf4_w4a4_ffn_M8192_N20480_K5120.md.
-# Reported only while the kernel's sources hash to the profiled version.
+# an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum of one launch
+# at this shape.  Reported only while the kernel's sources hash to the
+# profiled version (otherwise null).
 GEMM_TRAFFIC_BYTES = 87.85e6 + 292.76e6
 GEMM_TRAFFIC_SRC_SHA = "6c187c6de44d0cf0"
 GEMM_SOURCES = ("gemm.cu", "gemm.h", "ptx.cuh")
@@ -262,63 +263,73 @@ def time_e2e(wl: Workload, steps: int, warmup: int):
 
 
 # ------------------------------------------------------- CPU oracle timing
-def oracle_sample(rows: int = 1, cols: int = 4096, seed: int = 0):
-    """Oracle on a bounded sample of the step: quantize `rows` rows of A (with
-    the full-tensor amax pass) and compute their first `cols` outputs of the
-    FP64 GEMM against the oracle-quantized W.  Returns (seconds, flops)."""
+def oracle_sample(rows: int = 1, cols: int = 4096, seed: int = 0, threads: int = 1):
+    """Oracle on a bounded sample of the step: the tensor amax over all of A
+    (A's tensor scale needs it), quantize `rows` rows of A with that scale,
+    and compute their first `cols` outputs of the FP64 GEMM against the
+    oracle-quantized W, on `threads` host threads.  Returns (seconds, flops)."""
     import numpy as np
     import oracle
     from nvfp4_block_scaled_22_b200 import inputs
     cache = oracle_sample.__dict__.setdefault("cache", {})
     if "w" not in cache:
         w = inputs.ffn_weight()
-        st, qw = oracle.quantize(w)
+        st, qw = oracle.quantize_parallel(w)
         a = inputs.ffn_activation(M)
         cache["w"], cache["a"] = qw, a
     qw, a = cache["w"], cache["a"]
-    r0 = (seed * rows) % M
+    r0 = (seed * rows) % (M - rows + 1)
     t0 = time.perf_counter()
-    st, amax = oracle.tensor_amax(a)
+    st, amax = oracle.tensor_amax_parallel(a, threads)
     st, g = oracle.global_scale(amax)
     qa = oracle.quantize_with_global(a[r0:r0 + rows], g)
     ii, jj = np.meshgrid(np.arange(rows), np.arange(cols), indexing="ij")
-    oracle.gemm_ref(qa, qw, ii.ravel(), jj.ravel())
+    oracle.gemm_ref_parallel(qa, qw, ii.ravel(), jj.ravel(), threads)
     dt = time.perf_counter() - t0
     return dt, 2.0 * rows * cols * K
 
 
 def cpu_baseline_entry():
-    dt, flops = oracle_sample()
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": f"1 of {M} rows of A: tensor amax over all of A, quantize the row, "
-                      f"then 4096 of {N} outputs of the FP64 GEMM (K={K}) against the "
-                      f"oracle-quantized W; single-threaded C ({dt:.2f} s)"}
+    import oracle
+    cores = oracle.host_threads()
+    oracle_sample()                                   # setup (W quantized once), untimed
+    dt1, f1 = oracle_sample(rows=1, threads=1)
+    dtn, fn = oracle_sample(rows=cores, seed=1, threads=cores)
+    return {"value": fn / dtn / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "value_1core": f1 / dt1 / 1e12,
+            "sample": f"{cores} of {M} rows of A (one per thread): tensor amax over all of A, "
+                      f"quantize the rows, then 4096 of {N} outputs per row of the FP64 GEMM "
+                      f"(K={K}) against the oracle-quantized W, on {cores} host threads "
+                      f"({dtn:.2f} s); value_1core: 1 row on one thread ({dt1:.2f} s)"}
 
 
 def run_reference(args):
+    import oracle
     rank, _, world = env_rank()
     if rank != 0:
         return 0
+    cores = oracle.host_threads()
     oracle_sample()   # builds the oracle and quantizes W once (setup, untimed)
     for i in range(args.warmup):
-        oracle_sample(seed=i)
+        oracle_sample(rows=cores, seed=i, threads=cores)
     times, flops = [], 0.0
     for i in range(args.steps):
-        dt, f = oracle_sample(seed=args.warmup + i)
+        dt, f = oracle_sample(rows=cores, seed=args.warmup + i, threads=cores)
         times.append(dt)
         flops = f
     total = sum(times)
     value = flops * args.steps / total / 1e12
+    sample = (f"per step: {cores} rows of A quantized (after the full-tensor amax) and 4096 "
+              f"outputs per row of the FP64 GEMM, K=5120, on {cores} host threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": WORKLOAD + " [oracle sample per step: 1 row x 4096 outputs]",
+        "config": {"workload": WORKLOAD + f" [oracle sample per step: {cores} rows x 4096 outputs]",
                    "M": M, "N": N, "K": K},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": "per step: 1 row of A quantized (after the full-tensor "
-                                   "amax) and 4096 outputs of the FP64 GEMM, K=5120"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
