@@ -23,6 +23,7 @@ constexpr int kMaxDevices = 64;
 constexpr size_t kStatusBytes = 256;          // status word + reserved
 constexpr int kMaxPartials = 1024;            // CTAs of the amax pass
 constexpr long long kDefaultTimeoutCycles = 2000000000ll;   // ~1 s at 1.9 GHz
+constexpr int64_t kFlatCols = 2048;           // row width for contiguous row-major-scale tensors
 
 struct DeviceInfo {
     bool checked = false;
@@ -113,17 +114,19 @@ nvfp4_status get_encode() {
 }
 
 // Packed-code matrix [rows x cols/2 bytes] as a 2-D uint8 tensor, boxes of
-// 128 bytes x box_rows, 128-byte swizzle (the MMA's K-major operand layout).
+// box_bytes (128 or 64) x box_rows, swizzled over the box row (the MMA's
+// K-major operand layout).
 nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, int64_t cols,
-                              uint32_t box_rows) {
+                              uint32_t box_rows, uint32_t box_bytes) {
     cuuint64_t dims[2] = {(cuuint64_t)(cols / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)(kBoxK / 2), box_rows};
+    cuuint32_t box[2] = {box_bytes, box_rows};
     cuuint32_t estr[2] = {1, 1};
+    if (box_bytes != 128 && box_bytes != 64) return NVFP4_ERR_INVALID_ARG;
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -166,9 +169,20 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
     p.status = status;
     p.rht_mask = rht_mask;
     p.sr_seed = sr_seed;
-    const int64_t tasks = encode_tasks(out->rows, out->cols, out->sf_layout);
+    // Narrow rows with row-major scales and no row padding (the KV cache) are
+    // one contiguous run of 16-value blocks in x, codes and scales alike:
+    // encode them as 2048-value rows, which the chunked kernel streams
+    // faster.  Same bytes at the same offsets.  (Not for stochastic rounding,
+    // whose draws are keyed by the row and block column, nor for gathers.)
+    if (!sr && gather == nullptr && out->sf_layout == NVFP4_SF_LINEAR && ld == out->cols &&
+        tasks_are_groups(out->cols) && (out->rows * out->cols) % kFlatCols == 0) {
+        p.rows = out->rows * out->cols / kFlatCols;
+        p.cols = kFlatCols;
+        p.ld = kFlatCols;
+    }
+    const int64_t tasks = encode_tasks(p.rows, p.cols, out->sf_layout);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    const bool narrow = tasks_are_groups(out->cols);
+    const bool narrow = tasks_are_groups(p.cols);
     void (*kernel)(EncodeParams) =
         sr ? (rht ? (narrow ? k_encode_rht_sr_narrow : k_encode_rht_sr)
                   : (narrow ? k_encode_sr_narrow : k_encode_sr))
@@ -790,9 +804,9 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     p.cols = in->cols;
     p.y = static_cast<uint16_t *>(y);
     p.ld = ld;
-    const int64_t tasks = decode_tasks(in->rows, in->cols);
+    const int64_t tasks = decode_tasks(p.rows, p.cols);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
-    const bool narrow = tasks_are_groups(in->cols);
+    const bool narrow = tasks_are_groups(p.cols);
     void (*kernel)(DequantParams) = narrow ? k_dequantize_narrow : k_dequantize;
     int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms);
     if (grid < 1) grid = 1;
@@ -800,6 +814,65 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     return launched(cudaGetLastError());
 }
 
+
+// Few rows of A: the swapped-operand kernel over units of (128-row W tile,
+// K split).  Split count: fewest stages on the busiest SM (plus one for the
+// finalize pass when split), ties to fewer splits, if the FP32 slices fit in
+// the workspace and the output allows the finalize's 4-column stores.
+static nvfp4_status gemm_swap(const nvfp4_tensor *A, const nvfp4_tensor *W, int64_t m, int64_t n,
+                              int64_t k, void *D, int64_t ldd, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream, int sms) {
+    const uint32_t mp = (uint32_t)((m + 15) / 16 * 16);
+    CUtensorMap tmW, tmX;
+    nvfp4_status st = encode_codes_map(&tmW, W->codes, W->rows, k, 128, 128);
+    if (st != NVFP4_OK) return st;
+    st = encode_codes_map(&tmX, A->codes, A->rows, k, mp, 128);
+    if (st != NVFP4_OK) return st;
+    GemmParams p;
+    p.sfa = static_cast<const uint8_t *>(A->scales);
+    p.sfb = static_cast<const uint8_t *>(W->scales);
+    p.d = static_cast<uint16_t *>(D);
+    p.ldd = ldd;
+    p.d_vec16 = (aligned16(D) && ldd % 8 == 0) ? 1 : 0;
+    p.m = (int32_t)m;
+    p.n = (int32_t)n;
+    p.k = (int32_t)k;
+    p.groups = 0;
+    p.slot_offsets = nullptr;
+    p.group_rows = nullptr;
+    p.ga = A->global;
+    p.gw = W->global;
+    p.a_row_blocks = 1;
+    p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
+    p.n_fastest = 0;
+    p.status = reinterpret_cast<uint32_t *>(workspace);
+    p.timeout_cycles = g_timeout_cycles;
+    p.splits = 1;
+    p.partial = nullptr;
+    const int64_t ntiles = ceil_div(n, 128);
+    const int ktiles = (int)ceil_div(k / 64, 4);
+    int64_t best_cost = ceil_div(ntiles, sms) * ktiles;
+    if (n % 16 == 0 && p.d_vec16) {
+        for (int sp = 2; sp <= std::min(16, ktiles); ++sp) {
+            const int64_t cost = ceil_div(ntiles * sp, sms) * ceil_div(ktiles, sp) + 1;
+            const size_t need = kStatusBytes + (size_t)sp * (size_t)m * (size_t)n * 4;
+            if (cost < best_cost && need <= workspace_bytes) {
+                best_cost = cost;
+                p.splits = sp;
+            }
+        }
+    }
+    if (p.splits > 1)
+        p.partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles * p.splits, sms));
+    st = launched(launch_gemm_swap(tmW, tmX, p, grid, stream));
+    if (st != NVFP4_OK || p.splits == 1) return st;
+    const int64_t quads = m * (n / 4);
+    const int fgrid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(quads, 256), 4LL * sms));
+    k_splitk_finalize<<<fgrid, 256, 0, stream>>>(p.partial, p.splits, (int)m, (int)n, p.ga, p.gw,
+                                                 p.d, p.ldd);
+    return launched(cudaGetLastError());
+}
 
 static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
                                 const int32_t *d_group_rows, const nvfp4_tensor *A,
@@ -835,10 +908,14 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     st = get_encode();
     if (st != NVFP4_OK) return st;
     const bool pair = !mx && groups == 0 && m >= kPairMinRows && sms >= 2 && g_use_pairs;
+    if (!mx && groups == 0 && m <= kSwapMaxRows)
+        return gemm_swap(A, W, m, n, k, D, ldd, workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream), sms);
     CUtensorMap tmA, tmB;
-    st = encode_codes_map(&tmA, A->codes, A->rows, k, kBM);
+    const uint32_t box_bytes = pair ? kPairBoxBytes : kSingleBoxBytes;
+    st = encode_codes_map(&tmA, A->codes, A->rows, k, kBM, box_bytes);
     if (st != NVFP4_OK) return st;
-    st = encode_codes_map(&tmB, W->codes, W->rows, k, pair ? 128 : kBN);
+    st = encode_codes_map(&tmB, W->codes, W->rows, k, pair ? 128 : kBN, box_bytes);
     if (st != NVFP4_OK) return st;
 
     GemmParams p;
@@ -857,7 +934,10 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.gw = gw;
     p.a_row_blocks = (int32_t)ceil_div(A->rows, 128);
     p.b_row_blocks = (int32_t)ceil_div(W->rows, 128);
-    p.n_fastest = (A->rows * (k / 2) > kL2SweepBytes && A->rows > W->rows) ? 1 : 0;
+    // Grouped: N fastest, so the CTAs working at one time hold a few experts'
+    // rows and sweep their weights once; M fastest would re-read the whole
+    // grouped activation tensor (larger than L2) once per N tile.
+    p.n_fastest = groups > 0 ? 1 : (A->rows * (k / 2) > kL2SweepBytes && A->rows > W->rows) ? 1 : 0;
     p.status = reinterpret_cast<uint32_t *>(workspace);
     p.timeout_cycles = g_timeout_cycles;
     p.splits = 1;
@@ -866,7 +946,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     // pick the split count that minimises the stage count of the busiest SM
     // (ties: fewer splits), if the FP32 slices fit in the workspace.
     const int64_t tiles_mn = ceil_div(m, kBM) * ceil_div(n, kBN);
-    const int ktiles = (int)ceil_div(k / 64, 4);
+    const int ktiles = (int)ceil_div(k / 64, kKB);     // the kernel's stages per tile
     if (!mx && !pair && groups == 0 && tiles_mn < sms && n % 16 == 0 && p.d_vec16) {
         int best = 1;
         int64_t best_cost = ktiles;                              // one unit per SM

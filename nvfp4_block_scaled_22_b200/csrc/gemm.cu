@@ -10,18 +10,19 @@
 // shrank GLM-5.2 to 4 bits" (section 1, weights and activations in NVFP4;
 // section 2, 256 experts with 8 active per token).
 //
-// Design (one persistent CTA per SM, 14 warps, 4-stage ring of 256 K-values):
-//   warp 0     TMA producer: per stage a 128x128-byte A box and a 256x128-byte
-//              W box of packed codes (128-byte swizzle) on `tma_ready`, and
-//              the matching 512-byte 128x4 scale tiles by bulk copy on
-//              `sf_landed`.
+// Design (one persistent CTA per SM, 14 warps, a ring of kNS stages of kSK
+// K-values each; gemm.h sets the geometry):
+//   warp 0     TMA producer: per stage a 128-row A box and a 256-row W box of
+//              packed codes (kSK/2-byte rows, swizzled to match the MMA
+//              descriptors) on `tma_ready`, and the matching 512-byte 128x4
+//              scale tiles by bulk copy on `sf_landed`.
 //   warps 2-5  scale writers, one per 32-lane TMEM quarter.  The tensor core
 //              reads block scales from TMEM, and tcgen05.cp spends
 //              tensor-pipe time on every instruction, so these warps read
 //              their rows of the scale tiles from shared memory and write the
 //              MMA's scale layout into TMEM with tcgen05.st.  They also wait
-//              for the stage's codes, and signal `pair_ready` once for every
-//              two stages, so the MMA issuer synchronises once per eight MMAs
+//              for the stage's codes, and arrive on `ready` once per group of
+//              kGrp stages, so the MMA issuer synchronises once per group
 //              (a completed mbarrier wait costs the issuing thread about as
 //              long as one MMA).
 //   warp 1     MMA issuer: tcgen05.mma kind::mxf4nvf4 (M128 N256 K64, E4M3
@@ -49,7 +50,12 @@ namespace {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kBN;          // 256 FP32 columns
-constexpr uint32_t kSfCols = 48;            // per stage: 4 K blocks x (4 A + 8 W) columns
+constexpr uint32_t kSfCols = kKB * 12;      // per stage: kKB K blocks x (4 A + 8 W) columns
+constexpr uint32_t kSfbCol0 = kKB * 4;      // W scales after the stage's A scales
+// Shared-memory descriptor of a K-major operand in a stage: 128- or 64-byte
+// swizzle rows, 8-row groups kBoxBytes * 8 apart.
+constexpr uint32_t kSwizzleMode = kBoxBytes == 128 ? 2u : 4u;
+constexpr uint32_t kSbo = 8u * kBoxBytes;
 constexpr int kFirstEpiWarp = 2 + kSfWarps;
 // tcgen05.mma instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1),
 // K-major, N = 256 (>> 3), UE4M3 scales (bit 23 = 0), M = 128 (>> 4).
@@ -60,10 +66,10 @@ constexpr uint32_t kIdescMx = kIdesc | (1u << 23);
 constexpr long long kDrainCycles = 2000000000ll;
 
 struct Shared {
-    uint64_t tma_ready[kStages];  // packed codes of the stage landed (tx)
-    uint64_t sf_landed[kStages];  // scale tiles of the stage landed (tx)
-    uint64_t pair_ready[2];       // both stages of a pair loaded, scales in TMEM
-    uint64_t empty[kStages];      // MMAs of the stage done (commit)
+    uint64_t tma_ready[kNS];      // packed codes of the stage landed (tx)
+    uint64_t sf_landed[kNS];      // scale tiles of the stage landed (tx)
+    uint64_t ready[kReadyBufs];   // every stage of a group loaded, scales in TMEM
+    uint64_t empty[kNS];          // MMAs of the stage done (commit)
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -137,7 +143,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Shared *sh = reinterpret_cast<Shared *>(smem + kStages * kStageBytes);
+    Shared *sh = reinterpret_cast<Shared *>(smem + kNS * kStageBytes);
+    static_assert(sizeof(Shared) <= 512, "barrier block");
     int *s_off = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(sh) + 512);
     int *s_rows = s_off + (kMaxGroups + 1);
 
@@ -145,12 +152,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kNS; ++s) {
             mbar_init(&sh->tma_ready[s], 1);
             mbar_init(&sh->sf_landed[s], 1);
             mbar_init(&sh->empty[s], 1);
         }
-        for (int j = 0; j < 2; ++j) mbar_init(&sh->pair_ready[j], kSfWarps);
+        for (int j = 0; j < kReadyBufs; ++j) mbar_init(&sh->ready[j], kSfWarps);
         mbar_init(&sh->acc_full, 1);
         mbar_init(&sh->acc_empty, kEpiWarps);
         mbar_init(&sh->drain, 1);
@@ -194,10 +201,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     const int splits = kSplit ? p.splits : 1;
     const int tiles = tiles_mn * splits;
     const int kblocks = p.k / 64;                    // 64-value MMA steps
-    const int ktiles = (kblocks + 3) / 4;            // 256-value stages
+    const int ktiles = (kblocks + kKB - 1) / kKB;    // kSK-value stages
     // one 128-row band of scale tiles; a tile covers 64 (NVFP4) or 128 (MX) K
     const int64_t sf_rowblock_bytes = (int64_t)(kMx ? (kblocks + 1) / 2 : kblocks) * 512;
-    constexpr int64_t kSfStageStride = kMx ? 1024 : 2048;      // scale bytes per band and stage
+    constexpr int64_t kSfStageStride = (kMx ? kKB / 2 : kKB) * 512;   // scale bytes per band and stage
+    constexpr int kSfBand = kKB * 512;              // smem offset of the second W band
     auto krange = [&](int tile, int &kt0, int &kt1) {
         if (!kSplit) {
             kt0 = 0;
@@ -224,9 +232,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t armed_phase[kStages];
-            bool armed[kStages];
-            for (int s = 0; s < kStages; ++s) armed[s] = false;
+            uint32_t armed_phase[kNS];
+            bool armed[kNS];
+            for (int s = 0; s < kNS; ++s) armed[s] = false;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
                 const TileInfo t = tile_info(kSplit ? tile % tiles_mn : tile, mtiles, ntiles, p, s_off, s_rows);
@@ -237,7 +245,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                 krange(tile, kt0, kt1);
                 for (int kt = kt0; kt < kt1; ++kt) {
                     if (!wait_or_abort(&sh->empty[stage], phase ^ 1, sh, p)) { ok = false; break; }
-                    const int nkb = min(4, kblocks - 4 * kt);
+                    const int nkb = min(kKB, kblocks - kKB * kt);
                     const uint32_t sf_bytes = (uint32_t)(kMx ? (nkb + 1) / 2 : nkb) * 512;
                     uint8_t *sA = smem + stage * kStageBytes;
                     uint8_t *sB = sA + kStageA;
@@ -250,13 +258,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     bulk_load(sSFA, p.sfa + sfa_base + (int64_t)kt * kSfStageStride, sf_bytes,
                               &sh->sf_landed[stage]);
                     for (int h = 0; h < halves; ++h)
-                        bulk_load(sSFB + h * 2048,
+                        bulk_load(sSFB + h * kSfBand,
                                   p.sfb + (int64_t)(brb + h) * sf_rowblock_bytes +
                                       (int64_t)kt * kSfStageStride,
                                   sf_bytes, &sh->sf_landed[stage]);
-                    tma_load_2d(sA, &tmA, &sh->tma_ready[stage], kt * (kBK / 2), t.a_row0);
-                    tma_load_2d(sB, &tmB, &sh->tma_ready[stage], kt * (kBK / 2), t.b_row0);
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                    tma_load_2d(sA, &tmA, &sh->tma_ready[stage], kt * kBoxBytes, t.a_row0);
+                    tma_load_2d(sB, &tmB, &sh->tma_ready[stage], kt * kBoxBytes, t.b_row0);
+                    if (++stage == kNS) { stage = 0; phase ^= 1; }
                 }
             }
             // Let every copy already issued land before the CTA can exit: after
@@ -264,7 +272,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             // on the last stages armed; in a normal run those phases have
             // completed and each check returns at once.
             {
-                for (int s = 0; s < kStages; ++s) {
+                for (int s = 0; s < kNS; ++s) {
                     if (!armed[s]) continue;
                     const long long t0 = clock64();
                     while (!mbar_try_wait(&sh->sf_landed[s], armed_phase[s]) &&
@@ -279,11 +287,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     } else if (warp >= 2 && warp < kFirstEpiWarp) {
         // -------------------------------------------------- scale writers
         // TMEM scale columns of stage s start at kAccCols + s * kSfCols: A at
-        // +4*kb (K block kb), W at +16+8*kb.  Lane i of every 32-lane quarter
-        // holds, in column c, the four scales of row 32c+i: exactly row i of
-        // the 512-byte 128x4 scale tile (16 bytes = four columns).  Every
-        // quarter needs the full set, so each writer warp stores all 48
-        // columns of its own 32 lanes.
+        // +4*kb (K block kb), W at +kSfbCol0+8*kb.  Lane i of every 32-lane
+        // quarter holds, in column c, the four scales of row 32c+i: exactly
+        // row i of the 512-byte 128x4 scale tile (16 bytes = four columns).
+        // Every quarter needs the full set, so each writer warp stores all
+        // kSfCols columns of its own 32 lanes.
         const int quarter = warp & 3;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         int stage = 0;
@@ -299,37 +307,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             auto pick = [](uint32_t w, int kb) -> uint32_t {
                 return kMx ? (w >> (16 * (kb & 1))) & 0xFFFFu : w;
             };
-            uint32_t v[16];
+            uint32_t v[kKB * 4];
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
+            for (int kb = 0; kb < kKB; ++kb) {
                 const int tile = kMx ? kb / 2 : kb;
                 const uint4 w = *reinterpret_cast<const uint4 *>(sSFA + 512 * tile + 16 * lane);
                 v[4 * kb] = pick(w.x, kb); v[4 * kb + 1] = pick(w.y, kb);
                 v[4 * kb + 2] = pick(w.z, kb); v[4 * kb + 3] = pick(w.w, kb);
             }
-            tmem_st_32x32b_x16(col, v);
-            uint32_t u[32];
+            tmem_st_32x32b(col, v);
+            uint32_t u[kKB * 8];
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
+            for (int kb = 0; kb < kKB; ++kb) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int tile = kMx ? kb / 2 : kb;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(sSFB + 2048 * h + 512 * tile + 16 * lane);
+                    const uint4 w = *reinterpret_cast<const uint4 *>(sSFB + kSfBand * h + 512 * tile + 16 * lane);
                     const int o = 8 * kb + 4 * h;
                     u[o] = pick(w.x, kb); u[o + 1] = pick(w.y, kb);
                     u[o + 2] = pick(w.z, kb); u[o + 3] = pick(w.w, kb);
                 }
             }
-            tmem_st_32x32b_x32(col + 16, u);
+            tmem_st_32x32b(col + kSfbCol0, u);
             if (!wait_or_abort(&sh->tma_ready[stage], phase, sh, p)) break;
-            if ((g & 1) || g == total_k - 1) {
+            if ((g % kGrp) == kGrp - 1 || g == total_k - 1) {
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                const int pj = g >> 1;
-                if (lane == 0) mbar_arrive(&sh->pair_ready[pj & 1]);
+                if (lane == 0) mbar_arrive(&sh->ready[(g / kGrp) % kReadyBufs]);
             }
-            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            if (++stage == kNS) { stage = 0; phase ^= 1; }
         }
         tmem_st_wait();   // no store in flight when TMEM is released (abort path)
     } else if (warp == 1) {
@@ -337,13 +344,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         if (lane == 0) {
             // Descriptors are linear in the start address (field = address >> 4),
             // so stage s and K block kb are plain additions to the stage-0 value.
-            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
-            const uint64_t bdesc0 = smem_desc(smem_u32(smem) + kStageA, 16, 1024, 2);
+            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, kSbo, kSwizzleMode);
+            const uint64_t bdesc0 = smem_desc(smem_u32(smem) + kStageA, 16, kSbo, kSwizzleMode);
             static_assert(kStageBytes % 16 == 0, "stage stride must be 16-byte granular");
             // The tensor pipe queues very few MMAs, so everything between two
             // MMA issues is on the critical path: per-stage bookkeeping below
-            // is incremental (no divisions), and the MMA waits once per pair.
-            const int last_nkb = kblocks - 4 * (ktiles - 1);
+            // is incremental (no divisions), and the MMA waits once per group.
+            const int last_nkb = kblocks - kKB * (ktiles - 1);
             uint32_t acc_phase = 0;
             int stage = 0;
             int mma_tile = blockIdx.x, kt0, kt1;           // current tile and its stage range
@@ -352,9 +359,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             uint32_t stage_off = 0;                       // stage * kStageBytes / 16
             uint32_t sfa = tmem + kAccCols;               // stage's TMEM scale columns
             for (int g = 0; g < total_k; ++g) {
-                if ((g & 1) == 0) {
-                    const int pj = g >> 1;
-                    if (!wait_or_abort(&sh->pair_ready[pj & 1], (uint32_t)(pj >> 1) & 1u, sh, p))
+                if (g % kGrp == 0) {
+                    const int j = g / kGrp;
+                    if (!wait_or_abort(&sh->ready[j % kReadyBufs], (uint32_t)(j / kReadyBufs) & 1u, sh, p))
                         break;
                     tc_fence_after();
                 }
@@ -366,16 +373,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                 auto mma = [&](int kb, uint32_t acc) {
                     if (kMx)
                         mma_mxf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
-                                 kIdescMx, sfa + 4 * kb, sfa + 16 + 8 * kb, acc);
+                                 kIdescMx, sfa + 4 * kb, sfa + kSfbCol0 + 8 * kb, acc);
                     else
                         mma_nvf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
-                                 kIdesc, sfa + 4 * kb, sfa + 16 + 8 * kb, acc);
+                                 kIdesc, sfa + 4 * kb, sfa + kSfbCol0 + 8 * kb, acc);
                 };
-                if (kt != ktiles - 1 || last_nkb == 4) {
+                if (kt != ktiles - 1 || last_nkb == kKB) {
                     mma(0, first);
-                    mma(1, 1u);
-                    mma(2, 1u);
-                    mma(3, 1u);
+#pragma unroll
+                    for (int kb = 1; kb < kKB; ++kb) mma(kb, 1u);
                 } else {
                     for (int kb = 0; kb < last_nkb; ++kb) mma(kb, (kt != kt0 || kb != 0) ? 1u : 0u);
                 }
@@ -389,7 +395,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                 } else {
                     ++kt;
                 }
-                if (++stage == kStages) {
+                if (++stage == kNS) {
                     stage = 0;
                     stage_off = 0;
                     sfa = tmem + kAccCols;

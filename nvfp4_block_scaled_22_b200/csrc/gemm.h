@@ -7,25 +7,65 @@
 
 namespace nvfp4 {
 
-// Block-scaled GEMM tiling: 128 x 256 output tile; each pipeline stage
-// holds 256 K-values (one 128-byte swizzle column of packed codes).  The
-// MMA issuer takes stages in pairs, synchronising once per eight MMAs.
+// Block-scaled GEMM tiling: 128 x 256 output tile per CTA.
 constexpr int kBM = 128;
 constexpr int kBN = 256;
-constexpr int kBK = 256;                         // K values per stage
-constexpr int kBoxK = 256;                       // K values per TMA box (128 bytes)
-constexpr int kStages = 4;
-constexpr int kStageA = kBM * kBK / 2;           // 16 KiB
-constexpr int kStageB = kBN * kBK / 2;           // 32 KiB
-constexpr int kStageSFA = kBM * kBK / 16;        // 2 KiB: four 512-byte 128x4 scale tiles
-constexpr int kStageSFB = kBN * kBK / 16;        // 4 KiB: two 128-row bands
+
+// Pipeline of the single-CTA kernel: each stage holds kSK K-values (one TMA
+// box row of kSK/2 bytes, 128- or 64-byte swizzle), kNS stages in shared
+// memory, and the MMA issuer waits once per kGrp stages.  Measured on B200:
+// with 64-byte swizzle rows (kSK = 128) the tensor core takes about three
+// times as long per MMA as with 128-byte rows, although the data is ready
+// earlier, so the default keeps 256-value stages.
+#ifndef NVFP4_GEMM_STAGE_K
+#define NVFP4_GEMM_STAGE_K 256
+#endif
+#ifndef NVFP4_GEMM_STAGES
+#define NVFP4_GEMM_STAGES 4
+#endif
+#ifndef NVFP4_GEMM_GROUP
+#define NVFP4_GEMM_GROUP 2
+#endif
+constexpr int kSK = NVFP4_GEMM_STAGE_K;
+constexpr int kNS = NVFP4_GEMM_STAGES;
+constexpr int kGrp = NVFP4_GEMM_GROUP;
+constexpr int kKB = kSK / 64;                    // 64-value MMA steps per stage
+constexpr int kBoxBytes = kSK / 2;               // TMA box row (bytes of packed codes)
+constexpr int kStageA = kBM * kSK / 2;
+constexpr int kStageB = kBN * kSK / 2;
+constexpr int kStageSFA = kBM * kSK / 16;        // kKB 512-byte 128x4 scale tiles
+constexpr int kStageSFB = kBN * kSK / 16;        // two 128-row bands of kKB tiles
 constexpr int kStageBytes = kStageA + kStageB + kStageSFA + kStageSFB;
+constexpr int kReadyBufs = kNS / kGrp;           // one ready barrier per group slot of the ring
+static_assert(kSK == 128 || kSK == 256, "stage K must fill a 64- or 128-byte swizzle row");
+static_assert(kNS % kGrp == 0, "stages must form whole groups");
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 constexpr int kSfWarps = 4;                      // write block scales into TMEM
 constexpr int kEpiWarps = 8;                     // two per TMEM lane quarter
 constexpr int kMaxGroups = 512;
 constexpr int kGemmThreads = 32 * (2 + kSfWarps + kEpiWarps);   // 448
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ +
+constexpr int kGemmSmemBytes = kNS * kStageBytes + 1024 /*align*/ + 512 /*barriers*/ +
                                2 * (kMaxGroups + 1) * 4 /*group tables*/;
+static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kBN + kNS * kKB * 12 <= 512, "accumulator + scale columns fit TMEM");
+
+// Pipeline of the CTA-pair kernel (per CTA: 128 rows of A, 128 of W's 256,
+// and the scales of all 256 W rows): kPSK K-values per stage, kPNS stages,
+// the leader's MMA issuer waits once per kPGrp stages.
+#ifndef NVFP4_PAIR_STAGE_K
+#define NVFP4_PAIR_STAGE_K 256
+#endif
+#ifndef NVFP4_PAIR_STAGES
+#define NVFP4_PAIR_STAGES 5
+#endif
+#ifndef NVFP4_PAIR_GROUP
+#define NVFP4_PAIR_GROUP 1
+#endif
+constexpr int kPSK = NVFP4_PAIR_STAGE_K;
+constexpr int kPNS = NVFP4_PAIR_STAGES;
+constexpr int kPGrp = NVFP4_PAIR_GROUP;
+static_assert(kPSK == 128 || kPSK == 256, "stage K must fill a 64- or 128-byte swizzle row");
+static_assert(kPNS % kPGrp == 0, "stages must form whole groups");
 
 struct GemmParams {
     const uint8_t *sfa;       // A scales, 128x4 layout
@@ -50,9 +90,22 @@ struct GemmParams {
     long long timeout_cycles;
 };
 
+// TMA box of the single-CTA kernel's operands: kBoxBytes x rows, swizzled
+// to match the MMA descriptors.
+constexpr int kSingleBoxBytes = kBoxBytes;
+constexpr int kPairBoxBytes = kPSK / 2;
+
 // mx: MXFP4 operands (UE8M0 scales per 32 values, no tensor scales).
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t stream, bool mx = false);
+
+// Dense GEMM with few rows of A (m <= kSwapMaxRows): W on the MMA's M side,
+// A's rows (padded to a multiple of 16) on its N side.  tmW: 128-row boxes of
+// W; tmX: boxes of A's padded row count; both 128-byte rows.
+constexpr int kSwapMaxRows = 64;
+constexpr int kSwapThreads = 32 * (2 + kSfWarps + 4);   // 320
+cudaError_t launch_gemm_swap(const CUtensorMap &tmW, const CUtensorMap &tmX, const GemmParams &p,
+                             int grid, cudaStream_t stream);
 
 // Dense GEMM on CTA pairs (256x256 tiles); tmB must use 128-row boxes.
 cudaError_t launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,

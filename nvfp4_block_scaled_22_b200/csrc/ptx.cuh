@@ -326,6 +326,24 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         : "memory");
 }
 
+// Each thread of the warp writes 8 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+        :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+           "r"(v[6]), "r"(v[7])
+        : "memory");
+}
+
+// 8, 16 or 32 consecutive columns per lane, picked by the array's size.
+template <int N>
+__device__ __forceinline__ void tmem_st_32x32b(uint32_t taddr, const uint32_t (&v)[N]) {
+    static_assert(N == 8 || N == 16 || N == 32, "tcgen05.st shape");
+    if constexpr (N == 8) tmem_st_32x32b_x8(taddr, v);
+    else if constexpr (N == 16) tmem_st_32x32b_x16(taddr, v);
+    else tmem_st_32x32b_x32(taddr, v);
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -226,3 +226,28 @@ def test_split_k_against_oracle_and_unsplit(m, n, k):
     tol = gemm_tolerance(ref, ab)
     for d in (d1, d0):
         assert np.all(np.abs(bf16_to_f64(d).ravel() - ref) <= tol)
+
+
+@pytest.mark.parametrize("m", [1, 15, 16, 17, 33, 48, 64])
+@pytest.mark.parametrize("n,k", [(2048, 5120), (300, 192), (128, 64), (1000, 1088)])
+def test_small_m_swapped_operands(m, n, k):
+    """Few rows of A run with W on the MMA's 128-row side and A's rows
+    (padded to a multiple of 16) on its N side, split over K when the
+    workspace holds the FP32 slices.  Every output against the oracle, with
+    and without splits; the split result is the same on every call."""
+    qa, ra = _quant_both(_rand(m, k, 11 * m + n + k), f"small-M A {m}x{k}")
+    qw, rw = _quant_both(_rand(n, k, 7 * m + 3 * n + k, 0.02), f"small-M W {n}x{k}")
+    ii, jj = np.meshgrid(np.arange(m), np.arange(n), indexing="ij")
+    ref, ab = oracle.gemm_ref(ra, rw, ii.ravel(), jj.ravel())
+    tol = gemm_tolerance(ref, ab)
+    big, small = nb.Workspace(DEV, 64 << 20), nb.Workspace(DEV, 256)
+    d1 = nb.nvfp4_gemm(qa, qw, workspace=big)
+    d2 = nb.nvfp4_gemm(qa, qw, workspace=big)
+    d0 = nb.nvfp4_gemm(qa, qw, workspace=small)
+    torch.cuda.synchronize()
+    assert nb.nvfp4_check_status(big) == 0 and nb.nvfp4_check_status(small) == 0
+    assert torch.equal(d1, d2)
+    for d in (d1, d0):
+        err = np.abs(bf16_to_f64(d).ravel() - ref)
+        bad = np.nonzero(err > tol)[0]
+        assert bad.size == 0, f"{bad.size} outside tolerance, first (i,j)={ii.ravel()[bad[:4]]},{jj.ravel()[bad[:4]]}"

@@ -78,8 +78,11 @@ def test_dense_gemm_timeout_then_clean(m, n, k):
     _timed_out_then_clean(lambda: nb.nvfp4_gemm(qa, qw, workspace=ws), _full_check(ra, rw, m, n), ws)
 
 
-def test_split_k_gemm_timeout_then_clean():
-    m, n, k = 16, 2048, 5120                         # split-K instance at the small-M FFN shape
+@pytest.mark.parametrize("m", [16, 100])
+def test_small_m_gemm_timeout_then_clean(m):
+    """m = 16: the swapped-operand kernel with K splits; m = 100: the split-K
+    instance of the 128x256 kernel."""
+    n, k = 2048, 5120
     qa, ra = _quant(_rand(m, k, 3), "A")
     qw, rw = _quant(_rand(n, k, 4, 0.02), "W")
     ws = nb.Workspace(DEV, 64 << 20)
