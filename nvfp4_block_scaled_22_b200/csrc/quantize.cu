@@ -183,14 +183,15 @@ __device__ __forceinline__ void emit_block(const EncodeParams &p, const EncodeSh
 }
 
 // Source row of output row `row` (gathered or not); load = false for band
-// padding rows, gathered padding rows (-1) and invalid map entries.
-__device__ __forceinline__ int64_t source_row(const EncodeParams &p, int64_t row, bool &real,
-                                              bool &load) {
+// padding rows, gathered padding rows (-1) and invalid map entries.  `mapped`
+// is the row map's entry for `row`, already loaded by the caller.
+__device__ __forceinline__ int64_t source_row(const EncodeParams &p, int64_t row, int32_t mapped,
+                                              bool &real, bool &load) {
     real = row < p.rows;
     load = real;
     int64_t src = row;
     if (real && p.gather != nullptr) {
-        src = p.gather[row];
+        src = mapped;
         if (src >= p.src_rows) {             // out-of-range map entry: zero row + status
             set_status(p.status, ST_INVALID_ARG);
             src = -1;
@@ -229,12 +230,22 @@ __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     if (!kNarrow) {
         // Wide rows: a task is kChunkBlocks consecutive blocks of one row,
         // lane l taking blocks l, l+32, l+64, l+96; addresses once per task.
+        // With a row map, the next task's map entry is loaded one task ahead
+        // so that its latency overlaps this task's loads.
         const uint32_t chunks = (groups + kUnroll - 1) / kUnroll;
-        for (TaskWalk w(warp_id, warps, chunks); w.row < sh.rows_out; w.next()) {
+        TaskWalk w(warp_id, warps, chunks);
+        int32_t map_next = (p.gather != nullptr && w.row < p.rows) ? __ldg(p.gather + w.row) : 0;
+        for (; w.row < sh.rows_out; w.next()) {
             const int64_t row = w.row;
+            const int32_t mapped = map_next;
+            if (p.gather != nullptr) {
+                TaskWalk nx = w;
+                nx.next();
+                if (nx.row < p.rows) map_next = __ldg(p.gather + nx.row);
+            }
             const int64_t c0 = (int64_t)w.seg * kChunkBlocks + lane;   // this lane's first block
             bool real, load;
-            const int64_t src = source_row(p, row, real, load);
+            const int64_t src = source_row(p, row, mapped, real, load);
             const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + src * p.ld + c0 * 16);
             uint4 va[kUnroll], vb[kUnroll];
 #pragma unroll
