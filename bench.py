@@ -444,16 +444,18 @@ def workload_line(name, args, device):
             return q, g
         wu, gu = stacked("up", I, H)
         wd, gd = stacked("down", H, I)
-        gx = torch.zeros(1, dtype=torch.float32, device=device)
-        qx = nb.NVFP4Tensor.empty(r.padded_rows, H, device=device, global_scale=gx)
+        qxs = nb.NVFP4Tensor.empty(inputs.MOE_TOKENS, H, device=device)      # X, quantized once
+        qx = nb.NVFP4Tensor.empty(r.padded_rows, H, device=device)
         hbuf = torch.empty((r.padded_rows, I), dtype=torch.bfloat16, device=device)
         qh = nb.NVFP4Tensor.empty(r.padded_rows, I, device=device)
         y = torch.empty((r.padded_rows, H), dtype=torch.bfloat16, device=device)
         ev = {}
 
         def step(mark=False):
-            nb.nvfp4_global_scale(x, out=gx, workspace=ws)
-            nb.nvfp4_quantize_gather(x, gather, out=qx, global_supplied=True, workspace=ws)
+            # each token's row is quantized once (X's tensor scale), then its
+            # NVFP4 bytes are gathered into its 8 expert slots
+            nb.nvfp4_quantize(x, out=qxs, workspace=ws)
+            nb.nvfp4_gather_rows(qxs, gather, out=qx, workspace=ws)
             nb.nvfp4_grouped_gemm(slot, rows, qx, wu, gu, I, out=hbuf, workspace=ws)
             nb.nvfp4_quantize_gather(hbuf, ident, out=qh, workspace=ws)
             if mark:

@@ -134,6 +134,27 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, int64_t ld, const nvfp4_ten
                             int32_t global_supplied, void *workspace,
                             size_t workspace_bytes, void *stream);
 
+/* Row gather of an NVFP4 tensor, for MoE expert batches: output row r is
+ * source row d_gather[r] -- its packed codes and its block scales -- and
+ * d_gather[r] == -1 makes row r a zero padding row (codes and scales 0);
+ * *out->global = *src->global.  Quantization is row-wise once the tensor
+ * scale is fixed, so gathering the rows of nvfp4_quantize(x) gives the same
+ * bytes as nvfp4_quantize_gather(x, d_gather, global_supplied with x's
+ * tensor scale) while moving 0.5625 instead of 2 bytes per gathered value.
+ * ("NVIDIA shrank GLM-5.2 to 4 bits", section 1: the MoE expert linears take
+ * NVFP4 activations; section 2: each token goes to 8 of 256 experts.)
+ * src      : NVFP4 tensor, src->rows x src->cols, either scale layout.
+ * d_gather : device int32[out->rows].  An entry >= src->rows is not read:
+ *            its row is zeroed and NVFP4_ERR_INVALID_ARG is recorded in the
+ *            status word.
+ * out      : out->cols == src->cols; either scale layout (the 128x4 layout's
+ *            padding rows are zeroed).
+ * workspace: only its 256-byte status block is used.
+ * Errors: argument checks synchronously. */
+NVFP4_API nvfp4_status nvfp4_gather_rows(const nvfp4_tensor *src, const int32_t *d_gather,
+                                         const nvfp4_tensor *out, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
 /* Tensor scale only: *d_global = RN(2688 / max|x|) over a rows x cols BF16
  * matrix with pitch ld (1.0 if all zero).  Same status rules as
  * nvfp4_quantize.  Lets a caller share one g between tensors or take g from

@@ -15,7 +15,9 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+# The in-tree build; NVFP4_LIBRARY may name another build of the same C ABI
+# (for example one compiled with a different pipeline geometry).
+LIB_PATH = os.environ.get("NVFP4_LIBRARY") or os.path.join(HERE, "libnvfp4.so")
 
 SF_SWIZZLED = 0
 SF_LINEAR = 1
@@ -37,7 +39,7 @@ EXPORTED = (
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
     "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
     "nvfp4_gemm_mx", "nvfp4_moe_combine", "nvfp4_dequantize_fp8", "nvfp4_quantize_swiglu",
-    "nvfp4_attention_decode",
+    "nvfp4_attention_decode", "nvfp4_gather_rows",
 )
 
 
@@ -80,6 +82,7 @@ def lib() -> C.CDLL:
             "nvfp4_status_string": (C.c_char_p, [C.c_int]),
             "nvfp4_version": (i32, []),
             "nvfp4_launch_count": (i64, []),
+            "nvfp4_gather_rows": (C.c_int, [T, vp, T, vp, sz, vp]),
             "nvfp4_set_wait_limit_cycles": (C.c_longlong, [C.c_longlong]),
             "nvfp4_set_gemm_pairs": (i32, [i32]),
             "nvfp4_quantize_noalloc": (C.c_int, [vp, i64, T, i32, vp]),
@@ -402,6 +405,21 @@ def nvfp4_quantize_swiglu(gate_up: torch.Tensor, out: NVFP4Tensor | None = None,
     t = out.c_struct()
     _check(lib().nvfp4_quantize_swiglu(gate_up.data_ptr(), gate_up.stride(0), C.byref(t), ws.ptr,
                                        ws.nbytes, _stream(stream)), "nvfp4_quantize_swiglu")
+    return out
+
+
+def nvfp4_gather_rows(src: NVFP4Tensor, gather: torch.Tensor, out: NVFP4Tensor | None = None,
+                      layout: int = SF_SWIZZLED, workspace: Workspace | None = None,
+                      stream=None) -> NVFP4Tensor:
+    """Out row r = source row gather[r] (codes and scales), -1 = zero row;
+    the tensor scale is copied.  gather: int32 CUDA tensor."""
+    assert gather.dtype == torch.int32 and gather.is_cuda
+    if out is None:
+        out = NVFP4Tensor.empty(gather.numel(), src.cols, layout, src.codes.device)
+    ws = workspace or default_workspace(src.codes.device)
+    cs, co = src.c_struct(), out.c_struct()
+    _check(lib().nvfp4_gather_rows(C.byref(cs), gather.data_ptr(), C.byref(co), ws.ptr, ws.nbytes,
+                                   _stream(stream)), "nvfp4_gather_rows")
     return out
 
 

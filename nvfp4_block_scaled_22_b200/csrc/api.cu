@@ -24,6 +24,13 @@ constexpr size_t kStatusBytes = 256;          // status word + reserved
 constexpr int kMaxPartials = 1024;            // CTAs of the amax pass
 constexpr long long kDefaultTimeoutCycles = 2000000000ll;   // ~1 s at 1.9 GHz
 constexpr int64_t kFlatCols = 2048;           // row width for contiguous row-major-scale tensors
+// Most K splits of the few-row GEMM: each split costs an accumulator
+// hand-off and FP32 partials; measured at M = 16, N = 20480, K = 5120, a cap
+// of 4 beats 16 (29.7 vs 33.8 us).
+#ifndef NVFP4_SWAP_MAX_SPLITS
+#define NVFP4_SWAP_MAX_SPLITS 4
+#endif
+constexpr int kSwapMaxSplits = NVFP4_SWAP_MAX_SPLITS;
 
 struct DeviceInfo {
     bool checked = false;
@@ -130,6 +137,25 @@ nvfp4_status encode_codes_map(CUtensorMap *m, const void *codes, int64_t rows, i
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Launch a kernel with programmatic stream serialization: it may be
+// scheduled while the previous kernel on the stream finishes, and waits on
+// the device (griddepcontrol.wait) before reading that kernel's results.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3((unsigned)block, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32_t *gather,
                         const nvfp4_tensor *out, int32_t global_supplied, void *ws,
                         cudaStream_t stream, int sms, bool rht = false, uint32_t rht_mask = 0,
@@ -190,8 +216,7 @@ nvfp4_status run_encode(const void *x, int64_t ld, int64_t src_rows, const int32
                   : (narrow ? k_encode_narrow : k_encode));
     int grid = (int)std::min<int64_t>(ceil_div(tasks, 8 * (narrow ? 4 : 1)), 8LL * sms);
     if (grid < 1) grid = 1;
-    kernel<<<grid, 256, 0, stream>>>(p);
-    return launched(cudaGetLastError());
+    return launched(launch_pdl(kernel, grid, 256, 0, stream, p));
 }
 
 // Column-wise quantize (out = NVFP4 of x^T); arguments already validated.
@@ -562,6 +587,7 @@ nvfp4_status nvfp4_dequantize_mx(const nvfp4_tensor *in, void *y, int64_t ld, vo
     p.cols = in->cols;
     p.y = static_cast<uint16_t *>(y);
     p.ld = ld;
+    p.y_vec32 = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0 && ld % 16 == 0) ? 1 : 0;
     const int64_t tasks = in->rows * ceil_div(in->cols / 32, 32);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
     int grid = (int)std::min<int64_t>(ceil_div(tasks, 8), 8LL * sms);
@@ -752,6 +778,45 @@ nvfp4_status nvfp4_quantize_gather(const void *x, int64_t ld, int64_t src_rows,
                       static_cast<cudaStream_t>(stream), sms);
 }
 
+nvfp4_status nvfp4_gather_rows(const nvfp4_tensor *src, const int32_t *d_gather,
+                               const nvfp4_tensor *out, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    nvfp4_status st = check_tensor(src);
+    if (st != NVFP4_OK) return st;
+    st = check_tensor(out);
+    if (st != NVFP4_OK) return st;
+    if (out->cols != src->cols) return NVFP4_ERR_SHAPE;
+    if (out->rows > 0 && out->cols > 0 && d_gather == nullptr) return NVFP4_ERR_INVALID_ARG;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    GatherParams p;
+    p.src_codes = static_cast<const uint8_t *>(src->codes);
+    p.src_scales = static_cast<const uint8_t *>(src->scales);
+    p.src_global = src->global;
+    p.src_layout = src->sf_layout;
+    p.src_rows = src->rows;
+    p.dst_codes = static_cast<uint8_t *>(out->codes);
+    p.dst_scales = static_cast<uint8_t *>(out->scales);
+    p.dst_global = out->global;
+    p.dst_layout = out->sf_layout;
+    p.rows = out->rows;
+    p.cols = out->cols;
+    p.map = d_gather;
+    p.status = reinterpret_cast<uint32_t *>(workspace);
+    if (out->cols == 0) {           // only the tensor scale moves
+        p.rows = 0;
+    }
+    const int64_t rows_pad = out->sf_layout == NVFP4_SF_SWIZZLED_128x4 ? ceil_div(out->rows, 128) * 128
+                                                                      : out->rows;
+    int grid = (int)std::min<int64_t>(ceil_div(std::max<int64_t>(rows_pad, 1), 8), 16LL * sms);
+    if (grid < 1) grid = 1;
+    k_gather_rows<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched(cudaGetLastError());
+}
+
 nvfp4_status nvfp4_global_scale(const void *x, int64_t ld, int64_t rows, int64_t cols,
                                 float *d_global, void *workspace, size_t workspace_bytes,
                                 void *stream) {
@@ -804,6 +869,7 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor *in, void *y, int64_t ld, void 
     p.cols = in->cols;
     p.y = static_cast<uint16_t *>(y);
     p.ld = ld;
+    p.y_vec32 = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0 && ld % 16 == 0) ? 1 : 0;
     const int64_t tasks = decode_tasks(p.rows, p.cols);
     if (tasks >= (int64_t)UINT32_MAX - 65536LL * 1024) return NVFP4_ERR_SHAPE;
     const bool narrow = tasks_are_groups(p.cols);
@@ -853,7 +919,7 @@ static nvfp4_status gemm_swap(const nvfp4_tensor *A, const nvfp4_tensor *W, int6
     const int ktiles = (int)ceil_div(k / 64, 4);
     int64_t best_cost = ceil_div(ntiles, sms) * ktiles;
     if (n % 16 == 0 && p.d_vec16) {
-        for (int sp = 2; sp <= std::min(16, ktiles); ++sp) {
+        for (int sp = 2; sp <= std::min(kSwapMaxSplits, ktiles); ++sp) {
             const int64_t cost = ceil_div(ntiles * sp, sms) * ceil_div(ktiles, sp) + 1;
             const size_t need = kStatusBytes + (size_t)sp * (size_t)m * (size_t)n * 4;
             if (cost < best_cost && need <= workspace_bytes) {
@@ -869,9 +935,8 @@ static nvfp4_status gemm_swap(const nvfp4_tensor *A, const nvfp4_tensor *W, int6
     if (st != NVFP4_OK || p.splits == 1) return st;
     const int64_t quads = m * (n / 4);
     const int fgrid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(quads, 256), 4LL * sms));
-    k_splitk_finalize<<<fgrid, 256, 0, stream>>>(p.partial, p.splits, (int)m, (int)n, p.ga, p.gw,
-                                                 p.d, p.ldd);
-    return launched(cudaGetLastError());
+    return launched(launch_splitk_finalize(p.partial, p.splits, (int)m, (int)n, p.ga, p.gw, p.d,
+                                           p.ldd, fgrid, stream));
 }
 
 static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
@@ -974,9 +1039,8 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     if (st != NVFP4_OK || p.splits == 1) return st;
     const int64_t quads = m * (n / 4);
     const int fgrid = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(quads, 256), 4LL * sms));
-    k_splitk_finalize<<<fgrid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        p.partial, p.splits, (int)m, (int)n, p.ga, p.gw, p.d, p.ldd);
-    return launched(cudaGetLastError());
+    return launched(launch_splitk_finalize(p.partial, p.splits, (int)m, (int)n, p.ga, p.gw, p.d,
+                                           p.ldd, fgrid, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, void *D, int64_t ldd,

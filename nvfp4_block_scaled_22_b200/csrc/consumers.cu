@@ -49,9 +49,10 @@ __device__ __forceinline__ float exp_ref(float x) {
     return __fmul_rn(p, __uint_as_float((uint32_t)((int)n + 127) << 23));   // 2^n, |n| <= 126
 }
 
-// h = RN(RN(g * RN(1 / RN(1 + exp(-g)))) * u).
+// h = RN(RN(g * RN(1 / RN(1 + exp(-g)))) * u).  RN(1 / d) is the correctly
+// rounded reciprocal (d >= 1, so the result is normal or NaN).
 __device__ __forceinline__ float swiglu(float g, float u) {
-    const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_ref(-g)));
+    const float s = __frcp_rn(__fadd_rn(1.0f, exp_ref(-g)));
     return __fmul_rn(__fmul_rn(g, s), u);
 }
 

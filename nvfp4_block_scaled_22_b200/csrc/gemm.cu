@@ -170,6 +170,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         tmem_alloc(&sh->tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    // Launched with programmatic stream serialization: the setup above
+    // overlaps the previous kernel (e.g. the quantize of A); every global
+    // input is read after this wait.
+    grid_dependency_wait();
     if (p.groups > 0) {
         for (int i = threadIdx.x; i <= p.groups; i += blockDim.x) s_off[i] = p.slot_offsets[i];
         for (int i = threadIdx.x; i < p.groups; i += blockDim.x) s_rows[i] = p.group_rows[i];
@@ -177,6 +181,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (kSplit) grid_dependents_launch();   // the finalize may become resident and wait
     const uint32_t tmem = sh->tmem_base;
     if (p.groups > 0 && threadIdx.x == 0) {
         // Offsets must start at 0, rise in multiples of 128 within A's rows,
@@ -298,6 +303,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
         uint32_t phase = 0;
         for (int g = 0; g < total_k; ++g) {
             if (!wait_or_abort(&sh->sf_landed[stage], phase, sh, p)) break;
+            if (kSfCp && !kMx) {
+                // scales reach TMEM by the MMA issuer's tcgen05.cp: only
+                // signal that the stage's codes and scale tiles landed
+                if (!wait_or_abort(&sh->tma_ready[stage], phase, sh, p)) break;
+                if ((g % kGrp) == kGrp - 1 || g == total_k - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh->ready[(g / kGrp) % kReadyBufs]);
+                }
+                if (++stage == kNS) { stage = 0; phase ^= 1; }
+                continue;
+            }
             const uint8_t *sSFA = smem + stage * kStageBytes + kStageA + kStageB;
             const uint8_t *sSFB = sSFA + kStageSFA;
             const uint32_t col = lane_base + kAccCols + (uint32_t)stage * kSfCols;
@@ -370,6 +386,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     tc_fence_after();
                 }
                 const uint32_t first = kt != kt0 ? 1u : 0u;
+                if (kSfCp && !kMx) {
+                    // this stage's scale tiles: A tile kb -> columns 4kb, W band h
+                    // tile kb -> kSfbCol0 + 8kb + 4h; each 512-byte tile is
+                    // 32 rows x 16 bytes (no swizzle, 8-row core matrices 128
+                    // bytes apart), copied to lanes 0-31 of every quarter
+                    const uint32_t sf0 = smem_u32(smem) + (uint32_t)(stage * kStageBytes + kStageA + kStageB);
+#pragma unroll
+                    for (int kb = 0; kb < kKB; ++kb) {
+                        tc_cp_32x128b_x4(sfa + 4 * kb, smem_desc(sf0 + 512 * kb, 128, 128, 0));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_cp_32x128b_x4(sfa + kSfbCol0 + 8 * kb + 4 * h,
+                                             smem_desc(sf0 + kStageSFA + kSfBand * h + 512 * kb, 128, 128, 0));
+                    }
+                }
                 auto mma = [&](int kb, uint32_t acc) {
                     if (kMx)
                         mma_mxf4(tmem, adesc0 + stage_off + 2 * kb, bdesc0 + stage_off + 2 * kb,
@@ -452,17 +483,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                     : __frcp_rn(__fmul_rn(*p.ga, p.gw[tile_info(tile, mtiles, ntiles, p, s_off, s_rows).group]));
             if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
+            // Four 32-column loads per warp: each wait is a TMEM round trip
+            // during which the next tile's MMAs cannot start.
             uint32_t o[64];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t r[16];
-                tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) +
-                                       (uint32_t)(chalf * 128 + 16 * c), r);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                       (uint32_t)(chalf * 128 + 32 * c), r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    o[8 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                   __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                for (int i = 0; i < 16; ++i)
+                    o[16 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                    __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
             }
             tc_fence_before();
             __syncwarp();
@@ -493,6 +526,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
 __global__ void __launch_bounds__(256) k_splitk_finalize(const float *partial, int splits, int m,
                                                          int n, const float *ga, const float *gw,
                                                          uint16_t *d, int64_t ldd) {
+    grid_dependency_wait();   // the GEMM that wrote the slices (launched ahead of it)
     const float alpha = __frcp_rn(__fmul_rn(*ga, *gw));
     const int64_t quads = (int64_t)m * (n / 4);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < quads;
@@ -530,6 +564,22 @@ k_gemm_mxf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     gemm_body<true, false>(tmA, tmB, p);
 }
 
+cudaError_t launch_splitk_finalize(const float *partial, int splits, int m, int n, const float *ga,
+                                   const float *gw, uint16_t *d, int64_t ldd, int grid,
+                                   cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_splitk_finalize, partial, splits, m, n, ga, gw, d, ldd);
+}
+
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                         int grid, cudaStream_t stream, bool mx) {
     static bool attr_set[64][3] = {};
@@ -544,8 +594,17 @@ cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const Ge
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev][which] = true;
     }
-    kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tmA, tmB, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kGemmSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
 }
 
 }  // namespace nvfp4

@@ -26,6 +26,14 @@ constexpr int kBN = 256;
 #ifndef NVFP4_GEMM_GROUP
 #define NVFP4_GEMM_GROUP 2
 #endif
+// Block scales into TMEM: 0 = four scale-writer warps read the tiles from
+// shared memory and write every lane quarter with tcgen05.st (each warp
+// reads all of a stage's 6 KiB); 1 = the MMA issuer copies each 512-byte
+// tile once with tcgen05.cp (32x128b, broadcast to the four quarters).
+#ifndef NVFP4_GEMM_SF_CP
+#define NVFP4_GEMM_SF_CP 0
+#endif
+constexpr bool kSfCp = NVFP4_GEMM_SF_CP != 0;
 constexpr int kSK = NVFP4_GEMM_STAGE_K;
 constexpr int kNS = NVFP4_GEMM_STAGES;
 constexpr int kGrp = NVFP4_GEMM_GROUP;
@@ -49,23 +57,8 @@ constexpr int kGemmSmemBytes = kNS * kStageBytes + 1024 /*align*/ + 512 /*barrie
 static_assert(kGemmSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kBN + kNS * kKB * 12 <= 512, "accumulator + scale columns fit TMEM");
 
-// Pipeline of the CTA-pair kernel (per CTA: 128 rows of A, 128 of W's 256,
-// and the scales of all 256 W rows): kPSK K-values per stage, kPNS stages,
-// the leader's MMA issuer waits once per kPGrp stages.
-#ifndef NVFP4_PAIR_STAGE_K
-#define NVFP4_PAIR_STAGE_K 256
-#endif
-#ifndef NVFP4_PAIR_STAGES
-#define NVFP4_PAIR_STAGES 5
-#endif
-#ifndef NVFP4_PAIR_GROUP
-#define NVFP4_PAIR_GROUP 1
-#endif
-constexpr int kPSK = NVFP4_PAIR_STAGE_K;
-constexpr int kPNS = NVFP4_PAIR_STAGES;
-constexpr int kPGrp = NVFP4_PAIR_GROUP;
-static_assert(kPSK == 128 || kPSK == 256, "stage K must fill a 64- or 128-byte swizzle row");
-static_assert(kPNS % kPGrp == 0, "stages must form whole groups");
+// The CTA-pair kernel keeps 256-value stages (128-byte swizzle rows).
+constexpr int kBK = 256;
 
 struct GemmParams {
     const uint8_t *sfa;       // A scales, 128x4 layout
@@ -93,7 +86,7 @@ struct GemmParams {
 // TMA box of the single-CTA kernel's operands: kBoxBytes x rows, swizzled
 // to match the MMA descriptors.
 constexpr int kSingleBoxBytes = kBoxBytes;
-constexpr int kPairBoxBytes = kPSK / 2;
+constexpr int kPairBoxBytes = 128;
 
 // mx: MXFP4 operands (UE8M0 scales per 32 values, no tensor scales).
 cudaError_t launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
@@ -120,6 +113,12 @@ constexpr int64_t kL2SweepBytes = 48ll << 20;
 // order; 256 threads.
 __global__ void k_splitk_finalize(const float *partial, int splits, int m, int n, const float *ga,
                                   const float *gw, uint16_t *d, int64_t ldd);
+
+// k_splitk_finalize launched with programmatic stream serialization: it is
+// scheduled while the split GEMM runs and waits on the device for it.
+cudaError_t launch_splitk_finalize(const float *partial, int splits, int m, int n, const float *ga,
+                                   const float *gw, uint16_t *d, int64_t ldd, int grid,
+                                   cudaStream_t stream);
 
 // Dense GEMMs with at least this many rows run on CTA pairs.
 constexpr int64_t kPairMinRows = 256;

@@ -123,6 +123,7 @@ k_gemm_nvf4_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (p.splits > 1) grid_dependents_launch();   // the finalize may become resident and wait
     const uint32_t tmem = sh->tmem_base;
 
     const int ntiles = (p.n + 127) / 128;

@@ -61,7 +61,23 @@ struct DequantParams {
     int64_t rows, cols;
     uint16_t *y;
     int64_t ld;
+    int32_t y_vec32 = 0;    // 1: y and ld * 2 bytes are 32-byte aligned (one 256-bit store per block)
 };
+
+// Row gather of an NVFP4 tensor (gather.cu).
+struct GatherParams {
+    const uint8_t *src_codes, *src_scales;
+    const float *src_global;
+    int32_t src_layout;
+    int64_t src_rows;
+    uint8_t *dst_codes, *dst_scales;
+    float *dst_global;
+    int32_t dst_layout;
+    int64_t rows, cols;      // output rows, columns (values per row)
+    const int32_t *map;      // output row -> source row, -1 = zero row
+    uint32_t *status;
+};
+__global__ void k_gather_rows(GatherParams p);
 
 __global__ void k_amax(const uint16_t *x, int64_t ld, int64_t rows, int64_t cols,
                        const int32_t *gather, int64_t src_rows, uint32_t *partials,

@@ -104,9 +104,10 @@ __global__ void __launch_bounds__(kThreads) k_dequantize_mx(DequantParams p) {
                 o[4 * h + i] = bf16x2_from_f32(__fmul_rn(v.x, scale), __fmul_rn(v.y, scale));
             }
         }
-        uint4 *yp = reinterpret_cast<uint4 *>(p.y + row * p.ld + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) yp[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        uint16_t *yp = p.y + row * p.ld + c * 32;
+        store_32b(yp, make_uint4(o[0], o[1], o[2], o[3]), make_uint4(o[4], o[5], o[6], o[7]), p.y_vec32 != 0);
+        store_32b(yp + 16, make_uint4(o[8], o[9], o[10], o[11]), make_uint4(o[12], o[13], o[14], o[15]),
+                  p.y_vec32 != 0);
     }
 }
 

@@ -163,6 +163,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// 32 bytes to global memory: one 256-bit store when the address is 32-byte
+// aligned (a warp then writes 1 KiB contiguous per instruction), else two
+// 128-bit stores.
+__device__ __forceinline__ void store_32b(void *y, uint4 o0, uint4 o1, bool vec32) {
+    if (vec32) {
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     :: "l"(y), "r"(o0.x), "r"(o0.y), "r"(o0.z), "r"(o0.w), "r"(o1.x), "r"(o1.y),
+                        "r"(o1.z), "r"(o1.w)
+                     : "memory");
+    } else {
+        reinterpret_cast<uint4 *>(y)[0] = o0;
+        reinterpret_cast<uint4 *>(y)[1] = o1;
+    }
+}
+
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel on the stream is still running; before it touches
+// that kernel's results it waits here for the whole previous grid (and its
+// memory operations).  Without the launch attribute this returns at once.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel on the stream (if launched with programmatic stream
+// serialization) be scheduled before this grid finishes.
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ TMA / bulk
 __device__ __forceinline__ void tma_prefetch_desc(const void *desc) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(desc)) : "memory");

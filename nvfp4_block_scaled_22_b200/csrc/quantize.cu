@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint16_t *__restrict__ 
                                                    uint32_t *__restrict__ partials,
                                                    uint32_t *status) {
     __shared__ uint32_t red[kThreads / 32];
+    grid_dependents_launch();   // the encode pass may be scheduled and wait on the device
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t chunks = cols / 8;  // 16-byte chunks per row
@@ -205,6 +206,11 @@ template <bool kRht, bool kNarrow, bool kSR>
 __device__ __forceinline__ void encode_body(const EncodeParams &p) {
     __shared__ uint32_t red[kThreads / 32];
     __shared__ EncodeTables tab;
+    // Launched with programmatic stream serialization after the amax pass:
+    // let the next kernel (the GEMM) be scheduled as this grid drains, and
+    // wait for the previous kernel's partial maxima before reading them.
+    grid_dependents_launch();
+    grid_dependency_wait();
     float g;
     if (p.global_supplied) {
         g = *p.global;
@@ -504,14 +510,13 @@ __device__ __forceinline__ void dequantize_body(const DequantParams &p) {
                     sb[j] = __ldg(sp + sf_step * j);
                 }
             }
-            uint4 *yp = reinterpret_cast<uint4 *>(p.y + row * p.ld + c0 * 16);
+            uint16_t *yp = p.y + row * p.ld + c0 * 16;
 #pragma unroll
             for (int j = 0; j < kUnroll; ++j) {
                 if (c0 + 32 * j >= sf_cols) continue;
                 uint4 o0, o1;
                 decode_block(c[j], dtab[sb[j] & 0x7Fu], o0, o1);
-                yp[64 * j] = o0;
-                yp[64 * j + 1] = o1;
+                store_32b(yp + 512 * j, o0, o1, p.y_vec32 != 0);
             }
         }
     } else {
@@ -541,9 +546,7 @@ __device__ __forceinline__ void dequantize_body(const DequantParams &p) {
                 const float d = __fdiv_rn(f32_from_e4m3(sb[u]), g);
                 uint4 o0, o1;
                 decode_block(c[u], d, o0, o1);
-                uint4 *yp = reinterpret_cast<uint4 *>(p.y + rr[u] * p.ld + bb[u] * 16);
-                yp[0] = o0;
-                yp[1] = o1;
+                store_32b(p.y + rr[u] * p.ld + bb[u] * 16, o0, o1, p.y_vec32 != 0);
             }
         }
     }

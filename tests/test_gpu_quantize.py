@@ -221,3 +221,43 @@ def test_quantize_gather_own_amax():
     gathered[real] = x[gather[real].long()]
     st, ref = oracle.quantize(gathered)
     assert_quantized_equal(q, ref, "gather own amax")
+
+
+def test_gather_rows_moe_parity():
+    """Quantize X once, then gather its NVFP4 rows into the expert slots:
+    bit for bit the oracle's quantization of the gathered rows with X's
+    tensor scale, and the same bytes as the gathered quantize."""
+    r = inputs.MoeRouting()
+    x = inputs.moe_activation()
+    xd = x.to(DEV)
+    gather = r.gather.to(DEV)
+    qx = nb.nvfp4_quantize(xd)
+    q = nb.nvfp4_gather_rows(qx, gather)
+    qg = nb.NVFP4Tensor.empty(r.padded_rows, x.shape[1], device=DEV, global_scale=nb.nvfp4_global_scale(xd))
+    nb.nvfp4_quantize_gather(xd, gather, out=qg, global_supplied=True)
+    assert nb.nvfp4_check_status() == 0
+    gathered = torch.zeros(r.padded_rows, x.shape[1], dtype=torch.bfloat16)
+    real = r.gather >= 0
+    gathered[real] = x[r.gather[real].long()]
+    st, amax = oracle.tensor_amax(x)
+    ref = oracle.quantize_with_global(gathered, oracle.global_scale(amax)[1])
+    assert_quantized_equal(q, ref, "gathered rows")
+    assert torch.equal(q.codes, qg.codes) and torch.equal(q.scales, qg.scales)
+
+
+@pytest.mark.parametrize("src_layout,dst_layout", [(nb.SF_SWIZZLED, nb.SF_SWIZZLED),
+                                                   (nb.SF_LINEAR, nb.SF_SWIZZLED),
+                                                   (nb.SF_SWIZZLED, nb.SF_LINEAR)])
+@pytest.mark.parametrize("cols", [16, 48, 1040])
+def test_gather_rows_layouts_ragged_and_bad_entries(src_layout, dst_layout, cols):
+    x = _rand(70, cols, cols + src_layout)
+    qs = nb.nvfp4_quantize(x.to(DEV), layout=src_layout)
+    gather = torch.tensor([69, -1, 0, 5, 5, 130, -1, 33] * 17, dtype=torch.int32)   # 130: out of range
+    q = nb.nvfp4_gather_rows(qs, gather.to(DEV), layout=dst_layout)
+    assert nb.nvfp4_check_status() == 1                                              # NVFP4_ERR_INVALID_ARG
+    rows = torch.zeros(len(gather), cols, dtype=torch.bfloat16)
+    ok = (gather >= 0) & (gather < 70)
+    rows[ok] = x[gather[ok].long()]
+    st, amax = oracle.tensor_amax(x)
+    ref = oracle.quantize_with_global(rows, oracle.global_scale(amax)[1], dst_layout)
+    assert_quantized_equal(q, ref, f"gather {src_layout}->{dst_layout}")
