@@ -69,8 +69,12 @@ struct PairShared {
 template <bool kCluster>
 __device__ __forceinline__ bool pwait(uint64_t *bar, uint32_t parity, PairShared *sh,
                                       const GemmParams &p) {
-    auto test = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
-    if (kCluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity)) return true;
+    // Barriers the other CTA arrives on are waited on like local ones: its
+    // arrives carry their own release, and the waits' default acquire pairs
+    // with them (the same pattern as for CTA-local barriers).
+    (void)kCluster;
+    auto test = [&]() { return mbar_try_wait(bar, parity); };
+    if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (test()) return true;

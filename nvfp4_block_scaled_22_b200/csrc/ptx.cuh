@@ -408,9 +408,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
-// Arrive (release, cluster scope) on an mbarrier given by its cluster address.
+// Arrive on an mbarrier given by its cluster address (possibly the peer
+// CTA's), with the default release semantics at CTA scope.  An explicit
+// .release.cluster makes every arrive a cluster-wide fence: measured on the
+// CTA-pair GEMM, those fences were the dominant stall (the scale writers'
+// and the epilogue's arrives on the leader's barriers).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];"
                  :: "r"(cluster_addr) : "memory");
 }
 
