@@ -444,7 +444,9 @@ def workload_line(name, args, device):
             return q, g
         wu, gu = stacked("up", I, H)
         wd, gd = stacked("down", H, I)
-        qxs = nb.NVFP4Tensor.empty(inputs.MOE_TOKENS, H, device=device)      # X, quantized once
+        # X, quantized once; linear scale rows make the gather's scale reads
+        # whole row pieces (the slots' copy is in the GEMM's 128x4 layout)
+        qxs = nb.NVFP4Tensor.empty(inputs.MOE_TOKENS, H, nb.SF_LINEAR, device)
         qx = nb.NVFP4Tensor.empty(r.padded_rows, H, device=device)
         hbuf = torch.empty((r.padded_rows, I), dtype=torch.bfloat16, device=device)
         qh = nb.NVFP4Tensor.empty(r.padded_rows, I, device=device)

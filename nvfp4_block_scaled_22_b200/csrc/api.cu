@@ -811,8 +811,10 @@ nvfp4_status nvfp4_gather_rows(const nvfp4_tensor *src, const int32_t *d_gather,
     }
     const int64_t rows_pad = out->sf_layout == NVFP4_SF_SWIZZLED_128x4 ? ceil_div(out->rows, 128) * 128
                                                                       : out->rows;
-    int grid = (int)std::min<int64_t>(ceil_div(std::max<int64_t>(rows_pad, 1), 8), 16LL * sms);
-    if (grid < 1) grid = 1;
+    // One 128-row band per grid column, kGatherSplit CTAs per band
+    // (grid-stride beyond 64 bands per SM).
+    const int64_t bands = std::max<int64_t>(ceil_div(rows_pad, 128), 1);
+    const dim3 grid((unsigned)std::min<int64_t>(bands, 64LL * sms), kGatherSplit, 1);
     k_gather_rows<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return launched(cudaGetLastError());
 }

@@ -77,6 +77,7 @@ struct GatherParams {
     const int32_t *map;      // output row -> source row, -1 = zero row
     uint32_t *status;
 };
+constexpr int kGatherSplit = 2;   // CTAs per 128-row output band (grid.y of k_gather_rows)
 __global__ void k_gather_rows(GatherParams p);
 
 __global__ void k_amax(const uint16_t *x, int64_t ld, int64_t rows, int64_t cols,

@@ -223,7 +223,8 @@ def test_quantize_gather_own_amax():
     assert_quantized_equal(q, ref, "gather own amax")
 
 
-def test_gather_rows_moe_parity():
+@pytest.mark.parametrize("src_layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
+def test_gather_rows_moe_parity(src_layout):
     """Quantize X once, then gather its NVFP4 rows into the expert slots:
     bit for bit the oracle's quantization of the gathered rows with X's
     tensor scale, and the same bytes as the gathered quantize."""
@@ -231,7 +232,7 @@ def test_gather_rows_moe_parity():
     x = inputs.moe_activation()
     xd = x.to(DEV)
     gather = r.gather.to(DEV)
-    qx = nb.nvfp4_quantize(xd)
+    qx = nb.nvfp4_quantize(xd, layout=src_layout)
     q = nb.nvfp4_gather_rows(qx, gather)
     qg = nb.NVFP4Tensor.empty(r.padded_rows, x.shape[1], device=DEV, global_scale=nb.nvfp4_global_scale(xd))
     nb.nvfp4_quantize_gather(xd, gather, out=qg, global_supplied=True)
@@ -247,8 +248,9 @@ def test_gather_rows_moe_parity():
 
 @pytest.mark.parametrize("src_layout,dst_layout", [(nb.SF_SWIZZLED, nb.SF_SWIZZLED),
                                                    (nb.SF_LINEAR, nb.SF_SWIZZLED),
-                                                   (nb.SF_SWIZZLED, nb.SF_LINEAR)])
-@pytest.mark.parametrize("cols", [16, 48, 1040])
+                                                   (nb.SF_SWIZZLED, nb.SF_LINEAR),
+                                                   (nb.SF_LINEAR, nb.SF_LINEAR)])
+@pytest.mark.parametrize("cols", [16, 48, 1040, 8448])
 def test_gather_rows_layouts_ragged_and_bad_entries(src_layout, dst_layout, cols):
     x = _rand(70, cols, cols + src_layout)
     qs = nb.nvfp4_quantize(x.to(DEV), layout=src_layout)
