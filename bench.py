@@ -43,23 +43,32 @@ ENCODE_BYTES_PER_VALUE = 2.5625
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
 ATTN_FP32_LANES = 148 * 128  # FP32 FMA lanes of a B200 (148 SMs x 128)
 SM_MAX_MHZ = 1965           # clocks.max.sm of the B200
-# DRAM bytes (read + write) of one k_gemm_nvf4 launch on this workload, from
-# an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum of one launch
-# at this shape.  Reported only while the kernel's sources hash to the
-# profiled version (otherwise null).
-GEMM_TRAFFIC_BYTES = 87.85e6 + 292.76e6
-GEMM_TRAFFIC_SRC_SHA = "6c187c6de44d0cf0"
-GEMM_SOURCES = ("gemm.cu", "gemm.h", "ptx.cuh")
+# DRAM bytes (read + write) of one GEMM launch on this workload, per kernel,
+# from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum of one
+# launch at this shape: (bytes, hash of the kernel's sources when captured).
+# Reported only while the sources still hash to the captured version
+# (otherwise null).
+GEMM_TRAFFIC = {
+    "single": (None, ""),
+    "pair": (None, ""),
+}
+GEMM_SOURCES = {"single": ("gemm.cu", "gemm.h", "ptx.cuh"),
+                "pair": ("gemm_pair.cu", "gemm.h", "ptx.cuh")}
 
 
-def gemm_traffic():
+def gemm_sources_sha(kernel):
     import hashlib
     csrc = os.path.join(ROOT, "nvfp4_block_scaled_22_b200", "csrc")
     h = hashlib.sha256()
-    for f in GEMM_SOURCES:
+    for f in GEMM_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
-    return GEMM_TRAFFIC_BYTES if h.hexdigest()[:16] == GEMM_TRAFFIC_SRC_SHA else None
+    return h.hexdigest()[:16]
+
+
+def gemm_traffic(kernel):
+    nbytes, sha = GEMM_TRAFFIC[kernel]
+    return nbytes if nbytes is not None and gemm_sources_sha(kernel) == sha else None
 
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -797,8 +806,9 @@ def main():
     ap.add_argument("--layers", type=int, default=32,
                     help="kv / attention workloads: layers of the KV cache (the workload has 32; "
                          "fewer give a case small enough for a multi-pass ncu capture)")
-    ap.add_argument("--gemm-kernel", default="single", choices=["single", "pair"],
-                    help="GEMM kernel for M >= 256: one SM per 128x256 tile or CTA pairs")
+    ap.add_argument("--gemm-kernel", default="pair", choices=["single", "pair"],
+                    help="GEMM kernel for M >= 256: CTA pairs on 256x256 tiles (the library "
+                         "default) or one SM per 128x256 tile")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -876,12 +886,13 @@ def main():
                        "weights": "pre-quantized once, outside the timed region",
                        "gemm_kernel": "cta_pair_256x256" if args.gemm_kernel == "pair"
                        else "single_cta_128x256"},
-            "roofline": {"kernel": "k_gemm_nvf4", "bound": "tensor",
+            "roofline": {"kernel": "k_gemm_nvf4_pair" if args.gemm_kernel == "pair" else "k_gemm_nvf4",
+                         "bound": "tensor",
                          "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak,
                          "peak_source": f"{peak_src} bf16 burst {bf16_tf} TFLOP/s x "
                                         f"{FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
-                         "traffic": gemm_traffic(), "ms_per_launch": gemm_avg,
+                         "traffic": gemm_traffic(args.gemm_kernel), "ms_per_launch": gemm_avg,
                          "algorithmic_flops_per_launch": flops},
             "quantize": {"workload": "quantize sweep, 2^28 BF16 values [65536 x 4096]",
                          "gbs_two_pass": gbs_2pass, "frac_two_pass": gbs_2pass / hbm_gbs,

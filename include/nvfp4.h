@@ -459,12 +459,12 @@ NVFP4_API int64_t nvfp4_launch_count(void);
  * Meant for tests of the timeout path. */
 NVFP4_API long long nvfp4_set_wait_limit_cycles(long long cycles);
 
-/* Kernel choice for dense nvfp4_gemm calls with M >= 256: enable = 1 runs
- * them on pairs of SMs sharing 256x256 output tiles (half the operand
- * traffic from L2 per SM), enable = 0 (the default, faster at the measured
- * shapes) on one SM per 128x256 tile.  Smaller M and the grouped GEMM always
- * use one SM per tile.  Both give results within the same bound.  Returns
- * the previous setting. */
+/* Kernel choice for dense NVFP4 nvfp4_gemm calls with M >= 256: enable = 1
+ * (the default; 3-8 % faster at the measured shapes) runs them on pairs of
+ * SMs sharing 256x256 output tiles (half the operand traffic from L2 per
+ * SM), enable = 0 on one SM per 128x256 tile.  Smaller M, MXFP4 operands and
+ * the grouped GEMM always use one SM per tile.  Both give results within the
+ * same bound.  Process-wide; returns the previous setting. */
 NVFP4_API int32_t nvfp4_set_gemm_pairs(int32_t enable);
 
 #ifdef __cplusplus

@@ -40,7 +40,7 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 long long g_timeout_cycles = kDefaultTimeoutCycles;
-bool g_use_pairs = false;
+bool g_use_pairs = true;
 
 nvfp4_status current_device(int *sms) {
     int dev = 0;

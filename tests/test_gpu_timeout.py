@@ -1,9 +1,10 @@
 """Bounded pipeline waits of the GEMM kernels, exercised on the GPU without a
 fault or a hang.
 
-Every mbarrier wait in the single-CTA GEMM pipeline gives up after a cycle
-limit.  Cutting that limit to a few hundred SM cycles (the library's test
-hook) makes the first wait on a real TMA copy run out: the launch must record
+Every mbarrier wait in the GEMM pipelines (single-CTA, CTA-pair, swapped
+operands, split-K) gives up after a cycle limit.  Cutting that limit to a
+few hundred SM cycles (the library's test hook) makes the first wait on a
+real TMA copy run out: the launch must record
 NVFP4_ERR_TIMEOUT in the status word, stop every role, let its issued copies
 and MMAs finish, release TMEM and exit.  Each wait still ends by itself
 (copies land, the limit passes), so nothing here can hang.  After the default
@@ -27,7 +28,7 @@ TINY_LIMIT = 300       # SM cycles: below any TMA round trip
 @pytest.fixture(autouse=True)
 def _single_cta_and_default_limit():
     nb.lib()
-    prev_pairs = nb.nvfp4_set_gemm_pairs(False)     # the CTA-pair kernel is not exercised here
+    prev_pairs = nb.nvfp4_set_gemm_pairs(False)     # the CTA-pair kernel only where a test enables it
     yield
     nb.nvfp4_set_wait_limit_cycles(0)                # back to the default bound
     nb.nvfp4_set_gemm_pairs(prev_pairs)
@@ -75,6 +76,19 @@ def test_dense_gemm_timeout_then_clean(m, n, k):
     qa, ra = _quant(_rand(m, k, m + k), "A")
     qw, rw = _quant(_rand(n, k, n + k + 1, 0.02), "W")
     ws = nb.Workspace(DEV, 256)                      # status word only: no split-K
+    _timed_out_then_clean(lambda: nb.nvfp4_gemm(qa, qw, workspace=ws), _full_check(ra, rw, m, n), ws)
+
+
+@pytest.mark.parametrize("m,n,k", [(256, 256, 256), (768, 1280, 1024)])
+def test_pair_gemm_timeout_then_clean(m, n, k):
+    """The CTA-pair kernel: a timed-out wait in either CTA stops that CTA's
+    roles; the other CTA's waits on the pair's barriers then time out in turn
+    (each is bounded), every issued copy and MMA drains before the final
+    cluster barrier, and TMEM is released by both CTAs."""
+    nb.nvfp4_set_gemm_pairs(True)
+    qa, ra = _quant(_rand(m, k, m + k + 7), "A")
+    qw, rw = _quant(_rand(n, k, n + k + 8, 0.02), "W")
+    ws = nb.Workspace(DEV, 256)
     _timed_out_then_clean(lambda: nb.nvfp4_gemm(qa, qw, workspace=ws), _full_check(ra, rw, m, n), ws)
 
 
