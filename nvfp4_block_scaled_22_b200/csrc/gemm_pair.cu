@@ -88,6 +88,17 @@ __device__ __forceinline__ bool pwait(uint64_t *bar, uint32_t parity, PairShared
 }
 
 
+// Pair tile order: M fastest, or N fastest when the CTAs running at one time
+// should share A's rows and sweep W (the same rule as the single-CTA kernel:
+// chosen when A's codes are too large to stay in L2 across a sweep).
+__device__ __forceinline__ void pair_tile(int tile, int mtiles, int ntiles, int n_fastest, int &mt,
+                                          int &nt) {
+    const int fast = n_fastest ? ntiles : mtiles;
+    const int q = tile / fast, r = tile - q * fast;
+    mt = n_fastest ? q : r;
+    nt = n_fastest ? r : q;
+}
+
 }  // namespace
 
 constexpr int kPairSmemBytes = kPStages * kPStageBytes + 1024 + 512;
@@ -155,7 +166,8 @@ k_gemm_nvf4_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int s = 0; s < kPStages; ++s) armed[s] = false;
             bool ok = true;
             for (int tile = cluster; ok && tile < tiles; tile += nclusters) {
-                const int mt = tile % mtiles, nt = tile / mtiles;
+                int mt, nt;
+                pair_tile(tile, mtiles, ntiles, p.n_fastest, mt, nt);
                 const int a_row0 = mt * kPBM + 128 * (int)rank;
                 const int b_pair0 = nt * kPBN;
                 const int b_row0 = b_pair0 + 128 * (int)rank;
@@ -307,7 +319,8 @@ k_gemm_nvf4_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int chalf = (warp - kFirstEpiWarp) / 4;
         uint32_t acc_phase = 0;
         for (int tile = cluster; tile < tiles; tile += nclusters) {
-            const int mt = tile % mtiles, nt = tile / mtiles;
+            int mt, nt;
+            pair_tile(tile, mtiles, ntiles, p.n_fastest, mt, nt);
             if (!pwait<false>(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
             const float alpha = __frcp_rn(__fmul_rn(*p.ga, *p.gw));

@@ -51,3 +51,19 @@ def attention_chunking(tokens: int, heads_kv: int):
     want = max(1, min(subs, 148 // heads_kv))
     chunk = -(-subs // want) * 256
     return chunk, (-(-tokens // chunk) if tokens > 0 else 0)
+
+
+def tile_samples(m, n, rng, tm=128, tn=256):
+    """Outputs that touch every tm x tn output tile: per tile one random
+    interior output, its last row at a random column, its last column at a
+    random row, and its last (row, column) corner.  Any fault tied to a
+    tile index, a CTA's wave or a ragged edge lands on at least one."""
+    mt, nt = -(-m // tm), -(-n // tn)
+    ti, tj = np.meshgrid(np.arange(mt), np.arange(nt), indexing="ij")
+    ti, tj = ti.ravel(), tj.ravel()
+    r0, c0 = ti * tm, tj * tn
+    rl = np.minimum(r0 + tm, m) - 1                   # last row / column of the tile
+    cl = np.minimum(c0 + tn, n) - 1
+    ri = r0 + (rng.random(ti.size) * (rl - r0 + 1)).astype(np.int64)
+    ci = c0 + (rng.random(tj.size) * (cl - c0 + 1)).astype(np.int64)
+    return np.concatenate([ri, rl, ri, rl]), np.concatenate([ci, ci, cl, cl])

@@ -12,7 +12,7 @@ import torch
 import oracle
 from nvfp4_block_scaled_22_b200 import binding as nb
 from nvfp4_block_scaled_22_b200 import inputs
-from tests.gpu_util import assert_quantized_equal, bf16_to_f64, gemm_tolerance
+from tests.gpu_util import assert_quantized_equal, bf16_to_f64, gemm_tolerance, tile_samples
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -90,22 +90,6 @@ def test_output_pitch_and_untouched_padding():
     ref, ab = oracle.gemm_ref(ra, rw, ii.ravel(), jj.ravel())
     got = bf16_to_f64(out[:, :200]).ravel()
     assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab))
-
-
-def tile_samples(m, n, rng, tm=128, tn=256):
-    """Outputs that touch every tm x tn output tile: per tile one random
-    interior output, its last row at a random column, its last column at a
-    random row, and its last (row, column) corner.  Any fault tied to a
-    tile index, a CTA's wave or a ragged edge lands on at least one."""
-    mt, nt = -(-m // tm), -(-n // tn)
-    ti, tj = np.meshgrid(np.arange(mt), np.arange(nt), indexing="ij")
-    ti, tj = ti.ravel(), tj.ravel()
-    r0, c0 = ti * tm, tj * tn
-    rl = np.minimum(r0 + tm, m) - 1                   # last row / column of the tile
-    cl = np.minimum(c0 + tn, n) - 1
-    ri = r0 + (rng.random(ti.size) * (rl - r0 + 1)).astype(np.int64)
-    ci = c0 + (rng.random(tj.size) * (cl - c0 + 1)).astype(np.int64)
-    return np.concatenate([ri, rl, ri, rl]), np.concatenate([ci, ci, cl, cl])
 
 
 def _sampled(d, ra, rw, m, n, count, seed, gw=None, rows_map=None):

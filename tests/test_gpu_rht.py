@@ -14,7 +14,7 @@ import torch
 import oracle
 from nvfp4_block_scaled_22_b200 import binding as nb
 from nvfp4_block_scaled_22_b200 import inputs
-from tests.gpu_util import assert_quantized_equal, bf16_to_f64, gemm_tolerance
+from tests.gpu_util import assert_quantized_equal, bf16_to_f64, gemm_tolerance, tile_samples
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -93,7 +93,8 @@ def test_errors_and_supplied_scale():
 def test_wgrad_operands_full_size_and_gemm():
     """dW = dY^T X at M = 8192 tokens: both operands quantized after the
     transform with the same signs, full compare of codes and scales, then the
-    Wgrad GEMM (20480 x 5120, K = 8192) on sampled outputs."""
+    Wgrad GEMM (20480 x 5120, K = 8192, run in N-fastest tile order) on
+    sampled outputs that touch every output tile."""
     mask = inputs.rht_sign_mask(0)
     dy_t = inputs.wgrad_grad_output_t(device=DEV)
     x_t = inputs.wgrad_activation_t(device=DEV)
@@ -108,8 +109,9 @@ def test_wgrad_operands_full_size_and_gemm():
     assert st == oracle.OK
     assert_quantized_equal(qw, rw, "X^T")
     rng = np.random.default_rng(11)
-    ii = rng.integers(0, qa.rows, 600)
-    jj = rng.integers(0, qw.rows, 600)
+    ti, tj = tile_samples(qa.rows, qw.rows, rng)
+    ii = np.concatenate([rng.integers(0, qa.rows, 600), ti])
+    jj = np.concatenate([rng.integers(0, qw.rows, 600), tj])
     ref, ab = oracle.gemm_ref(ra, rw, ii, jj)
     got = bf16_to_f64(d)[ii, jj]
     assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab))
