@@ -49,8 +49,8 @@ SM_MAX_MHZ = 1965           # clocks.max.sm of the B200
 # Reported only while the sources still hash to the captured version
 # (otherwise null).
 GEMM_TRAFFIC = {
-    "single": (84.61e6 + 290.51e6, "75e9dd8a492872ae"),
-    "pair": (88.89e6 + 292.53e6, "b65722eb9a737775"),
+    "single": (87.46e6 + 291.25e6, "8a5a0e68c5a1fd2d"),
+    "pair": (88.97e6 + 292.48e6, "4c6002330205c7ae"),
 }
 GEMM_SOURCES = {"single": ("gemm.cu", "gemm.h", "ptx.cuh"),
                 "pair": ("gemm_pair.cu", "gemm.h", "ptx.cuh")}
