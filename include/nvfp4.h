@@ -436,6 +436,27 @@ NVFP4_API nvfp4_status nvfp4_grouped_gemm(int32_t groups, const int32_t *d_slot_
                                 void *D, int64_t ldd, void *workspace, size_t workspace_bytes,
                                 void *stream);
 
+/* nvfp4_grouped_gemm that also writes, to *d_out_global, the NVFP4 tensor
+ * scale g = RN(2688 / amax) of its BF16 output, amax = max |D| over the real
+ * rows and the n columns (the padding rows are not part of the tensor; g = 1
+ * when every value is zero).  That is the g nvfp4_quantize_gather computes
+ * in its own amax pass over the same rows, so the next projection's
+ * quantize can take it as supplied (global_supplied = 1) and skip that pass
+ * ("NVIDIA shrank GLM-5.2 to 4 bits", §1: the expert linears' activations
+ * are NVFP4; "NVFP4: how NVIDIA pre-trained a 12B model on 10T tokens",
+ * "E2M1 format and two-level scaling": the FP32 tensor scale from the
+ * tensor's amax).  The maximum is taken in the GEMM's epilogue over the
+ * rounded BF16 values it stores.  Arguments and errors as
+ * nvfp4_grouped_gemm; d_out_global: device float, 4-byte aligned.
+ * Non-finite output records NVFP4_ERR_NONFINITE, an amax too small for a
+ * finite g NVFP4_ERR_RANGE (as nvfp4_quantize).  Uses bytes 8..11 of the
+ * workspace's status block. */
+NVFP4_API nvfp4_status nvfp4_grouped_gemm_out_scale(int32_t groups, const int32_t *d_slot_offsets,
+                                                    const int32_t *d_group_rows, const nvfp4_tensor *A,
+                                                    const nvfp4_tensor *W, const float *d_w_globals,
+                                                    int64_t n, void *D, int64_t ldd, float *d_out_global,
+                                                    void *workspace, size_t workspace_bytes, void *stream);
+
 /* ---- status ----------------------------------------------------------- */
 
 /* Synchronise `stream`, return the workspace's status word and reset it to

@@ -34,7 +34,8 @@ STATUS_NAMES = {
 EXPORTED = (
     "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_workspace_bytes", "nvfp4_quantize",
     "nvfp4_global_scale", "nvfp4_quantize_gather", "nvfp4_dequantize", "nvfp4_gemm",
-    "nvfp4_grouped_gemm", "nvfp4_check_status", "nvfp4_status_string", "nvfp4_version",
+    "nvfp4_grouped_gemm", "nvfp4_grouped_gemm_out_scale", "nvfp4_check_status",
+    "nvfp4_status_string", "nvfp4_version",
     "nvfp4_launch_count", "nvfp4_set_wait_limit_cycles", "nvfp4_set_gemm_pairs",
     "nvfp4_quantize_noalloc", "nvfp4_quantize_rht", "nvfp4_quantize_t", "nvfp4_quantize_2d",
     "nvfp4_quantize_sr", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx", "nvfp4_dequantize_mx",
@@ -78,6 +79,8 @@ def lib() -> C.CDLL:
             "nvfp4_dequantize": (C.c_int, [T, vp, i64, vp]),
             "nvfp4_gemm": (C.c_int, [T, T, vp, i64, vp, sz, vp]),
             "nvfp4_grouped_gemm": (C.c_int, [i32, vp, vp, T, T, vp, i64, vp, i64, vp, sz, vp]),
+            "nvfp4_grouped_gemm_out_scale": (C.c_int, [i32, vp, vp, T, T, vp, i64, vp, i64, vp, vp,
+                                                       sz, vp]),
             "nvfp4_check_status": (C.c_int, [vp, vp]),
             "nvfp4_status_string": (C.c_char_p, [C.c_int]),
             "nvfp4_version": (i32, []),
@@ -489,6 +492,29 @@ def nvfp4_grouped_gemm(slot_offsets: torch.Tensor, group_rows: torch.Tensor, a: 
                                     out.data_ptr(), out.stride(0), ws.ptr, ws.nbytes,
                                     _stream(stream)), "nvfp4_grouped_gemm")
     return out
+
+
+def nvfp4_grouped_gemm_out_scale(slot_offsets: torch.Tensor, group_rows: torch.Tensor,
+                                 a: NVFP4Tensor, w: NVFP4Tensor, w_globals: torch.Tensor, n: int,
+                                 out: torch.Tensor | None = None,
+                                 out_global: torch.Tensor | None = None,
+                                 workspace: Workspace | None = None, stream=None):
+    """nvfp4_grouped_gemm that also writes the NVFP4 tensor scale of its BF16
+    output over the real rows into out_global (float32 CUDA, one element).
+    Returns (out, out_global)."""
+    groups = group_rows.numel()
+    if out is None:
+        out = torch.empty((a.rows, n), dtype=torch.bfloat16, device=a.codes.device)
+    if out_global is None:
+        out_global = torch.empty(1, dtype=torch.float32, device=a.codes.device)
+    ws = workspace or default_workspace(a.codes.device)
+    ca, cw = a.c_struct(), w.c_struct()
+    _check(lib().nvfp4_grouped_gemm_out_scale(groups, slot_offsets.data_ptr(), group_rows.data_ptr(),
+                                              C.byref(ca), C.byref(cw), w_globals.data_ptr(), n,
+                                              out.data_ptr(), out.stride(0), out_global.data_ptr(),
+                                              ws.ptr, ws.nbytes, _stream(stream)),
+           "nvfp4_grouped_gemm_out_scale")
+    return out, out_global
 
 
 def nvfp4_check_status(workspace: Workspace | None = None, stream=None) -> int:

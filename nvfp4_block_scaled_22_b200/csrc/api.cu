@@ -21,6 +21,7 @@ std::atomic<int64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kStatusBytes = 256;          // status word + reserved
+constexpr size_t kOutAmaxOffset = 8;          // in the status block: nvfp4_grouped_gemm_out_scale's max
 constexpr int kMaxPartials = 1024;            // CTAs of the amax pass
 constexpr long long kDefaultTimeoutCycles = 2000000000ll;   // ~1 s at 1.9 GHz
 constexpr int64_t kFlatCols = 2048;           // row width for contiguous row-major-scale tensors
@@ -917,6 +918,7 @@ static nvfp4_status gemm_swap(const nvfp4_tensor *A, const nvfp4_tensor *W, int6
     p.timeout_cycles = g_timeout_cycles;
     p.splits = 1;
     p.partial = nullptr;
+    p.out_amax = nullptr;
     const int64_t ntiles = ceil_div(n, 128);
     const int ktiles = (int)ceil_div(k / 64, 4);
     int64_t best_cost = ceil_div(ntiles, sms) * ktiles;
@@ -945,7 +947,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
                                 const int32_t *d_group_rows, const nvfp4_tensor *A,
                                 const nvfp4_tensor *W, const float *gw, int64_t n, void *D,
                                 int64_t ldd, void *workspace, size_t workspace_bytes,
-                                void *stream, bool mx = false) {
+                                void *stream, bool mx = false, uint32_t *out_amax = nullptr) {
     nvfp4_status st = mx ? check_mx_tensor(A) : check_tensor(A);
     if (st != NVFP4_OK) return st;
     st = mx ? check_mx_tensor(W) : check_tensor(W);
@@ -1009,6 +1011,7 @@ static nvfp4_status gemm_common(int32_t groups, const int32_t *d_slot_offsets,
     p.timeout_cycles = g_timeout_cycles;
     p.splits = 1;
     p.partial = nullptr;
+    p.out_amax = out_amax;
     // Split-K for dense GEMMs with fewer output tiles than SMs (small M):
     // pick the split count that minimises the stage count of the busiest SM
     // (ties: fewer splits), if the FP32 slices fit in the workspace.
@@ -1067,6 +1070,26 @@ nvfp4_status nvfp4_grouped_gemm(int32_t groups, const int32_t *d_slot_offsets,
     if (groups <= 0) return NVFP4_ERR_INVALID_ARG;
     return gemm_common(groups, d_slot_offsets, d_group_rows, A, W, d_w_globals, n, D, ldd,
                        workspace, workspace_bytes, stream);
+}
+
+nvfp4_status nvfp4_grouped_gemm_out_scale(int32_t groups, const int32_t *d_slot_offsets,
+                                          const int32_t *d_group_rows, const nvfp4_tensor *A,
+                                          const nvfp4_tensor *W, const float *d_w_globals,
+                                          int64_t n, void *D, int64_t ldd, float *d_out_global,
+                                          void *workspace, size_t workspace_bytes, void *stream) {
+    if (groups <= 0 || d_out_global == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_out_global) & 3u) != 0) return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(workspace);
+    uint32_t *amax = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kOutAmaxOffset);
+    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    st = gemm_common(groups, d_slot_offsets, d_group_rows, A, W, d_w_globals, n, D, ldd, workspace,
+                     workspace_bytes, stream, false, amax);
+    if (st != NVFP4_OK) return st;
+    k_finalize_g<<<1, 256, 0, s>>>(amax, 1, d_out_global, status);
+    return launched(cudaGetLastError());
 }
 
 nvfp4_status nvfp4_check_status(void *workspace, void *stream) {

@@ -481,6 +481,16 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             const float alpha =
                 kMx ? 1.0f
                     : __frcp_rn(__fmul_rn(*p.ga, p.gw[tile_info(tile, mtiles, ntiles, p, s_off, s_rows).group]));
+            // Output max wanted (grouped NVFP4, see out_amax): the number of
+            // this lane's columns that count (its row must be a real row);
+            // -1 when not wanted.
+            int amax_lim = -1;
+            uint32_t amax_m = 0;
+            if (!kMx && !kSplit && p.out_amax != nullptr) {
+                const TileInfo ta = tile_info(tile, mtiles, ntiles, p, s_off, s_rows);
+                const int ca = ta.nt * kBN + chalf * 128;
+                amax_lim = ta.a_row0 + quarter * 32 + lane < ta.row_end ? max(0, min(128, p.n - ca)) : 0;
+            }
             if (!wait_or_abort(&sh->acc_full, acc_phase, sh, p)) break;
             tc_fence_after();
             // Four 32-column loads per warp: each wait is a TMEM round trip
@@ -493,9 +503,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
                                        (uint32_t)(chalf * 128 + 32 * c), r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
+                for (int i = 0; i < 16; ++i) {
                     o[16 * c + i] = bf16x2_from_f32(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
                                                     __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                    // BF16 magnitudes order as their bit patterns (Inf, NaN above all finite)
+                    if (2 * (16 * c + i) < amax_lim) amax_m = max_u16x2(amax_m, o[16 * c + i] & 0x7FFF7FFFu);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -507,6 +520,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmA, const CUtensor
             // makes every store instruction cover one row's 128 bytes.
             const int row0 = t.a_row0 + quarter * 32;
             const int col0 = t.nt * kBN + chalf * 128;
+            if (amax_lim >= 0) {
+                const uint32_t lo = amax_m & 0xFFFFu, hi = amax_m >> 16;
+                const uint32_t v = __reduce_max_sync(0xFFFFFFFFu, (lo > hi ? lo : hi) << 16);
+                if (lane == 0 && v != 0u) atomicMax(p.out_amax, v);
+            }
             if (row0 < t.row_end && col0 < p.n)
                 store_rows_coalesced(o, p.d + (int64_t)row0 * p.ldd + col0, p.ldd,
                                      t.row_end - row0, min(128, p.n - col0), p.d_vec16 != 0, lane);

@@ -80,6 +80,9 @@ struct GemmParams {
     int32_t n_fastest;        // tile order: 0 = M fastest, 1 = N fastest
     int32_t splits;           // K splits (1 = none); > 1: FP32 slices to `partial`
     float *partial;           // splits x m x n FP32 partial sums (split-K only)
+    // when set (grouped NVFP4, unsplit): max |D| over the real rows, as f32
+    // bits, atomically maxed into this word (zeroed before the launch)
+    uint32_t *out_amax;
     uint32_t *status;
     long long timeout_cycles;
 };

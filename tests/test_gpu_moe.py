@@ -174,3 +174,61 @@ def test_down_projection_full_size(routing):
         ref, ab = oracle.gemm_ref(rq, ref_w, ii, jj)
         got = _at(y, ii, cols[jj])
         assert np.all(np.abs(got - ref) <= gemm_tolerance(ref, ab)), f"expert {e}"
+
+
+def _ident(routing):
+    return torch.where(routing.gather >= 0, torch.arange(routing.padded_rows, dtype=torch.int32),
+                       torch.full_like(routing.gather, -1)).to(DEV)
+
+
+@pytest.mark.parametrize("n", [256, 384])
+def test_out_scale_small_groups(n):
+    """The grouped GEMM's tensor scale of its output (max over real rows and
+    the n columns, from the epilogue) equals the one the intermediate's
+    quantize computes in its own amax pass over the same rows, bit for bit;
+    the output itself is unchanged.  n = 384: a 256-column tile reaches into
+    the next group's weights, which must not count."""
+    rows, k = [5, 130, 0, 128], 512
+    offs = np.concatenate([[0], np.cumsum([-(-r // 128) * 128 for r in rows])]).astype(np.int32)
+    gen = torch.Generator().manual_seed(77 + n)
+    a = torch.zeros(int(offs[-1]), k, dtype=torch.bfloat16)
+    for g, r in enumerate(rows):
+        a[offs[g]:offs[g] + r] = torch.randn(r, k, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(len(rows) * n, k, generator=gen) * 0.02).to(torch.bfloat16)
+    w[2 * n:3 * n] *= 50.0                 # the group with no rows has the largest weights
+    qa, qw = nb.nvfp4_quantize(a.to(DEV)), nb.nvfp4_quantize(w.to(DEV))
+    gws = qw.global_scale.repeat(len(rows))
+    off_d, rows_d = torch.from_numpy(offs).to(DEV), torch.tensor(rows, dtype=torch.int32, device=DEV)
+    d0 = torch.zeros((a.shape[0], n), dtype=torch.bfloat16, device=DEV)
+    d1 = torch.zeros_like(d0)
+    nb.nvfp4_grouped_gemm(off_d, rows_d, qa, qw, gws, n, out=d0)
+    _, g1 = nb.nvfp4_grouped_gemm_out_scale(off_d, rows_d, qa, qw, gws, n, out=d1)
+    assert nb.nvfp4_check_status() == 0
+    assert torch.equal(d0, d1)
+    real = torch.zeros(a.shape[0], dtype=torch.bool)
+    for g, r in enumerate(rows):
+        real[offs[g]:offs[g] + r] = True
+    ident = torch.where(real, torch.arange(a.shape[0], dtype=torch.int32),
+                        torch.full((a.shape[0],), -1, dtype=torch.int32)).to(DEV)
+    q_own = nb.nvfp4_quantize_gather(d1, ident)
+    assert nb.nvfp4_check_status() == 0
+    assert g1.item() == q_own.global_scale.item()
+
+
+def test_out_scale_full_size(routing):
+    """At the MoE shape: the up projection's output tensor scale equals the
+    intermediate quantize's own, and quantizing with it supplied gives the
+    same bytes."""
+    x = inputs.moe_activation(device=DEV)
+    qx = nb.nvfp4_quantize_gather(x, routing.gather.to(DEV))
+    wu, gu, _ = _stacked("up", I, H)
+    off_d, rows_d = routing.slot_offsets.to(DEV), routing.rows.to(DEV)
+    h, g1 = nb.nvfp4_grouped_gemm_out_scale(off_d, rows_d, qx, wu, gu, I)
+    assert nb.nvfp4_check_status() == 0
+    ident = _ident(routing)
+    q_own = nb.nvfp4_quantize_gather(h, ident)
+    q_sup = nb.NVFP4Tensor.empty(routing.padded_rows, I, device=DEV, global_scale=g1.clone())
+    nb.nvfp4_quantize_gather(h, ident, out=q_sup, global_supplied=True)
+    assert nb.nvfp4_check_status() == 0
+    assert g1.item() == q_own.global_scale.item()
+    assert torch.equal(q_sup.codes, q_own.codes) and torch.equal(q_sup.scales, q_own.scales)
