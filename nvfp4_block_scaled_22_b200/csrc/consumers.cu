@@ -115,31 +115,75 @@ __global__ void __launch_bounds__(256) k_moe_combine(CombineParams p) {
 
 // Lane per 16-value block: v = e2m1(code) * (s_b / 8) (exact), E4M3 by the
 // hardware RN-satfinite conversion, 16 bytes out; block 0 thread 0 writes
-// the per-tensor factor RN(8 / g).
+// the per-tensor factor RN(8 / g).  Two blocks per thread per step (their
+// loads issued together); a block's row and column come from a 32-bit
+// division, or none when the tensor is one flat run of blocks (row-major
+// scales, output pitch = columns: the KV cache).
+namespace {
+
+__device__ __forceinline__ uint4 fp8_block(uint2 codes, float sb8) {
+    const uint32_t cw[2] = {codes.x, codes.y};
+    uint32_t out[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 v = f32x2_from_f16x2(f16x2_from_e2m1x2((cw[h] >> (8 * j)) & 0xFFu));
+            b[j] = e4m3x2_from_f32(__fmul_rn(v.x, sb8), __fmul_rn(v.y, sb8));   // 16 bits
+        }
+        out[2 * h] = b[0] | (b[1] << 16);
+        out[2 * h + 1] = b[2] | (b[3] << 16);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+}  // namespace
+
 __global__ void __launch_bounds__(256) k_dequantize_fp8(Fp8Params p) {
     if (blockIdx.x == 0 && threadIdx.x == 0) *p.fp8_scale = __fdiv_rn(8.0f, *p.global);
     const int64_t sf_cols = p.cols / 16, col_tiles = (sf_cols + 3) / 4;
     const int64_t blocks = p.rows * sf_cols;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < blocks;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / sf_cols, c = i - r * sf_cols;
-        const uint2 codes = __ldg(reinterpret_cast<const uint2 *>(p.codes + r * (p.cols / 2) + c * 8));
-        const float sb8 = __fmul_rn(f32_from_e4m3(__ldg(p.scales + sf_offset(r, c, sf_cols, col_tiles, p.layout))),
-                                    0.125f);
-        const uint32_t cw[2] = {codes.x, codes.y};
-        uint32_t out[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t b[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 v = f32x2_from_f16x2(f16x2_from_e2m1x2((cw[h] >> (8 * j)) & 0xFFu));
-                b[j] = e4m3x2_from_f32(__fmul_rn(v.x, sb8), __fmul_rn(v.y, sb8));   // 16 bits
-            }
-            out[2 * h] = b[0] | (b[1] << 16);
-            out[2 * h + 1] = b[2] | (b[3] << 16);
+    const bool flat = p.layout == 1 && p.ld == p.cols;
+    const bool small = blocks <= 0x7FFFFFFFll;
+    auto locate = [&](int64_t i, int64_t &code_off, int64_t &sf_off, int64_t &y_off) {
+        if (flat) {
+            code_off = i * 8;
+            sf_off = i;
+            y_off = i * 16;
+            return;
         }
-        *reinterpret_cast<uint4 *>(p.y + r * p.ld + c * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+        int64_t r, c;
+        if (small) {
+            const uint32_t q = (uint32_t)i / (uint32_t)sf_cols;
+            r = q;
+            c = (uint32_t)i - q * (uint32_t)sf_cols;
+        } else {
+            r = i / sf_cols;
+            c = i - r * sf_cols;
+        }
+        code_off = r * (p.cols / 2) + c * 8;
+        sf_off = sf_offset(r, c, sf_cols, col_tiles, p.layout);
+        y_off = r * p.ld + c * 16;
+    };
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < blocks; i0 += 2 * stride) {
+        const int64_t i1 = i0 + stride;
+        int64_t co0, so0, yo0, co1 = 0, so1 = 0, yo1 = 0;
+        locate(i0, co0, so0, yo0);
+        const bool two = i1 < blocks;
+        if (two) locate(i1, co1, so1, yo1);
+        const uint2 c0 = __ldg(reinterpret_cast<const uint2 *>(p.codes + co0));
+        const uint32_t s0 = __ldg(p.scales + so0);
+        uint2 c1 = make_uint2(0u, 0u);
+        uint32_t s1 = 0u;
+        if (two) {
+            c1 = __ldg(reinterpret_cast<const uint2 *>(p.codes + co1));
+            s1 = __ldg(p.scales + so1);
+        }
+        *reinterpret_cast<uint4 *>(p.y + yo0) = fp8_block(c0, __fmul_rn(f32_from_e4m3(s0), 0.125f));
+        if (two)
+            *reinterpret_cast<uint4 *>(p.y + yo1) = fp8_block(c1, __fmul_rn(f32_from_e4m3(s1), 0.125f));
     }
 }
 
