@@ -88,3 +88,54 @@ def test_swiglu_quantize(rows, inter, layout):
     st, ref = oracle.quantize_swiglu(gu, layout)
     assert st == oracle.OK
     assert_quantized_equal(q, ref, f"swiglu {rows}x{inter}")
+
+
+def _swiglu_edge_tensor(case):
+    """Gate|up rows (256 x 2*160, BF16) for one screening edge case."""
+    rows, inter = 256, 160
+    g = torch.Generator().manual_seed(77)
+    gate = torch.randn(rows, inter, generator=g) * 3
+    up = torch.randn(rows, inter, generator=g) * 3
+    if case == "subnormal_gates":
+        # g * r below the normal range against ups that make h ~ 1e-10
+        sub = torch.randint(1, 128, (rows // 2, inter), generator=g).float() * 2.0 ** -133
+        gate[: rows // 2] = sub * torch.sign(gate[: rows // 2])
+        up[: rows // 2] = torch.sign(up[: rows // 2]) * torch.exp(
+            torch.rand(rows // 2, inter, generator=g) * 3 + 64)
+        gate[rows // 2:] *= 1e-5
+        up[rows // 2:] *= 1e-5
+    elif case == "tiny":
+        # every block max below 2^-90: all h from the defined formula
+        gate *= 1e-15
+        up *= 1e-15
+    elif case == "large":
+        gate *= 1e17
+        up *= 1e17
+    elif case == "clamp_zeros_ties":
+        gate[5] = torch.linspace(-120.0, -60.0, inter)     # exp clamp, deep negative gates
+        gate[6] = torch.linspace(60.0, 120.0, inter)
+        gate[7, ::2] = 0.0
+        gate[7, 1::2] = -0.0
+        up[8, ::3] = -0.0
+        gate[11, :16] = 2.0                                # sixteen values tie the block max
+        up[11, :16] = 1.5
+        gate[12, :16] = torch.tensor([2.0, 2.0078125] * 8)  # near-ties one BF16 step apart
+        up[12, :16] = 3.0
+        gate[13, :16] *= 1e-30                             # a tiny block in a normal row
+    return torch.cat([gate, up], dim=1).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("case", ["subnormal_gates", "tiny", "large", "clamp_zeros_ties"])
+@pytest.mark.parametrize("layout", [nb.SF_SWIZZLED, nb.SF_LINEAR])
+def test_swiglu_quantize_screening_edges(case, layout):
+    """Inputs that the kernel's cheap screening of h cannot decide alone:
+    subnormal gates (g * r not a normal number), blocks of tiny values (every
+    h from the defined formula), large finite h, gates at and beyond the exp
+    clamp, signed zeros and ties of the block maximum; codes, scales and g
+    must still equal the oracle's."""
+    gu = _swiglu_edge_tensor(case)
+    q = nb.nvfp4_quantize_swiglu(gu.to(DEV), layout=layout)
+    assert nb.nvfp4_check_status() == 0
+    st, ref = oracle.quantize_swiglu(gu, layout)
+    assert st == oracle.OK
+    assert_quantized_equal(q, ref, f"swiglu screening {case}")
