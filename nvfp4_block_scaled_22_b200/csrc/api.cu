@@ -709,8 +709,16 @@ nvfp4_status nvfp4_attention_decode(const void *q, int64_t ldq, int32_t heads_q,
         st = launched(cudaGetLastError());
         if (st != NVFP4_OK) return st;
     }
-    k_attn_combine<<<(unsigned)heads_q, kAttnDim, 0, s>>>(p);
-    return launched(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)heads_q, 1, 1);
+    cfg.blockDim = dim3(kAttnDim, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return launched(cudaLaunchKernelEx(&cfg, k_attn_combine, p));
 }
 
 nvfp4_status nvfp4_quantize_swiglu(const void *gate_up, int64_t ld, const nvfp4_tensor *out,

@@ -89,6 +89,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
     __shared__ float wred[kAttnThreads / 32][kAttnMaxGroup];
     __shared__ float m_sh[kAttnMaxGroup], alpha_sh[kAttnMaxGroup];
 
+    // the combine (launched with programmatic stream serialization) may be
+    // scheduled now; it waits on the device for this whole grid
+    grid_dependents_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;    // pass A: MMA fragment row group, column pair
     const int hk = blockIdx.y, G = p.group;
@@ -311,19 +314,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
     }
 }
 
+// The chunks' values are loaded eight at a time before they are used, so
+// that a batch costs one memory round trip; the sums still run in chunk
+// order.  Launched behind k_attn_partial with programmatic stream
+// serialization: the wait below returns once that grid has completed.
 __global__ void __launch_bounds__(kAttnDim) k_attn_combine(AttnParams p) {
+    constexpr int kBatch = 8;
+    grid_dependency_wait();
     const int qh = blockIdx.x, d = threadIdx.x;
     const int64_t heads_q = (int64_t)p.group * p.heads_kv;
+    const int n = p.n_chunks;
     float r = 0.0f;
-    if (p.n_chunks > 0) {
+    if (n > 0) {
         float M = neg_inf();
-        for (int c = 0; c < p.n_chunks; ++c) M = fmaxf(M, p.part_ml[(c * heads_q + qh) * 2]);
+        for (int c0 = 0; c0 < n; c0 += kBatch) {
+            float m[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                m[j] = c0 + j < n ? p.part_ml[((c0 + j) * heads_q + qh) * 2] : neg_inf();
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) M = fmaxf(M, m[j]);
+        }
         float L = 0.0f, O = 0.0f;
-        for (int c = 0; c < p.n_chunks; ++c) {
-            const int64_t slot = c * heads_q + qh;
-            const float w = exp2f(p.part_ml[slot * 2] - M);
-            L = __fmaf_rn(w, p.part_ml[slot * 2 + 1], L);
-            O = __fmaf_rn(w, p.part_o[slot * kAttnDim + d], O);
+        for (int c0 = 0; c0 < n; c0 += kBatch) {
+            float m[kBatch], l[kBatch], o[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int64_t slot = (c0 + j) * heads_q + qh;
+                const bool ok = c0 + j < n;
+                m[j] = ok ? p.part_ml[slot * 2] : 0.0f;
+                l[j] = ok ? p.part_ml[slot * 2 + 1] : 0.0f;
+                o[j] = ok ? p.part_o[slot * kAttnDim + d] : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                if (c0 + j < n) {
+                    const float w = exp2f(m[j] - M);
+                    L = __fmaf_rn(w, l[j], L);
+                    O = __fmaf_rn(w, o[j], O);
+                }
+            }
         }
         r = __fdiv_rn(__fdiv_rn(O, L), *p.gv);
     }
