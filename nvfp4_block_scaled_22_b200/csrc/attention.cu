@@ -23,12 +23,18 @@
 //      dims 32c .. 32c + 31); the query columns follow the same order.
 //      Scores times c, the CTA maximum per head -> new running maximum and
 //      rescale factor; weights -> shared memory.
-//   B  thread = (8 dims, token phase 0..15): the V values of its dims for
-//      every 16th token of the sub-tile times the weights of all 8 heads,
-//      into 64 FP32 accumulators (rescaled first, packed FP32 FMAs).
-// After the chunk the token phases are summed in a fixed order (a shuffle,
-// then three halvings through shared memory) and the chunk's O, m and l
-// are written.  k_attn_combine merges the chunks in chunk order:
+//   B  O^T[dim][head] += V^T[dim][token] P^T[token][head] on the tensor
+//      cores too (mma.sync m16n8k8, TF32 operands, FP32 accumulation), each
+//      warp over its own 32 tokens: the restored V values (6 significant
+//      bits) are exact TF32, and each FP32 weight is split exactly into
+//      three TF32 parts (p = p1 + p2 + p3, 11 + 11 + 2 bits), one MMA per
+//      part, so every product is exact as in the FP32 reading.  Lane
+//      (g, c) restores the 16 dims 16g .. 16g + 15 (one 8-byte piece and
+//      one scale of its token row) of tokens c and c + 4 of each 8-token
+//      k-step; M-tile j row r is dim 16(r mod 8) + 2j + r / 8.
+// After the chunk the warps' accumulators are summed in a fixed order
+// (three halvings through shared memory) and the chunk's O, m and l are
+// written.  k_attn_combine merges the chunks in chunk order:
 //   o = (sum_c 2^(m_c - M) O_c) / (sum_c 2^(m_c - M) l_c) / g_V.
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -41,20 +47,8 @@ namespace nvfp4 {
 namespace {
 
 constexpr float kLog2e = 1.44269504088896340736f;
-constexpr int kPhases = kAttnThreads / 16;     // token phases of pass B
 
 __device__ __forceinline__ float neg_inf() { return __uint_as_float(0xFF800000u); }
-
-// d = a * b + c lane-wise, one rounding per lane (one instruction).
-__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\t"
-        "mov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
 
 // The two values of one code byte (low nibble first) times the block scale
 // s2 = (s, s): exact, e2m1 has 2 significant bits and E4M3 has 4.
@@ -67,6 +61,30 @@ __device__ __forceinline__ float2 restore_pair(uint32_t byte, float2 s2) {
 __device__ __forceinline__ uint32_t restore_bf16x2(uint32_t byte, float s) {
     const float2 v = f32x2_from_f16x2(f16x2_from_e2m1x2(byte & 0xFFu));
     return bf16x2_from_f32(__fmul_rn(v.x, s), __fmul_rn(v.y, s));
+}
+
+// D += A B for one 16x8x8 tile: A 16x8 row-major, B 8x8 column-major, TF32
+// operands (FP32 bit patterns whose low 13 bits are zero), FP32
+// accumulators (fragments of the PTX mma.sync m16n8k8 shape).
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// p = w[0] + w[1] + w[2] exactly, each part a TF32 value (FP32 with the low
+// 13 mantissa bits zero): truncation leaves remainders that FP32 holds
+// exactly (13, then 2 significant bits).
+__device__ __forceinline__ void split_tf32x3(float p, uint32_t (&w)[3]) {
+    const float p1 = __uint_as_float(__float_as_uint(p) & 0xFFFFE000u);
+    const float r1 = __fsub_rn(p, p1);
+    const float p2 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+    w[0] = __float_as_uint(p1);
+    w[1] = __float_as_uint(p2);
+    w[2] = __float_as_uint(__fsub_rn(r1, p2));
 }
 
 // D += A B for one 16x8x16 tile: A 16x16 row-major, B 16x8 column-major,
@@ -84,8 +102,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 }  // namespace
 
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) {
-    // ps[t][hp] = (p[2hp], p[2hp], p[2hp+1], p[2hp+1]) of token t of the sub-tile
-    __shared__ float4 ps[kAttnSub][kAttnMaxGroup / 2];
+    // weights p[head][token of the sub-tile] (rows padded: the B-fragment
+    // reads of a warp hit 32 banks); reused for the warps' final sums
+    constexpr int kPwPitch = kAttnSub + 4;
+    __shared__ __align__(16) float sbuf[4 * 32 * 32];
+    static_assert(kAttnMaxGroup * kPwPitch <= 4 * 32 * 32, "weights fit the reduction buffer");
+    float(*pw)[kPwPitch] = reinterpret_cast<float(*)[kPwPitch]>(sbuf);
     __shared__ float wred[kAttnThreads / 32][kAttnMaxGroup];
     __shared__ float m_sh[kAttnMaxGroup], alpha_sh[kAttnMaxGroup];
 
@@ -115,12 +137,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
     __syncthreads();
 
     float lsum[2] = {0.0f, 0.0f};             // heads 2c, 2c + 1 over this lane's tokens
-    float2 oacc[kAttnMaxGroup][4];
+    // pass B accumulators: M-tile j, (dim 16g + 2j, head 2c), (.., 2c + 1),
+    // (dim 16g + 2j + 1, head 2c), (.., 2c + 1)
+    float oacc[8][4];
 #pragma unroll
-    for (int h = 0; h < kAttnMaxGroup; ++h)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) oacc[h][i] = make_float2(0.0f, 0.0f);
-    const int dg = tid & 15, tp = tid >> 4;   // pass B: dims 8dg .. 8dg + 7, token phase
+        for (int i = 0; i < 4; ++i) oacc[j][i] = 0.0f;
 
     // Pass A rows of this lane: tokens 32 warp + 16 u + g + 8 r of the
     // sub-tile (u = MMA tile 0/1, r = fragment row half), code bytes
@@ -144,16 +167,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
 
     for (int64_t base = t0; base < t1; base += kAttnSub) {
         const int64_t n_sub = min((int64_t)kAttnSub, t1 - base);
-        uint32_t vw[kAttnSub / kPhases], vsb[kAttnSub / kPhases];
+        // pass B operands of this lane: tokens 32 warp + 8 kk + c (+ 4) of
+        // the sub-tile, dims 16g .. 16g + 15 (code bytes 8g .. 8g + 7 of the
+        // KV head's 64, scale block g)
+        uint2 vw[8];
+        uint32_t vsb[8];
 #pragma unroll
-        for (int s = 0; s < kAttnSub / kPhases; ++s) {
-            const int tl = tp + kPhases * s;
-            vw[s] = 0u;
-            vsb[s] = 0u;
+        for (int e = 0; e < 8; ++e) {
+            const int tl = 32 * warp + 8 * (e >> 1) + c + 4 * (e & 1);
+            vw[e] = make_uint2(0u, 0u);
+            vsb[e] = 0u;
             if (tl < n_sub) {   // tokens past the end keep code 0 and scale 0, weight 0
                 const int64_t tv = base + tl;
-                vw[s] = __ldg(reinterpret_cast<const uint32_t *>(p.vc + tv * row_codes + hk * 64 + dg * 4));
-                vsb[s] = __ldg(p.vs + tv * row_scales + hk * 8 + (dg >> 1));
+                vw[e] = __ldg(reinterpret_cast<const uint2 *>(p.vc + tv * row_codes + hk * 64 + 8 * g));
+                vsb[e] = __ldg(p.vs + tv * row_scales + hk * 8 + g);
             }
         }
 
@@ -216,39 +243,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
                     const float p1 = ok ? exp2f(sc[u][2 * r + 1] - m1) : 0.0f;
                     l0 += p0;
                     l1 += p1;
-                    ps[tl][c] = make_float4(p0, p0, p1, p1);
+                    pw[2 * c][tl] = p0;
+                    pw[2 * c + 1][tl] = p1;
                 }
             lsum[0] = __fmaf_rn(lsum[0], alpha_sh[2 * c], l0);
             lsum[1] = __fmaf_rn(lsum[1], alpha_sh[2 * c + 1], l1);
         }
         __syncthreads();
 
-        // ---- B: weighted V of tokens tp, tp + 16, ... of the sub-tile
+        // ---- B: O^T += V^T P^T over this warp's 32 tokens (exact products)
+        {
+            const float a0 = alpha_sh[2 * c], a1 = alpha_sh[2 * c + 1];
 #pragma unroll
-        for (int h = 0; h < kAttnMaxGroup; ++h) {
-            const float a = alpha_sh[h];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) oacc[h][i] = mul_f32x2(oacc[h][i], make_float2(a, a));
-        }
-#pragma unroll
-        for (int s = 0; s < kAttnSub / kPhases; ++s) {
-            const int tl = tp + kPhases * s;
-            const float sv = f32_from_e4m3(vsb[s]);
-            const float2 sv2 = make_float2(sv, sv);
-            float2 v2[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v2[i] = restore_pair(vw[s] >> (8 * i), sv2);
-#pragma unroll
-            for (int hp = 0; hp < kAttnMaxGroup / 2; ++hp) {
-                const float4 pp = ps[tl][hp];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    oacc[2 * hp][i] = fma_f32x2(v2[i], make_float2(pp.x, pp.y), oacc[2 * hp][i]);
-                    oacc[2 * hp + 1][i] = fma_f32x2(v2[i], make_float2(pp.z, pp.w), oacc[2 * hp + 1][i]);
-                }
+            for (int j = 0; j < 8; ++j) {
+                oacc[j][0] = __fmul_rn(oacc[j][0], a0);
+                oacc[j][1] = __fmul_rn(oacc[j][1], a1);
+                oacc[j][2] = __fmul_rn(oacc[j][2], a0);
+                oacc[j][3] = __fmul_rn(oacc[j][3], a1);
             }
         }
-        __syncthreads();   // ps and alpha_sh are rewritten by the next sub-tile
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int ta = 32 * warp + 8 * kk + c;          // B rows c and c + 4
+            uint32_t wa[3], wb[3];
+            split_tf32x3(pw[g][ta], wa);
+            split_tf32x3(pw[g][ta + 4], wb);
+            const float sa = f32_from_e4m3(vsb[2 * kk]), sb = f32_from_e4m3(vsb[2 * kk + 1]);
+            const uint2 ca = vw[2 * kk], cb = vw[2 * kk + 1];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {                   // M-tile j: dims 16r + 2j (+1)
+                const uint32_t byte_a = (j < 4 ? ca.x : ca.y) >> (8 * (j & 3));
+                const uint32_t byte_b = (j < 4 ? cb.x : cb.y) >> (8 * (j & 3));
+                const float2 va = restore_pair(byte_a, make_float2(sa, sa));
+                const float2 vb = restore_pair(byte_b, make_float2(sb, sb));
+                const uint32_t a[4] = {__float_as_uint(va.x), __float_as_uint(va.y),
+                                       __float_as_uint(vb.x), __float_as_uint(vb.y)};
+#pragma unroll
+                for (int q = 0; q < 3; ++q) mma_tf32_1688(oacc[j], a, wa[q], wb[q]);
+            }
+        }
+        __syncthreads();   // pw and alpha_sh are rewritten by the next sub-tile
     }
 
     // ---- chunk totals: weight sums per head (lanes of one column pair c)
@@ -259,49 +293,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn_partial(AttnParams p) 
         for (int off = 4; off <= 16; off <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
         if (g == 0) wred[warp][2 * c + e] = v;
     }
-    // O: the two token phases of a warp, then warps 4..7 onto 0..3, 2..3
-    // onto 0..1, 1 onto 0, through the (now free) weight buffer.
-#pragma unroll
-    for (int h = 0; h < kAttnMaxGroup; ++h)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            oacc[h][i].x += __shfl_xor_sync(0xFFFFFFFFu, oacc[h][i].x, 16);
-            oacc[h][i].y += __shfl_xor_sync(0xFFFFFFFFu, oacc[h][i].y, 16);
-        }
-    float *red = reinterpret_cast<float *>(&ps[0][0]);   // [4 warps][64 values][16 lanes]
+    // O: warps 4..7 onto 0..3, 2..3 onto 0..1, 1 onto 0, through the (now
+    // free) weight buffer
 #pragma unroll
     for (int half = 4; half >= 1; half >>= 1) {
-        if (warp >= half && warp < 2 * half && lane < 16) {
-            float *dst = red + (warp - half) * 1024 + lane;
+        if (warp >= half && warp < 2 * half) {
+            float *dst = sbuf + (warp - half) * 1024 + lane;
 #pragma unroll
-            for (int h = 0; h < kAttnMaxGroup; ++h)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    dst[(h * 8 + 2 * i) * 16] = oacc[h][i].x;
-                    dst[(h * 8 + 2 * i + 1) * 16] = oacc[h][i].y;
-                }
+                for (int i = 0; i < 4; ++i) dst[(4 * j + i) * 32] = oacc[j][i];
         }
         __syncthreads();
-        if (warp < half && lane < 16) {
-            const float *src = red + warp * 1024 + lane;
+        if (warp < half) {
+            const float *src = sbuf + warp * 1024 + lane;
 #pragma unroll
-            for (int h = 0; h < kAttnMaxGroup; ++h)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    oacc[h][i].x += src[(h * 8 + 2 * i) * 16];
-                    oacc[h][i].y += src[(h * 8 + 2 * i + 1) * 16];
-                }
+                for (int i = 0; i < 4; ++i) oacc[j][i] = __fadd_rn(oacc[j][i], src[(4 * j + i) * 32]);
         }
         __syncthreads();
     }
     const int64_t slot0 = (int64_t)blockIdx.x * heads_q + (int64_t)hk * G;
-    if (warp == 0 && lane < 16) {
+    if (warp == 0) {
 #pragma unroll
-        for (int h = 0; h < kAttnMaxGroup; ++h) {
-            if (h < G) {
-                float4 *dst = reinterpret_cast<float4 *>(p.part_o + (slot0 + h) * kAttnDim + 8 * lane);
-                dst[0] = make_float4(oacc[h][0].x, oacc[h][0].y, oacc[h][1].x, oacc[h][1].y);
-                dst[1] = make_float4(oacc[h][2].x, oacc[h][2].y, oacc[h][3].x, oacc[h][3].y);
+        for (int e = 0; e < 2; ++e) {                        // heads 2c + e
+            if (2 * c + e < G) {
+                float *dst = p.part_o + (slot0 + 2 * c + e) * kAttnDim + 16 * g;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float2 *>(dst + 2 * j) = make_float2(oacc[j][e], oacc[j][2 + e]);
             }
         }
     }

@@ -14,8 +14,14 @@ Tolerance, derived from the kernel's FP32 arithmetic (u = 2^-24):
     (ln 2 * log2 e = 1);
   * a weighted mean with weights perturbed by eps moves by at most
     2 eps * sum_t p_t |v_t| / sum_t p_t (the oracle's abs_o); the FP32 sums
-    add n u * abs_o to numerator and denominator, n = tokens per thread
-    chain + rescales + reduction levels + chunks; two final divisions 2u.
+    add n u * abs_o to numerator and denominator, n = twice the tensor-core
+    steps of an accumulator chain (each step adds 8 exact products -- the
+    restored V values times the three exact TF32 parts of a weight -- to
+    the accumulator and is off by at most 2 ulp of the sum of its terms'
+    magnitudes, as for the scores; 4 k-steps x 3 weight parts = 12 steps per
+    256 tokens of a chunk) + rescales + reduction levels + chunks (the
+    weight sums run as plain FP32 additions, fewer per chain); two final
+    divisions 2u.
 The bound below is twice that, plus half a BF16 ulp for the output rounding.
 Where the FP64 result lies farther than the FP32 bound from a BF16 rounding
 midpoint, the BF16 output must equal its correct rounding exactly; that
@@ -47,7 +53,7 @@ def _lib():
 def _fp32_bound(abs_o, score_abs, tokens, heads_kv):
     chunk, n_chunks = attention_chunking(max(tokens, 1), heads_kv)
     eps = 72 * U * score_abs[:, None] + 8 * U
-    n = chunk / 16 + 2 * chunk / 256 + 8 + n_chunks + 8
+    n = 2 * 12 * chunk / 256 + 2 * chunk / 256 + 8 + n_chunks + 8
     return 2 * (2 * eps + 2 * n * U + 2 * U) * abs_o
 
 
