@@ -324,7 +324,10 @@ NVFP4_API nvfp4_status nvfp4_dequantize_fp8(const nvfp4_tensor *in, void *y, int
  * Arithmetic: scores q . (e2m1 * s_b) on the tensor cores (BF16 operands,
  *   both exact; FP32 accumulation) times RN(RN(scale * log2(e)) / g_K), so
  *   in log2 units; exp2 and an online softmax over token chunks merged in
- *   chunk order; the weighted V sum in FP32.  Deterministic for given sizes.
+ *   chunk order; the weighted V sum on the tensor cores as well, with exact
+ *   products (TF32 operands: the restored V values, and each FP32 weight
+ *   split exactly into three TF32 parts; FP32 accumulation).  Deterministic
+ *   for given sizes.
  *   Non-finite q or scale bytes give unspecified (NaN) outputs; no status
  *   is recorded. */
 NVFP4_API nvfp4_status nvfp4_attention_decode(const void *q, int64_t ldq, int32_t heads_q,
