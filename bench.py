@@ -41,8 +41,6 @@ L2_FLUSH_BYTES = 256 << 20
 QUANT_BYTES_PER_VALUE_2PASS = 4.5625
 ENCODE_BYTES_PER_VALUE = 2.5625
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor throughput on B200
-ATTN_FP32_LANES = 148 * 128  # FP32 FMA lanes of a B200 (148 SMs x 128)
-SM_MAX_MHZ = 1965           # clocks.max.sm of the B200
 # DRAM bytes (read + write) of one GEMM launch on this workload, per kernel,
 # from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum of one
 # launch at this shape: (bytes, hash of the kernel's sources when captured).
@@ -796,11 +794,11 @@ def workload_line(name, args, device):
         st = nb.nvfp4_check_status(ws)
         cache_bytes = len(layers) * 2 * T * H * 128 * 0.5625
         gbs = cache_bytes / ms / 1e6
-        # Scores run on the tensor cores; the weighted V sum (2 flops per
-        # MAC, heads_q x T x 128 MACs) on the FP32 pipes bounds the design.
-        fp32_flops_layer = 2.0 * heads_q * T * 128
-        alu_peak = ATTN_FP32_LANES * 2 * SM_MAX_MHZ * 1e6 / 1e12
-        achieved = fp32_flops_layer / one / 1e9
+        # Scores and the weighted V sum both run on the tensor cores (2 x 2
+        # flops per MAC, heads_q x T x 128 MACs each); the roofline is the
+        # layer's cache read (K and V codes and scales, once).
+        layer_bytes = T * H * 128 * 2 * 0.5625
+        achieved = layer_bytes / one / 1e6
         line.update({"metric": "NVFP4 KV-cache decode attention GB/s of cache read (32 layers x K,V, "
                                "128K tokens, 64 query / 8 KV heads)",
                      "value": gbs, "unit": "GB/s", "higher_is_better": True, "ms_per_step": ms,
@@ -809,13 +807,12 @@ def workload_line(name, args, device):
                                 "l2": "inputs (4.8 GB cache) larger than L2; one-layer timing flushed"},
                      "tokens_per_s": 1e3 / ms, "ms_per_layer": one, "status": st,
                      "hbm_frac": gbs / hbm_gbs,
-                     "roofline": {"kernel": "k_attn_partial + k_attn_combine (one layer)", "bound": "alu",
-                                  "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                                  "frac": achieved / alu_peak,
-                                  "algorithmic_flops_per_launch": fp32_flops_layer,
-                                  "tensor_flops_per_launch": 2.0 * heads_q * T * 128,
-                                  "peak_source": "148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz",
-                                  "hbm_frac_per_layer": T * H * 128 * 2 * 0.5625 / one / 1e6 / hbm_gbs}})
+                     "roofline": {"kernel": "k_attn_partial + k_attn_combine (one layer)", "bound": "hbm",
+                                  "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                                  "frac": achieved / hbm_gbs,
+                                  "algorithmic_bytes_per_launch": layer_bytes,
+                                  "tensor_flops_per_launch": 2 * 2.0 * heads_q * T * 128,
+                                  "peak_source": f"{peak_src} hbm_gbs"}})
         return line
     raise ValueError(name)
 
