@@ -76,8 +76,10 @@ __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)
 }
 
 // p = w[0] + w[1] + w[2] exactly, each part a TF32 value (FP32 with the low
-// 13 mantissa bits zero): truncation leaves remainders that FP32 holds
-// exactly (13, then 2 significant bits).
+// 13 mantissa bits zero), for p >= 2^-113: truncation leaves remainders that
+// FP32 holds exactly (13, then 2 significant bits).  Below that p - p1 can
+// be subnormal and the third part keeps low bits that the TF32 operand
+// drops: an absolute error under 2^-136 per weight.
 __device__ __forceinline__ void split_tf32x3(float p, uint32_t (&w)[3]) {
     const float p1 = __uint_as_float(__float_as_uint(p) & 0xFFFFE000u);
     const float r1 = __fsub_rn(p, p1);

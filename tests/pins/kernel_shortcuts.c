@@ -17,6 +17,15 @@
  *    integer compare of the draw with the cleared bits), against the
  *    oracle's definition (neighbouring grid values, fraction compared with
  *    u / 2^16 in double).
+ * 4. rint(y) of the gated activation's exponential, y = RN(x * RN(log2 e))
+ *    for |x| <= 87, by adding and subtracting 1.5 * 2^23 (the sum's unit in
+ *    the last place is 1), the integer read from the sum's low mantissa
+ *    bits, against rintf.
+ * 5. The attention read's split of an FP32 weight p into three TF32 parts
+ *    (FP32 values with the low 13 mantissa bits zero) by truncation:
+ *    p1 = trunc(p), p2 = trunc(p - p1), p3 = (p - p1) - p2, checked to sum
+ *    to p exactly with p3 a TF32 value, for p >= 2^-113 (below, p - p1 may
+ *    be a subnormal number whose low 13 bits survive in p3, under 2^-136).
  */
 #include <math.h>
 #include <stdint.h>
@@ -92,3 +101,40 @@ int64_t shortcut_sr(uint32_t lo, uint32_t hi, const uint32_t *draws, int n_draws
             }
     return bad;
 }
+
+/* Shortcut 4 over the binary32 patterns [lo, hi) of x (both signs, |x| <=
+ * 87 expected).  Returns mismatches. */
+int64_t shortcut_rint_shift(uint32_t lo, uint32_t hi, uint32_t stride)
+{
+    const float log2e = 0x1.715476p+0f, c = 0x1.8p23f;
+    int64_t bad = 0;
+    for (uint64_t p = lo; p < hi; p += stride)
+        for (uint32_t s = 0; s < 2; ++s) {
+            const float x = f32((uint32_t)p | (s << 31));
+            const float y = x * log2e;
+            const float shifted = y + c;
+            const float n = shifted - c;
+            const int ni = (int)bits(shifted) - 0x4B400000;
+            const float r = rintf(y);
+            if (n != r || (float)ni != r) ++bad;
+        }
+    return bad;
+}
+
+/* Shortcut 5 over the binary32 patterns [lo, hi) of p > 0.  Returns the
+ * patterns whose three parts do not sum to p exactly or whose third part
+ * is not a TF32 value. */
+int64_t shortcut_tf32_split(uint32_t lo, uint32_t hi, uint32_t stride)
+{
+    int64_t bad = 0;
+    for (uint64_t q = lo; q < hi; q += stride) {
+        const float p = f32((uint32_t)q);
+        const float p1 = f32(bits(p) & 0xFFFFE000u);
+        const float r1 = p - p1;
+        const float p2 = f32(bits(r1) & 0xFFFFE000u);
+        const float p3 = r1 - p2;
+        if ((double)p1 + (double)p2 + (double)p3 != (double)p || (bits(p3) & 0x1FFFu) != 0) ++bad;
+    }
+    return bad;
+}
+

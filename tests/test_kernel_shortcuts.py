@@ -14,6 +14,9 @@ def _lib():
     L.shortcut_div6_fma.argtypes = [C.c_uint32, C.c_uint32]
     L.shortcut_sr.restype = C.c_int64
     L.shortcut_sr.argtypes = [C.c_uint32, C.c_uint32, C.c_void_p, C.c_int, C.c_uint32]
+    for f in (L.shortcut_rint_shift, L.shortcut_tf32_split):
+        f.restype = C.c_int64
+        f.argtypes = [C.c_uint32, C.c_uint32, C.c_uint32]
     return L
 
 
@@ -49,3 +52,32 @@ def test_stochastic_rounding_on_the_bit_pattern():
         b = struct.unpack("<I", struct.pack("<f", v))[0]
         assert L.shortcut_sr(b - (1 << 14), b + (1 << 14), draws.ctypes.data, len(draws), 1) == 0
     assert L.shortcut_sr(0, 1 << 15, draws.ctypes.data, len(draws), 1) == 0   # zero and subnormals
+
+
+def _bits(x: float) -> int:
+    import struct
+    return struct.unpack("<I", struct.pack("<f", x))[0]
+
+
+def test_exp_rint_by_shift():
+    """The gated activation's exponential rounds y = RN(x * log2 e) to an
+    integer by adding and subtracting 1.5 * 2^23 and reads the integer from
+    the sum's bits: equal to rintf for every 5th binary32 x up to 87 (both
+    signs), every pattern around the values where y is a half-integer, and
+    the clamp ends."""
+    L = _lib()
+    assert L.shortcut_rint_shift(0, _bits(87.0) + 1, 5) == 0
+    for k in range(-125, 126):
+        b = _bits((k + 0.5) / 1.4426950408889634)
+        assert L.shortcut_rint_shift(max(b - 4096, 0), b + 4096, 1) == 0, k
+
+
+def test_attention_weight_split_into_three_tf32_parts():
+    """p = p1 + p2 + p3 exactly with each part a TF32 value, for every
+    binary32 p in [1, 2) and every 7th one from 2^-113 to 1: the three
+    tensor-core products of a weight with a restored value sum to the exact
+    product."""
+    L = _lib()
+    assert L.shortcut_tf32_split(_bits(1.0), _bits(2.0), 1) == 0
+    assert L.shortcut_tf32_split(_bits(2.0 ** -113), _bits(1.0) + 1, 7) == 0
+
